@@ -1,0 +1,168 @@
+"""Routing, permutation and the W4A8 expert layer (oracle; test
+infrastructure only).
+
+The pages fix the expert numerics (INT4 group-128 weights, FP8 per-token
+activations, INT4 converted to FP8 for the tensor-core product, GLM-5.3-W4A8
+model card, intro and "quantisation method") and the layer shape (256 routed
+experts per layer, three projections per expert: gate, up and down, "From
+755GB to 395GB" blog, "what was quantised" and "the hard part is the memory
+limit").  They do not print the gating function, the activation function or
+the combine.  Readings taken here:
+
+* routing: for each token take the k largest raw logits (ties go to the lower
+  expert id); the k weights are the softmax of the selected logits
+  (renormalised top-k), stored as float32;
+* permutation: a stable counting sort of the (token, slot) assignments by
+  expert: segment e holds the tokens routed to expert e in ascending token
+  order; ``row_of[t, j]`` is the segment row of assignment (t, j);
+* gate/up: rows [0, I) of the [2I, H] weight are the gate projection, rows
+  [I, 2I) the up projection; intermediate h = silu(gate) * up with
+  silu(x) = x / (1 + exp(-x)); no clamp;
+* the intermediate is requantised to FP8 per segment row with the same rule
+  as the input activations (scale = float32(absmax / 448));
+* down: Y = (h-scale * h-codes) @ (q2 * s2)^T;
+* combine: out[t] = bf16(sum_j w[t, j] * Y[row_of[t, j]]), summed in slot
+  order; no extra routed scaling factor, no shared expert.
+
+All products and sums are float64; the only roundings are the quantisation
+points of the method (bf16 scales, INT4 values, FP8 codes, float32 scales and
+routing weights, the bf16 output).
+"""
+from __future__ import annotations
+
+from typing import Callable, Dict, Optional, Sequence
+
+import numpy as np
+
+from .numerics import bf16_round, e4m3_decode, f32_round
+from .quant import (dequantize_int4, pack_uint4b8, quant_act_fp8_per_token,
+                    rtn_quantize_int4)
+
+
+def route_topk(logits, k: int):
+    """Top-k routing: ids int32 [T, k] (best first), weights float32 [T, k].
+
+    Order key per token: (-logit, expert id).  Weights: softmax over the k
+    selected logits, computed in float64 and rounded to float32.
+    """
+    l = np.asarray(logits, dtype=np.float64)
+    T, E = l.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    ids_key = np.broadcast_to(np.arange(E), (T, E))
+    order = np.lexsort((ids_key, -l), axis=-1)
+    ids = order[:, :k].astype(np.int32)
+    sel = np.take_along_axis(l, ids.astype(np.int64), axis=1)
+    ex = np.exp(sel - sel[:, :1])
+    w = f32_round(ex / ex.sum(axis=1, keepdims=True))
+    return ids, w.astype(np.float32)
+
+
+def permute_by_expert(ids, E: int):
+    """Stable counting sort of assignments by expert.
+
+    Returns ``expert_offsets`` int32 [E+1], ``sorted_token_ids`` int32 [T*k]
+    (token of each segment row) and ``row_of`` int32 [T, k].
+    """
+    ids = np.asarray(ids, dtype=np.int64)
+    T, k = ids.shape
+    flat = ids.reshape(-1)
+    counts = np.bincount(flat, minlength=E)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    order = np.argsort(flat, kind="stable")       # by expert, then by t*k + j
+    sorted_tok = (order // k).astype(np.int32)
+    row_of = np.empty(T * k, dtype=np.int64)
+    row_of[order] = np.arange(T * k)
+    return offsets.astype(np.int32), sorted_tok, row_of.reshape(T, k).astype(np.int32)
+
+
+class ExpertStore:
+    """The oracle's own quantised experts, built lazily from bf16 weights.
+
+    ``get_weights(e)`` returns float64 arrays ``(w13 [2I, H], w2 [H, I])``
+    holding bf16 values.  Indexing returns
+    ``(w13_packed int32 [2I, H/8], s13 [2I, H/128], w2_packed int32 [H, I/8],
+    s2 [H, I/128])``.
+    """
+
+    def __init__(self, E: int, get_weights: Callable[[int], tuple]):
+        self.E = E
+        self._get = get_weights
+        self._cache: Dict[int, tuple] = {}
+
+    def __getitem__(self, e: int):
+        if e not in self._cache:
+            w13, w2 = self._get(e)
+            q13, s13 = rtn_quantize_int4(w13)
+            q2, s2 = rtn_quantize_int4(w2)
+            self._cache[e] = (pack_uint4b8(q13), s13, pack_uint4b8(q2), s2)
+        return self._cache[e]
+
+    def __len__(self):
+        return self.E
+
+
+def _silu(x):
+    return x / (1.0 + np.exp(-x))
+
+
+def moe_forward(hidden, logits, experts: Sequence, k: int,
+                tokens: Optional[np.ndarray] = None):
+    """The whole layer for all tokens, or for the token subset ``tokens``.
+
+    ``hidden``: float64 [T, H] (bf16 values); ``logits``: float32 [T, E];
+    ``experts[e]`` = ``(w13_packed, s13, w2_packed, s2)``.  Routing and the
+    permutation always cover all T tokens (they are cheap); the expert GEMMs
+    and the combine run only for the assignments of ``tokens`` (all tokens by
+    default).
+
+    Returns a dict with ``topk_ids``, ``topk_w``, ``expert_offsets``,
+    ``sorted_token_ids``, ``row_of``, ``act_codes`` / ``act_scales`` (rows of
+    ``tokens``), ``inter_codes`` / ``inter_scales`` (keyed by segment row, for
+    the rows computed), ``out`` float64 [len(tokens), H] bf16 values and
+    ``tokens``.
+    """
+    hidden = np.asarray(hidden, dtype=np.float64)
+    T, H = hidden.shape
+    E = logits.shape[1]
+    ids, w = route_topk(logits, k)
+    offsets, sorted_tok, row_of = permute_by_expert(ids, E)
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    pos = {int(t): i for i, t in enumerate(tokens)}
+
+    codes, a_scale = quant_act_fp8_per_token(hidden[tokens])
+    x_deq = a_scale[:, None] * e4m3_decode(codes)          # exact: 24-bit x 4-bit significands
+
+    need_rows = np.sort(row_of[tokens].reshape(-1))
+    Y: Dict[int, np.ndarray] = {}
+    inter_codes: Dict[int, np.ndarray] = {}
+    inter_scales: Dict[int, float] = {}
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        rows = need_rows[(need_rows >= lo) & (need_rows < hi)]
+        if rows.size == 0:
+            continue
+        w13p, s13, w2p, s2 = experts[e]
+        I = w13p.shape[0] // 2
+        X = x_deq[[pos[int(sorted_tok[r])] for r in rows]]  # [n, H]
+        G = X @ dequantize_int4(w13p, s13).T                 # [n, 2I]
+        h = _silu(G[:, :I]) * G[:, I:]
+        hc, hs = quant_act_fp8_per_token(h)
+        hd = hs[:, None] * e4m3_decode(hc)
+        Ye = hd @ dequantize_int4(w2p, s2).T                 # [n, H]
+        for i, r in enumerate(rows):
+            Y[int(r)] = Ye[i]
+            inter_codes[int(r)] = hc[i]
+            inter_scales[int(r)] = float(hs[i])
+
+    out = np.zeros((len(tokens), H), dtype=np.float64)
+    for i, t in enumerate(tokens):
+        acc = np.zeros(H, dtype=np.float64)
+        for j in range(k):
+            acc = acc + float(w[t, j]) * Y[int(row_of[t, j])]
+        out[i] = bf16_round(acc)
+
+    return dict(topk_ids=ids, topk_w=w, expert_offsets=offsets, sorted_token_ids=sorted_tok,
+                row_of=row_of, act_codes=codes, act_scales=a_scale, inter_codes=inter_codes,
+                inter_scales=inter_scales, out=out, tokens=tokens)
