@@ -1,0 +1,347 @@
+"""Benchmark of the W4A8 routed-expert MoE layer on B200.
+
+One step = one ``w4a8_moe_forward`` (activation quantisation, routing +
+permutation, gate/up grouped GEMM + SwiGLU, intermediate requantisation, down
+grouped GEMM, combine) over one batch of synthetic tokens.  Prints one JSON
+line.  ``--impl reference`` times the CPU oracle instead (the only other
+place this script runs ``oracle/``).
+
+Multi-GPU: one process per GPU (torchrun); each rank runs its own batch
+through its own copy of the experts (data parallel, no collective on the data
+path): weak scaling, value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200 + % of HBM (decode) / FP8-peak (prefill) roofline"
+DEFAULT_CONFIG = workloads.CONFIGS[1].name
+KERNELS_PER_STEP = 8   # act_quant, route topk/scan/scatter, gemm1, inter_quant, gemm2, combine
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sus=d.get("bf16_tflops_sustained", d["bf16_tflops"]), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def build_layer(cfg, device, w4):
+    """Pack every expert's seeded bf16 weights on the device (not timed)."""
+    E, H, I = cfg.E, cfg.H, cfg.I
+    p13 = torch.empty(E, 2 * I, H // 8, dtype=torch.int32, device=device)
+    s13 = torch.empty(E, 2 * I, H // 128, dtype=torch.bfloat16, device=device)
+    p2 = torch.empty(E, H, I // 8, dtype=torch.int32, device=device)
+    s2 = torch.empty(E, H, I // 128, dtype=torch.bfloat16, device=device)
+    for e in range(E):
+        w13, w2 = workloads.gen_expert_weights(cfg, e, device=device)
+        w4.w4a8_pack_int4(w13, packed=p13[e], scales=s13[e])
+        w4.w4a8_pack_int4(w2, packed=p2[e], scales=s2[e])
+    torch.cuda.synchronize(device)
+    return w4.W4A8MoELayer(p13, s13, p2, s2, cfg.k)
+
+
+def algorithmic_work(cfg, counts):
+    """Algorithmic bytes and FLOPs of each grouped GEMM for the given expert counts."""
+    T, H, I, k = cfg.T, cfg.H, cfg.I, cfg.k
+    A = T * k
+    active = int(np.count_nonzero(counts))
+    w13_bytes = 2 * I * H // 2 + 2 * I * (H // 128) * 2
+    w2_bytes = H * I // 2 + H * (I // 128) * 2
+    g1 = dict(bytes=active * w13_bytes + T * H + T * 4 + A * I * 4 + A * 4 + A * 8,
+              flops=2 * A * 2 * I * H)
+    g2 = dict(bytes=active * w2_bytes + A * I + A * 4 + A * H * 4, flops=2 * A * H * I)
+    return g1, g2, active
+
+
+class OracleSample:
+    """The CPU oracle on a seeded sample of tokens, experts quantised up front."""
+
+    def __init__(self, cfg, n_tokens: int, seed_tokens: int = 7):
+        import oracle
+        self.oracle, self.cfg = oracle, cfg
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max((p.get("num_threads", 1) for p in threadpool_info()), default=None)
+        except Exception:
+            self.cores = None
+        self.cores = self.cores or os.cpu_count()
+        f = lambda t: oracle.bf16_bits_to_f64(t.contiguous().view(torch.int16).numpy()
+                                              .view(np.uint16))
+        self.hidden = f(workloads.gen_hidden(cfg))
+        self.logits = workloads.gen_logits(cfg).numpy()
+        rng = np.random.default_rng(seed_tokens)
+        self.tokens = np.sort(rng.choice(cfg.T, size=min(n_tokens, cfg.T), replace=False))
+        ids, _ = oracle.route_topk(self.logits, cfg.k)
+
+        def weights(e):
+            a, b = workloads.gen_expert_weights(cfg, e)
+            return f(a), f(b)
+
+        self.store = oracle.ExpertStore(cfg.E, weights)
+        for e in sorted(set(ids[self.tokens].reshape(-1).tolist())):
+            self.store[e]                          # quantise outside the timed region
+
+    def run(self) -> float:
+        t0 = time.perf_counter()
+        self.oracle.moe_forward(self.hidden, self.logits, self.store, self.cfg.k,
+                                tokens=self.tokens)
+        return time.perf_counter() - t0
+
+    def describe(self, dt: float) -> str:
+        return (f"{len(self.tokens)} of {self.cfg.T} tokens of {self.cfg.name} per step "
+                f"(their {self.cfg.k} experts each, RTN-quantised before timing), float64 "
+                f"numpy, {dt:.2f} s per step")
+
+
+def cpu_baseline(cfg, n_tokens: int):
+    s = OracleSample(cfg, n_tokens)
+    dt = s.run()
+    return dict(value=len(s.tokens) / dt, unit="tokens/s", cores=s.cores, kind="oracle",
+                sample=s.describe(dt))
+
+
+def bench_reference(args, cfg, rank):
+    if rank != 0:
+        return 0
+    s = OracleSample(cfg, max(1, args.ref_tokens))
+    for _ in range(args.warmup):
+        s.run()
+    times = [s.run() for _ in range(args.steps)]
+    tot = sum(times)
+    value = len(s.tokens) * args.steps / tot
+    line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * tot / args.steps, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                impl="reference",
+                config=dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
+                            sample_tokens_per_step=len(s.tokens)),
+                cpu_baseline=dict(value=value, unit="tokens/s", cores=s.cores, kind="oracle",
+                                  sample=s.describe(tot / args.steps)),
+                e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0,
+                         d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG,
+                    choices=[c.name for c in workloads.CONFIGS])
+    ap.add_argument("--cpu-tokens", type=int, default=2,
+                    help="tokens in the oracle sample of cpu_baseline (0: skip)")
+    ap.add_argument("--ref-tokens", type=int, default=1,
+                    help="tokens per step of the --impl reference arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    cfg = workloads.config_by_name(args.config)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return bench_reference(args, cfg, rank)
+
+    import w4a8_quantized_moe_b200 as w4
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    layer = build_layer(cfg, device, w4)
+    rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)      # each rank its own batch
+    hidden = workloads.gen_hidden(rank_cfg, device=device)
+    logits = workloads.gen_logits(rank_cfg, device=device)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=device)
+    ws = layer.workspace(cfg.T)
+    offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(events=None):
+        layer(hidden, logits, out=out, aux={"expert_offsets": offsets}, stage_events=events)
+
+    for _ in range(args.warmup):
+        step()
+    w4.w4a8_check_device_error(device)
+    counts = np.diff(offsets.cpu().numpy().astype(np.int64))
+
+    # ---------------- device-resident timing (kernel path)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * w4.NUM_STAGES)]
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    w4.w4a8_check_device_error(device)
+    ms = t_start.elapsed_time(t_end)
+    stage_ms = [statistics.mean(ev[i][2 * s].elapsed_time(ev[i][2 * s + 1])
+                                for i in range(args.steps)) for s in range(w4.NUM_STAGES)]
+
+    # ---------------- end to end through the public API, host buffers
+    h_host = hidden.cpu().pin_memory()
+    l_host = logits.cpu().pin_memory()
+    o_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    h_dev = torch.empty_like(hidden)
+    l_dev = torch.empty_like(logits)
+
+    def e2e_step():
+        h_dev.copy_(h_host, non_blocking=True)
+        l_dev.copy_(l_host, non_blocking=True)
+        layer(h_dev, l_dev, out=out)
+        o_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e_start.elapsed_time(e_end)
+
+    if dist:
+        t = torch.tensor([ms, e2e_ms] + stage_ms, device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+        stage_ms = [float(x) for x in t[2:]]
+
+    tokens = cfg.T * world * args.steps
+    value = tokens / (ms / 1e3)
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    pk = peaks()
+    g1, g2, active = algorithmic_work(cfg, counts)
+    prefill = cfg.T >= 4096
+    gi = 2 if stage_ms[2] >= stage_ms[4] else 4          # dominant kernel: the slower GEMM
+    work = g1 if gi == 2 else g2
+    kname = "grouped_gemm_gate_up" if gi == 2 else "grouped_gemm_down"
+    if prefill:
+        achieved = work["flops"] / (stage_ms[gi] / 1e3) / 1e12
+        peak = 2.0 * pk["bf16_sus"]                     # FP8 = 2 x bf16 (nominal ratio)
+        roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
+                    frac=achieved / peak, traffic=None, kernel=kname,
+                    peak_source=f"{pk['src']} sustained bf16 x 2")
+    else:
+        achieved = work["bytes"] / (stage_ms[gi] / 1e3) / 1e9
+        peak = pk["hbm"]
+        roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
+                    traffic=None, kernel=kname, peak_source=f"{pk['src']} HBM copy")
+
+    line = dict(
+        metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=ms / args.steps, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="e4m3xint4-f32acc", data="synthetic",
+        config=dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
+                    active_experts=active, parallelism=f"dp{world}" if world > 1 else "single",
+                    l2=("inputs larger than L2: %.2f GB of packed experts streamed per step"
+                        % ((g1["bytes"] + g2["bytes"]) / 1e9))),
+        stage_ms={n: round(x, 5) for n, x in zip(w4.STAGE_NAMES, stage_ms)},
+        roofline=roof,
+        e2e=dict(value=e2e_value, unit="tokens/s",
+                 h2d_bytes_per_step=cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
+                 d2h_bytes_per_step=cfg.T * cfg.H * 2),
+        gpu_launches=KERNELS_PER_STEP * args.steps,
+        clocks=clk.summary(),
+    )
+    if rank == 0 and world == 1 and args.cpu_tokens > 0:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * w4a8.h - C ABI of the B200 (sm_100a) W4A8 routed-expert MoE library.
+ *
+ * The library computes one routed-expert MoE layer whose experts hold INT4
+ * weights and take FP8 (E4M3) activations, as described by the GLM-5.3-W4A8
+ * model card (intro; table "differences from the other 4-bit releases";
+ * section "quantisation method"): routed experts in symmetric INT4 with one
+ * scale per group of 128 weights along K, packed as compressed-tensors
+ * "pack-quantized" uint4b8 nibbles, 8 per int32 word; activations quantised
+ * to FP8 at run time with one dynamic scale per token; INT4 converted to FP8
+ * inside the GEMM, never dequantised to BF16 in memory.
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument is DEVICE memory owned by the caller, unless its
+ *    comment says otherwise.  The library never allocates device memory and
+ *    never frees caller memory; scratch space comes from a caller-supplied
+ *    workspace whose size is given by the matching *_workspace_size call.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  The returned status covers host-side argument checks
+ *    and kernel-launch errors only.  Kernels with inter-warp waits bound every
+ *    wait; a wait that runs out sets a device error latch that
+ *    w4a8_check_device_error() reports.
+ *  - Row-major layouts, element strides as stated, no padding between rows.
+ *    Device pointers must be 16-byte aligned.
+ *  - The device must be compute capability 10.x (the code is built for
+ *    sm_100a); other devices get W4A8_ERR_UNSUPPORTED_ARCH.
+ *  - On error nothing is launched and w4a8_last_error() (thread-local) holds
+ *    a message.
+ */
+#ifndef W4A8_H_
+#define W4A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W4A8_API __attribute__((visibility("default")))
+#else
+#define W4A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t w4a8_status;
+#define W4A8_OK                      0
+#define W4A8_ERR_INVALID_ARG         1  /* null pointer, misalignment, negative size */
+#define W4A8_ERR_UNSUPPORTED_SHAPE   2  /* shape outside the supported set (see each call) */
+#define W4A8_ERR_UNSUPPORTED_ARCH    3  /* device is not compute capability 10.x */
+#define W4A8_ERR_WORKSPACE_TOO_SMALL 4  /* workspace_bytes below the *_workspace_size value */
+#define W4A8_ERR_CUDA                5  /* a CUDA runtime call or launch failed */
+#define W4A8_ERR_DEVICE_TIMEOUT      6  /* a bounded in-kernel wait ran out (reported later) */
+
+/* Number of timed stages of w4a8_moe_forward (see w4a8_moe_aux.stage_events). */
+#define W4A8_NUM_STAGES 6
+
+/* ABI version of this header (incremented on incompatible changes). */
+W4A8_API int32_t w4a8_abi_version(void);
+
+/* Static text of a status code. */
+W4A8_API const char* w4a8_status_string(w4a8_status status);
+
+/* Message of the last failing call on this host thread ("" if none). */
+W4A8_API const char* w4a8_last_error(void);
+
+/*
+ * w4a8_check_device_error - report and clear the device error latch.
+ * Synchronises `stream`, then returns W4A8_ERR_DEVICE_TIMEOUT if any kernel of
+ * this library on the current device gave up a bounded wait since the last
+ * check, W4A8_ERR_CUDA if the stream holds a CUDA error, else W4A8_OK.
+ */
+W4A8_API w4a8_status w4a8_check_device_error(void* stream);
+
+/*
+ * w4a8_pack_int4 - symmetric INT4 round-to-nearest weight quantisation with
+ * one bf16 scale per group of `group` weights along K, packed as uint4b8.
+ * (GLM-5.3-W4A8 model card, "quantisation method": symmetric INT4, group
+ * size 128, compressed-tensors pack-quantized uint4b8 / int32.)
+ *
+ * For every row r and group g:  s = bf16(absmax / 7) (float32 division, then
+ * round-to-nearest-even to bf16);  q = clamp(rint(w / s), -8, 7) with the
+ * float32 quotient (q = 0 when s == 0);  nibble q + 8 of element kappa goes to
+ * word kappa / 8, bits 4*(kappa % 8) .. +3.
+ *
+ *   w_bf16       [R, K] bf16, row-major (R = experts * rows per expert)
+ *   R, K         R >= 0; K > 0 and K % 128 == 0
+ *   group        must be 128 (else W4A8_ERR_UNSUPPORTED_SHAPE)
+ *   packed       [R, K / 8] int32, written
+ *   scales_bf16  [R, K / 128] bf16, written
+ */
+W4A8_API w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, int32_t group,
+                           int32_t* packed, void* scales_bf16, void* stream);
+
+/*
+ * w4a8_quant_act_fp8_per_token - dynamic per-token FP8 E4M3 quantisation.
+ * (Model card, "quantisation method" and the table above: FP8 per-token
+ * dynamic activations.)
+ *
+ * Per row t:  scale[t] = absmax(x[t]) / 448 (float32 division);
+ * codes[t, :] = E4M3(x / scale[t]) rounded to nearest even, saturating to
+ * +-448, sign of zero kept; a row whose absmax is 0 gets scale 0 and codes 0.
+ *
+ *   x_bf16      [T, H] bf16
+ *   T, H        T >= 0 (T == 0 is a no-op); H > 0 and H % 16 == 0
+ *   codes_e4m3  [T, H] uint8, written
+ *   scales      [T] float32, written
+ */
+W4A8_API w4a8_status w4a8_quant_act_fp8_per_token(const void* x_bf16, int64_t T, int64_t H,
+                                         uint8_t* codes_e4m3, float* scales, void* stream);
+
+/*
+ * w4a8_moe_route_workspace_size - bytes of scratch w4a8_moe_route_permute needs.
+ */
+W4A8_API size_t w4a8_moe_route_workspace_size(int64_t T, int32_t E);
+
+/*
+ * w4a8_moe_route_permute - top-k routing and the token -> expert permutation
+ * that forms the grouped-GEMM segments (the layer's experts run as one
+ * grouped GEMM per projection: model card intro "CUTLASS W4A8 grouped GEMM").
+ *
+ * Routing: per token, the k largest logits (a tie goes to the lower expert
+ * id); slot j holds the j-th best.  topk_w = softmax of the k selected logits
+ * (float32 arithmetic, the renormalised top-k).  Precondition: logits are not
+ * NaN and each token has at least k finite logits.
+ * Permutation: stable counting sort of the (t, j) pairs by expert.  Segment e
+ * is rows [expert_offsets[e], expert_offsets[e+1]) and lists its tokens in
+ * ascending order in sorted_token_ids; row_of[t, j] is the row of (t, j).
+ *
+ *   logits            [T, E] float32
+ *   T, E, k           T >= 0; 1 <= E <= 1024; 1 <= k <= min(E, 32)
+ *   topk_ids          [T, k] int32, written
+ *   topk_w            [T, k] float32, written
+ *   expert_offsets    [E + 1] int32, written
+ *   sorted_token_ids  [T * k] int32, written
+ *   row_of            [T, k] int32, written
+ *   workspace         scratch of >= w4a8_moe_route_workspace_size(T, E) bytes
+ */
+W4A8_API w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int32_t E, int32_t k,
+                                   int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                   int32_t* sorted_token_ids, int32_t* row_of,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Optional outputs and instrumentation of w4a8_moe_forward.  Every member may
+ * be NULL.  A non-NULL buffer replaces the workspace region of the same
+ * intermediate, so it receives exactly what the layer computed.  Shapes use
+ * A = T * k assignments.
+ */
+typedef struct w4a8_moe_aux {
+    int32_t* topk_ids;          /* [T, k] */
+    float* topk_w;              /* [T, k] */
+    int32_t* expert_offsets;    /* [E + 1] */
+    int32_t* sorted_token_ids;  /* [A] */
+    int32_t* row_of;            /* [T, k] */
+    uint8_t* act_codes;         /* [T, H] E4M3 codes of the hidden states */
+    float* act_scales;          /* [T] */
+    float* inter_h;             /* [A, I] float32 SwiGLU output before requantisation */
+    uint8_t* inter_codes;       /* [A, I] E4M3 codes of the intermediate (segment rows) */
+    float* inter_scales;        /* [A] */
+    float* y_rows;              /* [A, H] float32 down-projection output per segment row */
+    /* If non-NULL: 2 * W4A8_NUM_STAGES cudaEvent_t handles (host memory array).
+     * Event 2i is recorded before stage i and 2i+1 after it, on `stream`.
+     * Stages: 0 activation quantisation, 1 routing + permutation, 2 gate/up
+     * GEMM + SwiGLU, 3 intermediate requantisation, 4 down GEMM, 5 combine. */
+    void* const* stage_events;
+} w4a8_moe_aux;
+
+/*
+ * w4a8_moe_workspace_size - bytes of scratch w4a8_moe_forward needs.
+ */
+W4A8_API size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k);
+
+/*
+ * w4a8_moe_forward - one W4A8 routed-expert MoE layer.
+ *
+ *   1. activation quantisation (as w4a8_quant_act_fp8_per_token);
+ *   2. routing + permutation (as w4a8_moe_route_permute);
+ *   3. gate/up grouped GEMM on the tensor cores: for segment row r of expert
+ *      e, G[r, n] = a_s[t] * sum_g s13[e, n, g] * sum_{kappa in g}
+ *      e4m3(x[t, kappa]) * q13[e, n, kappa]; INT4 is converted to E4M3 (exact
+ *      for -8..7) in the kernel, each 128-wide K group is accumulated in FP32
+ *      and scaled by its group scale; then h = silu(G[:, :I]) * G[:, I:];
+ *   4. per-row FP8 requantisation of h (same rule as step 1);
+ *   5. down grouped GEMM: Y[r, n] = h_s[r] * sum_g s2[e, n, g] * sum e4m3 * q2;
+ *   6. combine: out[t] = bf16(sum_j topk_w[t, j] * Y[row_of[t, j]]), slot order.
+ *
+ *   hidden_bf16   [T, H] bf16
+ *   logits        [T, E] float32 router logits
+ *   w13_packed    [E, 2I, H / 8] int32 (w4a8_pack_int4 of the [E*2I, H]
+ *                 gate/up weight; rows [0, I) of each expert are the gate
+ *                 projection, rows [I, 2I) the up projection)
+ *   w13_scales    [E, 2I, H / 128] bf16
+ *   w2_packed     [E, H, I / 8] int32
+ *   w2_scales     [E, H, I / 128] bf16
+ *   T, H, I, E, k T >= 0 (0: no-op); H % 128 == 0, I % 128 == 0, both > 0;
+ *                 1 <= E <= 1024; 1 <= k <= min(E, 32)
+ *   out_bf16      [T, H] bf16, written
+ *   workspace     scratch of >= w4a8_moe_workspace_size(T, H, I, E, k) bytes
+ *   aux           optional, see w4a8_moe_aux (NULL for none)
+ */
+W4A8_API w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
+                             const int32_t* w13_packed, const void* w13_scales,
+                             const int32_t* w2_packed, const void* w2_scales,
+                             int64_t T, int64_t H, int64_t I, int32_t E, int32_t k,
+                             void* out_bf16, void* workspace, size_t workspace_bytes,
+                             const w4a8_moe_aux* aux, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* W4A8_H_ */

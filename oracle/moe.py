@@ -119,9 +119,9 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
 
     Returns a dict with ``topk_ids``, ``topk_w``, ``expert_offsets``,
     ``sorted_token_ids``, ``row_of``, ``act_codes`` / ``act_scales`` (rows of
-    ``tokens``), ``inter_codes`` / ``inter_scales`` (keyed by segment row, for
-    the rows computed), ``out`` float64 [len(tokens), H] bf16 values and
-    ``tokens``.
+    ``tokens``), ``inter_h`` / ``inter_codes`` / ``inter_scales`` / ``y_rows``
+    (keyed by segment row, for the rows computed), ``out`` float64
+    [len(tokens), H] bf16 values and ``tokens``.
     """
     hidden = np.asarray(hidden, dtype=np.float64)
     T, H = hidden.shape
@@ -136,6 +136,7 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
 
     need_rows = np.sort(row_of[tokens].reshape(-1))
     Y: Dict[int, np.ndarray] = {}
+    inter_h: Dict[int, np.ndarray] = {}
     inter_codes: Dict[int, np.ndarray] = {}
     inter_scales: Dict[int, float] = {}
     for e in range(E):
@@ -153,6 +154,7 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
         Ye = hd @ dequantize_int4(w2p, s2).T                 # [n, H]
         for i, r in enumerate(rows):
             Y[int(r)] = Ye[i]
+            inter_h[int(r)] = h[i]
             inter_codes[int(r)] = hc[i]
             inter_scales[int(r)] = float(hs[i])
 
@@ -164,5 +166,6 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
         out[i] = bf16_round(acc)
 
     return dict(topk_ids=ids, topk_w=w, expert_offsets=offsets, sorted_token_ids=sorted_tok,
-                row_of=row_of, act_codes=codes, act_scales=a_scale, inter_codes=inter_codes,
-                inter_scales=inter_scales, out=out, tokens=tokens)
+                row_of=row_of, act_codes=codes, act_scales=a_scale, inter_h=inter_h,
+                inter_codes=inter_codes, inter_scales=inter_scales, y_rows=Y, out=out,
+                tokens=tokens)

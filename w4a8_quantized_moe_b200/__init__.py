@@ -1,0 +1,286 @@
+"""Python binding of the B200 W4A8 routed-expert MoE library (``libw4a8.so``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  The
+functions carry the names of the C entry points in ``include/w4a8.h``.
+There is no CPU fallback: without the built library, or without a CUDA
+device, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+import torch
+
+__all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_abi_version",
+           "w4a8_status_string", "w4a8_pack_int4", "w4a8_quant_act_fp8_per_token",
+           "w4a8_moe_route_workspace_size", "w4a8_moe_route_permute", "w4a8_moe_workspace_size",
+           "w4a8_moe_forward", "w4a8_check_device_error", "W4A8MoELayer"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a8.so")
+NUM_STAGES = 6
+STAGE_NAMES = ["act_quant", "route_permute", "gemm_gate_up", "inter_quant", "gemm_down",
+               "combine"]
+
+_lib = None
+
+
+class W4A8Error(RuntimeError):
+    """A library call returned a non-zero status."""
+
+    def __init__(self, func: str, status: int, message: str):
+        self.status = status
+        super().__init__(f"{func}: {_status_name(status)}: {message}")
+
+
+class MoEAux(ctypes.Structure):
+    _fields_ = [("topk_ids", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
+                ("expert_offsets", ctypes.c_void_p), ("sorted_token_ids", ctypes.c_void_p),
+                ("row_of", ctypes.c_void_p), ("act_codes", ctypes.c_void_p),
+                ("act_scales", ctypes.c_void_p), ("inter_h", ctypes.c_void_p),
+                ("inter_codes", ctypes.c_void_p), ("inter_scales", ctypes.c_void_p),
+                ("y_rows", ctypes.c_void_p), ("stage_events", ctypes.c_void_p)]
+
+
+def _declare(L):
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "w4a8_abi_version": (i32, []),
+        "w4a8_status_string": (ctypes.c_char_p, [i32]),
+        "w4a8_last_error": (ctypes.c_char_p, []),
+        "w4a8_check_device_error": (i32, [vp]),
+        "w4a8_pack_int4": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+        "w4a8_quant_act_fp8_per_token": (i32, [vp, i64, i64, vp, vp, vp]),
+        "w4a8_moe_route_workspace_size": (sz, [i64, i32]),
+        "w4a8_moe_route_permute": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "w4a8_moe_workspace_size": (sz, [i64, i64, i64, i32, i32]),
+        "w4a8_moe_forward": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, sz,
+                                   vp, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+
+
+def lib():
+    """The loaded ``libw4a8.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m w4a8_quantized_moe_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+def _status_name(status: int) -> str:
+    try:
+        return lib().w4a8_status_string(status).decode()
+    except Exception:  # pragma: no cover - only reached while reporting another error
+        return f"status {status}"
+
+
+def _check(func: str, status: int):
+    if status != 0:
+        raise W4A8Error(func, status, lib().w4a8_last_error().decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def w4a8_abi_version() -> int:
+    return int(lib().w4a8_abi_version())
+
+
+def w4a8_status_string(status: int) -> str:
+    return lib().w4a8_status_string(status).decode()
+
+
+def w4a8_check_device_error(device=None):
+    """Synchronise the current stream and raise if a bounded in-kernel wait ran out."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check("w4a8_check_device_error", lib().w4a8_check_device_error(_stream(dev)))
+
+
+def w4a8_pack_int4(w: torch.Tensor, group: int = 128, packed: Optional[torch.Tensor] = None,
+                   scales: Optional[torch.Tensor] = None):
+    """INT4 RTN group-128 quantisation + uint4b8 packing of bf16 ``w`` [..., K].
+
+    Returns ``(packed int32 [..., K/8], scales bf16 [..., K/128])``.
+    """
+    if w.dim() < 2:
+        raise ValueError("w must have at least 2 dims")
+    lead, K = tuple(w.shape[:-1]), w.shape[-1]
+    w2 = w.reshape(-1, K)
+    _need(w2, "w", torch.bfloat16, 2)
+    R = w2.shape[0]
+    if packed is None:
+        packed = torch.empty(*lead, K // 8, dtype=torch.int32, device=w.device)
+    if scales is None:
+        scales = torch.empty(*lead, max(K // group, 0), dtype=torch.bfloat16, device=w.device)
+    _check("w4a8_pack_int4", lib().w4a8_pack_int4(_p(w2), R, K, group, _p(packed), _p(scales),
+                                                  _stream(w.device)))
+    return packed, scales
+
+
+def w4a8_quant_act_fp8_per_token(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                                 scales: Optional[torch.Tensor] = None):
+    """Per-token dynamic E4M3 quantisation of bf16 ``x`` [T, H] -> (uint8 codes, f32 scales)."""
+    _need(x, "x", torch.bfloat16, 2)
+    T, H = x.shape
+    if codes is None:
+        codes = torch.empty(T, H, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check("w4a8_quant_act_fp8_per_token",
+           lib().w4a8_quant_act_fp8_per_token(_p(x), T, H, _p(codes), _p(scales),
+                                              _stream(x.device)))
+    return codes, scales
+
+
+def w4a8_moe_route_workspace_size(T: int, E: int) -> int:
+    return int(lib().w4a8_moe_route_workspace_size(T, E))
+
+
+def w4a8_moe_route_permute(logits: torch.Tensor, k: int,
+                           workspace: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Top-k routing + stable permutation by expert (see include/w4a8.h)."""
+    _need(logits, "logits", torch.float32, 2)
+    T, E = logits.shape
+    dev = logits.device
+    out = dict(topk_ids=torch.empty(T, k, dtype=torch.int32, device=dev),
+               topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+               expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               sorted_token_ids=torch.empty(T * k, dtype=torch.int32, device=dev),
+               row_of=torch.empty(T, k, dtype=torch.int32, device=dev))
+    need = w4a8_moe_route_workspace_size(T, E)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("w4a8_moe_route_permute",
+           lib().w4a8_moe_route_permute(_p(logits), T, E, k, _p(out["topk_ids"]),
+                                        _p(out["topk_w"]), _p(out["expert_offsets"]),
+                                        _p(out["sorted_token_ids"]), _p(out["row_of"]),
+                                        _p(workspace), workspace.numel(), _stream(dev)))
+    return out
+
+
+def w4a8_moe_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(lib().w4a8_moe_workspace_size(T, H, I, E, k))
+
+
+_AUX_FIELDS = ["topk_ids", "topk_w", "expert_offsets", "sorted_token_ids", "row_of", "act_codes",
+               "act_scales", "inter_h", "inter_codes", "inter_scales", "y_rows"]
+
+
+def w4a8_moe_forward(hidden: torch.Tensor, logits: torch.Tensor, w13_packed: torch.Tensor,
+                     w13_scales: torch.Tensor, w2_packed: torch.Tensor, w2_scales: torch.Tensor,
+                     k: int, out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None,
+                     aux: Optional[Dict[str, torch.Tensor]] = None,
+                     stage_events: Optional[Sequence[torch.cuda.Event]] = None) -> torch.Tensor:
+    """One W4A8 MoE layer: returns bf16 [T, H].
+
+    ``aux`` maps names of ``w4a8_moe_aux`` members to caller tensors that then
+    receive the intermediates; ``stage_events`` (2 * NUM_STAGES timing-enabled
+    CUDA events) are recorded around the stages.
+    """
+    _need(hidden, "hidden", torch.bfloat16, 2)
+    _need(logits, "logits", torch.float32, 2)
+    _need(w13_packed, "w13_packed", torch.int32, 3)
+    _need(w13_scales, "w13_scales", torch.bfloat16, 3)
+    _need(w2_packed, "w2_packed", torch.int32, 3)
+    _need(w2_scales, "w2_scales", torch.bfloat16, 3)
+    T, H = hidden.shape
+    E = logits.shape[1]
+    I = w2_packed.shape[2] * 8
+    if logits.shape[0] != T or w13_packed.shape != (E, 2 * I, H // 8) or \
+            w2_packed.shape != (E, H, I // 8):
+        raise ValueError("inconsistent shapes: hidden [T,H], logits [T,E], w13 [E,2I,H/8], "
+                         "w2 [E,H,I/8]")
+    dev = hidden.device
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    need = w4a8_moe_workspace_size(T, H, I, E, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    aux_struct = None
+    keep = []
+    if aux or stage_events:
+        aux_struct = MoEAux()
+        for name, t in (aux or {}).items():
+            if name not in _AUX_FIELDS:
+                raise KeyError(f"unknown aux buffer {name!r}")
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"aux[{name!r}] must be a contiguous CUDA tensor")
+            setattr(aux_struct, name, t.data_ptr())
+        if stage_events:
+            if len(stage_events) != 2 * NUM_STAGES:
+                raise ValueError(f"need {2 * NUM_STAGES} events")
+            arr = (ctypes.c_void_p * (2 * NUM_STAGES))(*[e.cuda_event for e in stage_events])
+            keep.append(arr)
+            aux_struct.stage_events = ctypes.cast(arr, ctypes.c_void_p)
+    _check("w4a8_moe_forward",
+           lib().w4a8_moe_forward(_p(hidden), _p(logits), _p(w13_packed), _p(w13_scales),
+                                  _p(w2_packed), _p(w2_scales), T, H, I, E, k, _p(out),
+                                  _p(workspace), workspace.numel(),
+                                  None if aux_struct is None else ctypes.byref(aux_struct),
+                                  _stream(dev)))
+    return out
+
+
+class W4A8MoELayer:
+    """A layer with packed experts resident on the device and a reusable workspace.
+
+    ``W4A8MoELayer.from_bf16(w13, w2, k)`` packs bf16 ``w13`` [E, 2I, H] and
+    ``w2`` [E, H, I] with ``w4a8_pack_int4``; calling the layer runs
+    ``w4a8_moe_forward``.
+    """
+
+    def __init__(self, w13_packed, w13_scales, w2_packed, w2_scales, k: int):
+        self.w13_packed, self.w13_scales = w13_packed, w13_scales
+        self.w2_packed, self.w2_scales = w2_packed, w2_scales
+        self.k = k
+        self.E, twoI, h8 = w13_packed.shape
+        self.H, self.I = h8 * 8, twoI // 2
+        self._ws = None
+
+    @classmethod
+    def from_bf16(cls, w13: torch.Tensor, w2: torch.Tensor, k: int) -> "W4A8MoELayer":
+        p13, s13 = w4a8_pack_int4(w13)
+        p2, s2 = w4a8_pack_int4(w2)
+        return cls(p13, s13, p2, s2, k)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = max(w4a8_moe_workspace_size(T, self.H, self.I, self.E, self.k), 1)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.w13_packed.device)
+        return self._ws
+
+    def __call__(self, hidden: torch.Tensor, logits: torch.Tensor,
+                 out: Optional[torch.Tensor] = None, **kw) -> torch.Tensor:
+        return w4a8_moe_forward(hidden, logits, self.w13_packed, self.w13_scales, self.w2_packed,
+                                self.w2_scales, self.k, out=out,
+                                workspace=self.workspace(hidden.shape[0]), **kw)

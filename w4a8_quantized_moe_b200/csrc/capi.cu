@@ -1,0 +1,453 @@
+// capi.cu - the extern "C" entry points declared in include/w4a8.h: argument
+// checks, workspace layout, TMA descriptors and the launch sequence.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/w4a8.h"
+#include "internal.h"
+
+namespace w4a8 {
+cudaError_t read_and_clear_device_error(int* value);
+}
+
+using namespace w4a8;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+w4a8_status fail(w4a8_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+w4a8_status cuda_fail(cudaError_t err, const char* where) {
+  return fail(W4A8_ERR_CUDA, "%s: %s", where, cudaGetErrorString(err));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int major = 0;
+  int sms = 0;
+};
+
+// Current device's compute capability and SM count (cached per device).
+w4a8_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err, "cudaGetDevice");
+  DeviceInfo d;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && have[dev]) d = cache[dev];
+  }
+  if (d.sms == 0) {
+    err = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (err == cudaSuccess)
+      err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return cuda_fail(err, "cudaDeviceGetAttribute");
+    if (dev < 64) {
+      std::lock_guard<std::mutex> lock(mu);
+      cache[dev] = d;
+      have[dev] = true;
+    }
+  }
+  *out = d;
+  if (d.major != 10)
+    return fail(W4A8_ERR_UNSUPPORTED_ARCH,
+                "device compute capability %d.x; this library is built for sm_100a (10.x)",
+                d.major);
+  return W4A8_OK;
+}
+
+// Bump allocator over the caller's workspace (or over nullptr to size it).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = reinterpret_cast<T*>(base + off);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct RouteBufs {
+  int32_t* block_counts;
+  int32_t* block_base;
+  int32_t* tile_prefix;
+};
+
+RouteBufs carve_route(Carver& c, int64_t T, int E) {
+  RouteBufs b;
+  const size_t n = static_cast<size_t>(route_blocks(T)) * static_cast<size_t>(E);
+  b.block_counts = c.take<int32_t>(n);
+  b.block_base = c.take<int32_t>(n);
+  b.tile_prefix = c.take<int32_t>(static_cast<size_t>(E) + 1);
+  return b;
+}
+
+struct ForwardBufs {
+  int32_t* topk_ids;
+  float* topk_w;
+  int32_t* expert_offsets;
+  int32_t* sorted_token_ids;
+  int32_t* row_of;
+  RouteBufs route;
+  uint8_t* act_codes;
+  float* act_scales;
+  float* h;
+  uint32_t* row_amax;
+  uint8_t* inter_codes;
+  float* inter_scales;
+  float* y;
+};
+
+ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int k) {
+  ForwardBufs b;
+  const size_t A = static_cast<size_t>(T) * static_cast<size_t>(k);
+  b.topk_ids = c.take<int32_t>(A);
+  b.topk_w = c.take<float>(A);
+  b.expert_offsets = c.take<int32_t>(static_cast<size_t>(E) + 1);
+  b.sorted_token_ids = c.take<int32_t>(A);
+  b.row_of = c.take<int32_t>(A);
+  b.route = carve_route(c, T, E);
+  b.act_codes = c.take<uint8_t>(static_cast<size_t>(T) * static_cast<size_t>(H));
+  b.act_scales = c.take<float>(static_cast<size_t>(T));
+  b.h = c.take<float>(A * static_cast<size_t>(I));
+  b.row_amax = c.take<uint32_t>(A);
+  b.inter_codes = c.take<uint8_t>(A * static_cast<size_t>(I));
+  b.inter_scales = c.take<float>(A);
+  b.y = c.take<float>(A * static_cast<size_t>(H));
+  return b;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [outer, inner] with row pitch `inner` bytes.
+w4a8_status encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                         uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(W4A8_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(W4A8_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for [%llu x %llu]",
+                static_cast<int>(r), static_cast<unsigned long long>(outer),
+                static_cast<unsigned long long>(inner));
+  return W4A8_OK;
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t v = [] {
+    const char* s = std::getenv("W4A8_WAIT_TIMEOUT_MS");
+    uint64_t ms = s ? std::strtoull(s, nullptr, 10) : 0;
+    if (ms == 0) ms = 2000;
+    return ms * 1000000ull;
+  }();
+  return v;
+}
+
+w4a8_status check_route_args(const void* logits, int64_t T, int32_t E, int32_t k) {
+  if (T < 0) return fail(W4A8_ERR_INVALID_ARG, "T = %lld < 0", static_cast<long long>(T));
+  if (E < 1 || E > kMaxExperts)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "E = %d outside [1, %d]", E, kMaxExperts);
+  if (k < 1 || k > E || k > kMaxTopK)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "k = %d outside [1, min(E, %d)]", k, kMaxTopK);
+  if (T * static_cast<int64_t>(k) > INT32_MAX)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "T * k exceeds 2^31 - 1");
+  if (T > 0 && !logits) return fail(W4A8_ERR_INVALID_ARG, "logits is NULL");
+  if (!aligned16(logits)) return fail(W4A8_ERR_INVALID_ARG, "logits is not 16-byte aligned");
+  return W4A8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t w4a8_abi_version(void) { return 1; }
+
+const char* w4a8_status_string(w4a8_status s) {
+  switch (s) {
+    case W4A8_OK: return "W4A8_OK";
+    case W4A8_ERR_INVALID_ARG: return "W4A8_ERR_INVALID_ARG";
+    case W4A8_ERR_UNSUPPORTED_SHAPE: return "W4A8_ERR_UNSUPPORTED_SHAPE";
+    case W4A8_ERR_UNSUPPORTED_ARCH: return "W4A8_ERR_UNSUPPORTED_ARCH";
+    case W4A8_ERR_WORKSPACE_TOO_SMALL: return "W4A8_ERR_WORKSPACE_TOO_SMALL";
+    case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
+    case W4A8_ERR_DEVICE_TIMEOUT: return "W4A8_ERR_DEVICE_TIMEOUT";
+    default: return "W4A8_ERR_UNKNOWN";
+  }
+}
+
+const char* w4a8_last_error(void) { return g_last_error.c_str(); }
+
+w4a8_status w4a8_check_device_error(void* stream) {
+  cudaError_t err = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "cudaStreamSynchronize");
+  int v = 0;
+  err = read_and_clear_device_error(&v);
+  if (err != cudaSuccess) return cuda_fail(err, "reading the device error latch");
+  if (v != 0)
+    return fail(W4A8_ERR_DEVICE_TIMEOUT, "a bounded in-kernel wait ran out (latch 0x%x)", v);
+  return W4A8_OK;
+}
+
+w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, int32_t group,
+                           int32_t* packed, void* scales_bf16, void* stream) {
+  if (group != kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "group = %d; only 128", group);
+  if (R < 0 || K <= 0) return fail(W4A8_ERR_INVALID_ARG, "R = %lld, K = %lld",
+                                   static_cast<long long>(R), static_cast<long long>(K));
+  if (K % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "K = %lld is not a multiple of 128",
+                              static_cast<long long>(K));
+  if (R == 0) return W4A8_OK;
+  if (!w_bf16 || !packed || !scales_bf16) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(w_bf16) || !aligned16(packed) || !aligned16(scales_bf16))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_pack_int4(w_bf16, R, K, packed, scales_bf16, di.sms,
+                                     static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "pack_int4 launch");
+}
+
+w4a8_status w4a8_quant_act_fp8_per_token(const void* x_bf16, int64_t T, int64_t H,
+                                         uint8_t* codes_e4m3, float* scales, void* stream) {
+  if (T < 0 || H <= 0) return fail(W4A8_ERR_INVALID_ARG, "T = %lld, H = %lld",
+                                   static_cast<long long>(T), static_cast<long long>(H));
+  if (H % 16) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld is not a multiple of 16",
+                          static_cast<long long>(H));
+  if (T == 0) return W4A8_OK;
+  if (!x_bf16 || !codes_e4m3 || !scales) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(x_bf16) || !aligned16(codes_e4m3) || !aligned16(scales))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_act_quant(x_bf16, T, H, codes_e4m3, scales, di.sms,
+                                     static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "act_quant launch");
+}
+
+size_t w4a8_moe_route_workspace_size(int64_t T, int32_t E) {
+  if (T < 0 || E < 1) return 0;
+  Carver c(nullptr);
+  carve_route(c, T, E);
+  return c.off + 256;
+}
+
+w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int32_t E, int32_t k,
+                                   int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                   int32_t* sorted_token_ids, int32_t* row_of, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (w4a8_status st = check_route_args(logits, T, E, k)) return st;
+  if (!expert_offsets || !workspace)
+    return fail(W4A8_ERR_INVALID_ARG, "expert_offsets / workspace is NULL");
+  if (T > 0 && (!topk_ids || !topk_w || !sorted_token_ids || !row_of))
+    return fail(W4A8_ERR_INVALID_ARG, "NULL output pointer");
+  for (const void* p : {static_cast<const void*>(topk_ids), static_cast<const void*>(topk_w),
+                        static_cast<const void*>(expert_offsets),
+                        static_cast<const void*>(sorted_token_ids),
+                        static_cast<const void*>(row_of), static_cast<const void*>(workspace)})
+    if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = w4a8_moe_route_workspace_size(T, E);
+  if (workspace_bytes < need)
+    return fail(W4A8_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu", workspace_bytes, need);
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  Carver c(workspace);
+  RouteBufs rb = carve_route(c, T, E);
+  cudaError_t err = launch_route(logits, T, E, k, topk_ids, topk_w, expert_offsets,
+                                 sorted_token_ids, row_of, rb.block_counts, rb.block_base,
+                                 rb.tile_prefix, nullptr, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "route launch");
+}
+
+size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k) {
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1) return 0;
+  Carver c(nullptr);
+  carve_forward(c, T, H, I, E, k);
+  return c.off + 256;
+}
+
+w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
+                             const int32_t* w13_packed, const void* w13_scales,
+                             const int32_t* w2_packed, const void* w2_scales, int64_t T,
+                             int64_t H, int64_t I, int32_t E, int32_t k, void* out_bf16,
+                             void* workspace, size_t workspace_bytes, const w4a8_moe_aux* aux,
+                             void* stream) {
+  if (w4a8_status st = check_route_args(logits, T, E, k)) return st;
+  if (H <= 0 || I <= 0 || H % kGroup || I % kGroup)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld and I = %lld must be positive multiples of 128",
+                static_cast<long long>(H), static_cast<long long>(I));
+  if (static_cast<int64_t>(E) * 2 * I > INT32_MAX || static_cast<int64_t>(E) * H > INT32_MAX)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "E * rows exceeds 2^31 - 1");
+  if (T == 0) return W4A8_OK;
+  const void* ptrs[] = {hidden_bf16, w13_packed, w13_scales, w2_packed, w2_scales, out_bf16,
+                        workspace};
+  for (const void* p : ptrs) {
+    if (!p) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  const size_t need = w4a8_moe_workspace_size(T, H, I, E, k);
+  if (workspace_bytes < need)
+    return fail(W4A8_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu", workspace_bytes, need);
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  Carver c(workspace);
+  ForwardBufs b = carve_forward(c, T, H, I, E, k);
+  void* const* ev = nullptr;
+  if (aux) {
+    auto pick = [](auto* user, auto* ws) { return user ? user : ws; };
+    b.topk_ids = pick(aux->topk_ids, b.topk_ids);
+    b.topk_w = pick(aux->topk_w, b.topk_w);
+    b.expert_offsets = pick(aux->expert_offsets, b.expert_offsets);
+    b.sorted_token_ids = pick(aux->sorted_token_ids, b.sorted_token_ids);
+    b.row_of = pick(aux->row_of, b.row_of);
+    b.act_codes = pick(aux->act_codes, b.act_codes);
+    b.act_scales = pick(aux->act_scales, b.act_scales);
+    b.h = pick(aux->inter_h, b.h);
+    b.inter_codes = pick(aux->inter_codes, b.inter_codes);
+    b.inter_scales = pick(aux->inter_scales, b.inter_scales);
+    b.y = pick(aux->y_rows, b.y);
+    for (const void* p : {static_cast<const void*>(b.topk_ids), static_cast<const void*>(b.topk_w),
+                          static_cast<const void*>(b.expert_offsets),
+                          static_cast<const void*>(b.sorted_token_ids),
+                          static_cast<const void*>(b.row_of), static_cast<const void*>(b.act_codes),
+                          static_cast<const void*>(b.act_scales), static_cast<const void*>(b.h),
+                          static_cast<const void*>(b.inter_codes),
+                          static_cast<const void*>(b.inter_scales), static_cast<const void*>(b.y)})
+      if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "aux buffers must be 16-byte aligned");
+    ev = aux->stage_events;
+  }
+  const int64_t A = T * k;
+
+  // TMA descriptors: packed weights [E * rows, K / 2] bytes, 64-byte swizzle;
+  // activation codes [rows, K] bytes, 128-byte swizzle, one-row boxes for gather4.
+  CUtensorMap tw1, ta1, tw2, ta2;
+  if (w4a8_status st = encode_u8_2d(&tw1, w13_packed, static_cast<uint64_t>(H / 2),
+                                    static_cast<uint64_t>(E) * 2 * I, 64, 64,
+                                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ta1, b.act_codes, static_cast<uint64_t>(H),
+                                    static_cast<uint64_t>(T), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&tw2, w2_packed, static_cast<uint64_t>(I / 2),
+                                    static_cast<uint64_t>(E) * H, 64, 128,
+                                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ta2, b.inter_codes, static_cast<uint64_t>(I),
+                                    static_cast<uint64_t>(A), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+
+  auto record = [&](int i) -> cudaError_t {
+    return ev && ev[i] ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+  cudaError_t err = cudaSuccess;
+#define W4A8_STEP(call, what)                     \
+  do {                                            \
+    err = (call);                                 \
+    if (err != cudaSuccess) return cuda_fail(err, what); \
+  } while (0)
+
+  W4A8_STEP(record(0), "cudaEventRecord");
+  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, di.sms, s),
+            "act_quant launch");
+  W4A8_STEP(record(1), "cudaEventRecord");
+  W4A8_STEP(record(2), "cudaEventRecord");
+  W4A8_STEP(launch_route(logits, T, E, k, b.topk_ids, b.topk_w, b.expert_offsets,
+                         b.sorted_token_ids, b.row_of, b.route.block_counts, b.route.block_base,
+                         b.route.tile_prefix, b.row_amax, s),
+            "route launch");
+  W4A8_STEP(record(3), "cudaEventRecord");
+
+  GemmArgs g1{};
+  g1.K = static_cast<int>(H);
+  g1.n_rows = static_cast<int>(2 * I);
+  g1.half_rows = static_cast<int>(I);
+  g1.E = E;
+  g1.expert_offsets = b.expert_offsets;
+  g1.tile_prefix = b.route.tile_prefix;
+  g1.row_tokens = b.sorted_token_ids;
+  g1.act_scale = b.act_scales;
+  g1.wscale = w13_scales;
+  g1.out = b.h;
+  g1.out_ld = I;
+  g1.row_amax = b.row_amax;
+  g1.act_rows = T;
+  g1.timeout_ns = wait_timeout_ns();
+  W4A8_STEP(record(4), "cudaEventRecord");
+  W4A8_STEP(launch_grouped_gemm(true, tw1, ta1, g1, di.sms, s), "gate/up GEMM launch");
+  W4A8_STEP(record(5), "cudaEventRecord");
+
+  W4A8_STEP(record(6), "cudaEventRecord");
+  W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales, di.sms, s),
+            "intermediate quant launch");
+  W4A8_STEP(record(7), "cudaEventRecord");
+
+  GemmArgs g2{};
+  g2.K = static_cast<int>(I);
+  g2.n_rows = static_cast<int>(H);
+  g2.half_rows = 0;
+  g2.E = E;
+  g2.expert_offsets = b.expert_offsets;
+  g2.tile_prefix = b.route.tile_prefix;
+  g2.row_tokens = nullptr;
+  g2.act_scale = b.inter_scales;
+  g2.wscale = w2_scales;
+  g2.out = b.y;
+  g2.out_ld = H;
+  g2.row_amax = nullptr;
+  g2.act_rows = A;
+  g2.timeout_ns = wait_timeout_ns();
+  W4A8_STEP(record(8), "cudaEventRecord");
+  W4A8_STEP(launch_grouped_gemm(false, tw2, ta2, g2, di.sms, s), "down GEMM launch");
+  W4A8_STEP(record(9), "cudaEventRecord");
+
+  W4A8_STEP(record(10), "cudaEventRecord");
+  W4A8_STEP(launch_combine(b.y, b.row_of, b.topk_w, T, H, k, out_bf16, di.sms, s),
+            "combine launch");
+  W4A8_STEP(record(11), "cudaEventRecord");
+#undef W4A8_STEP
+  return W4A8_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,454 @@
+// grouped_gemm.cu - W4A8 grouped GEMM on the sm_100a tensor cores.
+//
+// One persistent kernel runs either projection of every expert:
+//   gate/up: G[r, n] = a_s[t_r] * sum_g s13[e, n, g] * P_g(r, n),  n < 2I
+//            then h = silu(G[:, :I]) * G[:, I:] and the row absmax of h;
+//   down:    Y[r, n] = h_s[r]   * sum_g s2[e, n, g]  * P_g(r, n),  n < H
+// with P_g the exact E4M3 x INT4 dot product over the 128-wide K group g
+// (GLM-5.3-W4A8 model card, intro and "quantisation method": INT4 group-128
+// experts, INT4 turned into FP8 inside the kernel, no BF16 dequantisation).
+//
+// Tile = 128 weight rows (the MMA M side, TMEM lanes) x up to 128 segment
+// rows of one expert (the MMA N side).  For gate/up the 128 weight rows are
+// 64 gate rows and the 64 matching up rows, so SwiGLU finishes inside the
+// tile.  Per 128-wide K group:
+//   warp 8 (TMA)      packed INT4 box [128 rows x 64 B] (64-byte swizzle) and
+//                     the activation codes [n rows x 128 B] (128-byte swizzle,
+//                     rows gathered four at a time) into a 6-stage ring;
+//   warps 0-3 (cvt)   each thread owns one weight row: 64 B of nibbles ->
+//                     128 E4M3 bytes with byte permutes, stored straight into
+//                     a TMEM A slot (tcgen05.st), 4 slots;
+//   warp 9 (MMA)      4 x tcgen05.mma kind::f8f6f4 (K = 32 each), A from
+//                     TMEM, B from shared memory, into one of two TMEM
+//                     accumulators (FP32, fresh per group);
+//   warps 4-7 (epi)   tcgen05.ld the group's partial sums, multiply by the
+//                     row's group scale and add into FP32 registers.
+// After the last group the epilogue applies the token (or row) scale and
+// writes h (plus the SwiGLU and absmax) or Y.
+//
+// Every wait is bounded (see ptx.cuh); a timed-out CTA drains its own
+// in-flight copies and MMAs, frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace w4a8 {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kThreads = 320;  // warps 0-3 convert, 4-7 epilogue, 8 TMA, 9 MMA
+constexpr int kStages = 6;
+constexpr int kASlots = 4;
+constexpr int kBM = 128;
+constexpr int kWStageBytes = kBM * kGroup / 2;  // 8 KB of packed INT4
+constexpr int kBStageBytes = kTileN * kGroup;   // 16 KB of E4M3 codes
+constexpr int kUpBytes = 64 * kTileN * 4;       // up-projection exchange for SwiGLU
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemA = 0;    // A slots: 32 columns (128 E4M3 per lane) each
+constexpr uint32_t kTmemD = 128;  // two accumulators of kTileN columns
+constexpr int kNumBars = 2 * kStages + 2 * kASlots + 4 + 3;
+
+static_assert(kTmemA + kASlots * 32 <= kTmemD, "TMEM A slots overlap the accumulators");
+static_assert(kTmemD + 2 * kTileN <= kTmemCols, "TMEM accumulators exceed the allocation");
+
+__host__ __device__ constexpr int smem_bytes(bool gate_up) {
+  return 1024 /* alignment slack */ + kStages * (kWStageBytes + kBStageBytes) +
+         (gate_up ? kUpBytes : 0) + kNumBars * 8 + 16;
+}
+
+struct Tile {
+  int e, mb, n_valid, n_mma;
+  int64_t row0;
+};
+
+// Linear tile index -> (expert, weight-row block, segment rows).  Tiles are
+// ordered by global token block, then weight-row block, so CTAs running at
+// the same time share one activation block through L2.
+__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, int mb_count, int idx) {
+  const int nbg = idx / mb_count;
+  Tile t;
+  t.mb = idx - nbg * mb_count;
+  int lo = 0, hi = a.E;  // tile_prefix[lo] <= nbg < tile_prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a.tile_prefix + mid) <= nbg) lo = mid;
+    else hi = mid;
+  }
+  t.e = lo;
+  const int nb = nbg - __ldg(a.tile_prefix + lo);
+  const int seg0 = __ldg(a.expert_offsets + lo);
+  const int cnt = __ldg(a.expert_offsets + lo + 1) - seg0;
+  t.row0 = static_cast<int64_t>(seg0) + static_cast<int64_t>(nb) * kTileN;
+  t.n_valid = min(kTileN, cnt - nb * kTileN);
+  t.n_mma = (t.n_valid + 15) & ~15;
+  return t;
+}
+
+// Eight uint4b8 nibbles (value q + 8, little-endian) -> eight E4M3 bytes of q.
+// Low three bits index an 8-entry table of q >= 0 (nibbles 8..15) and one of
+// q < 0 (nibbles 0..7); bit 3 picks the table per byte.
+__device__ __forceinline__ void cvt8_uint4b8_e4m3(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  constexpr uint32_t kPosLo = 0x44403800u;  // E4M3 of 0, 1, 2, 3
+  constexpr uint32_t kPosHi = 0x4E4C4A48u;  // 4, 5, 6, 7
+  constexpr uint32_t kNegLo = 0xCACCCED0u;  // -8, -7, -6, -5
+  constexpr uint32_t kNegHi = 0xB8C0C4C8u;  // -4, -3, -2, -1
+  const uint32_t idx = w & 0x77777777u;
+  const uint32_t sel = ((w >> 1) & 0x44444444u) | 0x32103210u;
+  const uint32_t idx_hi = idx >> 16, sel_hi = sel >> 16;
+  lo = prmt(prmt(kNegLo, kNegHi, idx), prmt(kPosLo, kPosHi, idx), sel);
+  hi = prmt(prmt(kNegLo, kNegHi, idx_hi), prmt(kPosLo, kPosHi, idx_hi), sel_hi);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+// Wait used only while draining: ignores the abort flag, still bounded.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      atomicOr(&g_device_error, 1);
+      return;
+    }
+  }
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                        const __grid_constant__ CUtensorMap tmap_act, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sW = smem;
+  uint8_t* sB = sW + kStages * kWStageBytes;
+  float* sU = reinterpret_cast<float*>(sB + kStages * kBStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBStageBytes +
+                                               (kGateUp ? kUpBytes : 0));
+  uint64_t* full = bars;                 // [kStages]  TMA bytes landed
+  uint64_t* empty = full + kStages;      // [kStages]  4 converter warps + MMA done
+  uint64_t* afull = empty + kStages;     // [kASlots]  converted A in TMEM
+  uint64_t* aempty = afull + kASlots;    // [kASlots]  MMAs reading the slot done
+  uint64_t* dfull = aempty + kASlots;    // [2]        group partial sums ready
+  uint64_t* dempty = dfull + 2;          // [2]        epilogue read them
+  uint64_t* upfull = dempty + 2;         // up rows staged in sU
+  uint64_t* upempty = upfull + 1;        // sU consumed
+  uint64_t* drain = upempty + 1;         // all MMAs of this CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = a.K / kGroup;
+  const int mb_count = kGateUp ? a.half_rows / 64 : a.n_rows / kBM;
+  const uint64_t tmo = a.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 5);
+    }
+    for (int s = 0; s < kASlots; ++s) {
+      mbar_init(&afull[s], 4);
+      mbar_init(&aempty[s], 1);
+    }
+    for (int d = 0; d < 2; ++d) {
+      mbar_init(&dfull[d], 1);
+      mbar_init(&dempty[d], 4);
+    }
+    mbar_init(upfull, 2);
+    mbar_init(upempty, 2);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_act);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = __ldg(a.tile_prefix + a.E) * mb_count;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      const Tile t = decode_tile(a, mb_count, tile);
+      int32_t ry[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t r = t.row0 + min(4 * lane + q, t.n_valid - 1);
+        ry[q] = kGateUp ? __ldg(a.row_tokens + r) : static_cast<int32_t>(r);
+      }
+      const int n_ops = t.n_mma >> 2;
+      const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
+      const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
+      const uint32_t tx = kWStageBytes + t.n_mma * kGroup;
+      for (int g = 0; g < G; ++g) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
+        const uint32_t dW = smem_u32(sW + s * kWStageBytes);
+        const uint32_t dB = smem_u32(sB + s * kBStageBytes);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], tx);
+          if (kGateUp) {
+            tma_load_2d(dW, &tmap_w, &full[s], g * 64, wy0);
+            tma_load_2d(dW + kWStageBytes / 2, &tmap_w, &full[s], g * 64, wy1);
+          } else {
+            tma_load_2d(dW, &tmap_w, &full[s], g * 64, wy0);
+          }
+        }
+        __syncwarp();
+        if (lane < n_ops)
+          tma_gather4(dB + lane * 4 * kGroup, &tmap_act, &full[s], g * kGroup, ry[0], ry[1], ry[2],
+                      ry[3]);
+        ++it;
+      }
+    }
+    // The latest fill of every stage must have landed before the CTA exits.
+    for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
+      mbar_wait_drain(&full[i % kStages], (i / kStages) & 1, tmo);
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const Tile t = decode_tile(a, mb_count, tile);
+        const uint32_t idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
+        for (int g = 0; g < G; ++g) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          const int as = it % kASlots;
+          const uint32_t pha = (it / kASlots) & 1;
+          const int d = it & 1;
+          const uint32_t phd = (it >> 1) & 1;
+          if (!mbar_wait(&dempty[d], phd ^ 1, abort_flag, tmo) ||
+              !mbar_wait(&full[s], ph, abort_flag, tmo) ||
+              !mbar_wait(&afull[as], pha, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * kBStageBytes));
+          const uint32_t dt = tmem + kTmemD + d * kTileN;
+          const uint32_t at = tmem + kTmemA + as * 32;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // K = 32 E4M3 per MMA: 8 TMEM columns, 32 B of smem
+            mma_f8_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                      kk > 0 ? 1u : 0u);
+          tc_commit(&dfull[d]);
+          tc_commit(&aempty[as]);
+          tc_commit(&empty[s]);
+          ++it;
+        }
+      }
+      tc_commit(drain);
+      mbar_wait_drain(drain, 0, tmo);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ INT4 -> E4M3 converters
+    const int m = warp * 32 + lane;                 // weight row of the tile = TMEM lane
+    const uint32_t swz = (m >> 1) & 3;              // 64-byte swizzle of the TMA box
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+      for (int g = 0; g < G; ++g) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const int as = it % kASlots;
+        const uint32_t pha = (it / kASlots) & 1;
+        if (!mbar_wait(&full[s], ph, abort_flag, tmo) ||
+            !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t row = smem_u32(sW + s * kWStageBytes) + m * 64;
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = ld_shared_v4(row + ((c ^ swz) << 4));
+          cvt8_uint4b8_e4m3(v.x, r[8 * c + 0], r[8 * c + 1]);
+          cvt8_uint4b8_e4m3(v.y, r[8 * c + 2], r[8 * c + 3]);
+          cvt8_uint4b8_e4m3(v.z, r[8 * c + 4], r[8 * c + 5]);
+          cvt8_uint4b8_e4m3(v.w, r[8 * c + 6], r[8 * c + 7]);
+        }
+        tmem_st_32x32b_x32(tmem + lane_base + kTmemA + as * 32, r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&afull[as]);
+          mbar_arrive(&empty[s]);
+        }
+        ++it;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                         // TMEM lane quadrant
+    const int m = q * 32 + lane;                    // weight row of the tile
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const __nv_bfloat16* wscale = static_cast<const __nv_bfloat16*>(a.wscale);
+    int it = 0, ntile = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++ntile) {
+      const Tile t = decode_tile(a, mb_count, tile);
+      const int wrow = kGateUp ? (m < 64 ? t.mb * 64 + m : a.half_rows + t.mb * 64 + (m - 64))
+                               : t.mb * kBM + m;
+      const __nv_bfloat16* srow =
+          wscale + (static_cast<int64_t>(t.e) * a.n_rows + wrow) * static_cast<int64_t>(G);
+      float ts[kTileN / 32];  // token (gate/up) or row (down) scales, lane-strided
+#pragma unroll
+      for (int i = 0; i < kTileN / 32; ++i) {
+        const int j = lane + 32 * i;
+        float v = 0.0f;
+        if (j < t.n_valid) {
+          const int64_t r = t.row0 + j;
+          v = kGateUp ? __ldg(a.act_scale + __ldg(a.row_tokens + r)) : __ldg(a.act_scale + r);
+        }
+        ts[i] = v;
+      }
+      float acc[kTileN];
+#pragma unroll
+      for (int j = 0; j < kTileN; ++j) acc[j] = 0.0f;
+      float s_next = __bfloat162float(srow[0]);
+      for (int g = 0; g < G; ++g) {
+        const float sg = s_next;
+        if (g + 1 < G) s_next = __bfloat162float(srow[g + 1]);
+        const int d = it & 1;
+        const uint32_t phd = (it >> 1) & 1;
+        if (!mbar_wait(&dfull[d], phd, abort_flag, tmo)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem + lane_base + kTmemD + d * kTileN;
+#pragma unroll
+        for (int c = 0; c < kTileN / 32; ++c) {
+          if (c * 32 < t.n_mma) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              acc[c * 32 + i] = fmaf(sg, __uint_as_float(v[i]), acc[c * 32 + i]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dempty[d]);
+        ++it;
+      }
+      if (!ok) break;
+
+      if constexpr (kGateUp) {
+        const uint32_t phu = ntile & 1;
+        if (q >= 2) {  // up rows: stage u = acc * token scale for the gate warps
+          if (!mbar_wait(upempty, phu ^ 1, abort_flag, tmo)) break;
+#pragma unroll
+          for (int j = 0; j < kTileN; ++j) {
+            if (j < t.n_valid) {
+              const float tsj = __shfl_sync(kFull, ts[j >> 5], j & 31);
+              sU[j * 64 + (m - 64)] = acc[j] * tsj;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(upfull);
+        } else {  // gate rows: h = silu(gate) * up, store, row absmax
+          if (!mbar_wait(upfull, phu, abort_flag, tmo)) break;
+#pragma unroll
+          for (int j = 0; j < kTileN; ++j) {
+            if (j < t.n_valid) {
+              const float tsj = __shfl_sync(kFull, ts[j >> 5], j & 31);
+              const float gt = acc[j] * tsj;
+              const float u = sU[j * 64 + m];
+              const float h = __fdiv_rn(gt, 1.0f + expf(-gt)) * u;
+              const int64_t r = t.row0 + j;
+              a.out[r * a.out_ld + t.mb * 64 + m] = h;
+              const float hm = warp_max(fabsf(h));
+              if (lane == 0) atomicMax(a.row_amax + r, __float_as_uint(hm));
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(upempty);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kTileN; ++j) {
+          if (j < t.n_valid) {
+            const float tsj = __shfl_sync(kFull, ts[j >> 5], j & 31);
+            a.out[(t.row0 + j) * a.out_ld + t.mb * kBM + m] = acc[j] * tsj;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+bool g_attr_set[2][64] = {};
+
+}  // namespace
+
+size_t grouped_gemm_smem_bytes(bool gate_up) { return static_cast<size_t>(smem_bytes(gate_up)); }
+
+cudaError_t launch_grouped_gemm(bool gate_up, const CUtensorMap& tmap_w,
+                                const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
+                                cudaStream_t s) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const int smem = smem_bytes(gate_up);
+  if (dev < 64 && !g_attr_set[gate_up][dev]) {
+    err = gate_up ? cudaFuncSetAttribute(grouped_gemm_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                  : cudaFuncSetAttribute(grouped_gemm_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    g_attr_set[gate_up][dev] = true;
+  }
+  if (gate_up)
+    grouped_gemm_kernel<true><<<num_ctas, kThreads, smem, s>>>(tmap_w, tmap_act, a);
+  else
+    grouped_gemm_kernel<false><<<num_ctas, kThreads, smem, s>>>(tmap_w, tmap_act, a);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(int* value) {
+  int v = 0;
+  cudaError_t err = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (err != cudaSuccess) return err;
+  *value = v;
+  if (v != 0) {
+    const int zero = 0;
+    err = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  }
+  return err;
+}
+
+}  // namespace w4a8

@@ -1,0 +1,56 @@
+// internal.h - launchers shared between the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda.h>
+
+namespace w4a8 {
+
+constexpr int kGroup = 128;        // INT4 group size along K
+constexpr int kRouteTok = 256;     // tokens per routing block
+constexpr int kTileN = 128;        // max tokens per grouped-GEMM tile
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+
+inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok; }
+
+// ---- kernels_small.cu
+cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
+                             int num_sms, cudaStream_t s);
+cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
+                             int num_sms, cudaStream_t s);
+// routing: top-k + per-block expert histogram; scan; stable scatter.
+cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
+                         float* topk_w, int32_t* expert_offsets, int32_t* sorted_token_ids,
+                         int32_t* row_of, int32_t* block_counts, int32_t* block_base,
+                         int32_t* tile_prefix, uint32_t* row_amax_to_zero, cudaStream_t s);
+cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
+                               uint8_t* codes, float* scales, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
+                           int64_t H, int k, void* out, int num_sms, cudaStream_t s);
+
+// ---- grouped_gemm.cu
+struct GemmArgs {
+  int K;                          // reduction length (H for gate/up, I for down)
+  int n_rows;                     // weight rows per expert (2I or H)
+  int half_rows;                  // gate/up: I (first up row); down: 0
+  int E;
+  const int32_t* expert_offsets;  // [E + 1]
+  const int32_t* tile_prefix;     // [E + 1] prefix of ceil(count / kTileN)
+  const int32_t* row_tokens;      // gate/up: sorted_token_ids (gather rows); down: nullptr
+  const float* act_scale;         // gate/up: per token [T]; down: per segment row [A]
+  const void* wscale;             // bf16 [E, n_rows, K / 128]
+  float* out;                     // gate/up: h [A, I]; down: Y [A, H]
+  int64_t out_ld;
+  uint32_t* row_amax;             // gate/up only: float bits of max |h| per segment row
+  int64_t act_rows;               // rows of the activation tensor (T or A)
+  uint64_t timeout_ns;
+};
+cudaError_t launch_grouped_gemm(bool gate_up, const CUtensorMap& tmap_w,
+                                const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
+                                cudaStream_t s);
+size_t grouped_gemm_smem_bytes(bool gate_up);
+
+}  // namespace w4a8

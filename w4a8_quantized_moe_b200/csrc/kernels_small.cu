@@ -1,0 +1,475 @@
+// kernels_small.cu - the HBM-bound and latency-bound steps of the layer:
+// per-token FP8 activation quantisation, INT4 RTN packing, top-k routing and
+// the expert permutation, the intermediate requantisation, the combine.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace w4a8 {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ float absmax8(uint4 c) {
+  float m = fmaxf(fabsf(bf16_lo(c.x)), fabsf(bf16_hi(c.x)));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(c.y)), fabsf(bf16_hi(c.y))));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(c.z)), fabsf(bf16_hi(c.z))));
+  m = fmaxf(m, fmaxf(fabsf(bf16_lo(c.w)), fabsf(bf16_hi(c.w))));
+  return m;
+}
+
+// Two floats -> two E4M3 codes (first in the low byte), nearest-even, saturating.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Eight values / scale -> eight E4M3 codes (little-endian in a uint2).
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float scale) {
+  if (scale == 0.0f) return make_uint2(0u, 0u);
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    c[i] = e4m3x2(__fdiv_rn(v[2 * i], scale), __fdiv_rn(v[2 * i + 1], scale));
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__device__ __forceinline__ void unpack8(uint4 c, float (&v)[8]) {
+  v[0] = bf16_lo(c.x); v[1] = bf16_hi(c.x); v[2] = bf16_lo(c.y); v[3] = bf16_hi(c.y);
+  v[4] = bf16_lo(c.z); v[5] = bf16_hi(c.z); v[6] = bf16_lo(c.w); v[7] = bf16_hi(c.w);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------- activation quant
+// One CTA per token row (grid-stride): absmax over the row, scale = absmax/448,
+// codes = E4M3(x / scale).  Up to kAqCache 16-byte chunks per thread stay in
+// registers between the two passes; longer rows are re-read (L1/L2 hits).
+constexpr int kAqThreads = 256;
+constexpr int kAqCache = 4;
+
+__global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat16* __restrict__ x,
+                                                               int64_t T, int64_t H,
+                                                               uint8_t* __restrict__ codes,
+                                                               float* __restrict__ scales) {
+  __shared__ float red[kAqThreads / 32];
+  const int64_t nchunk = H / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
+    uint4 cache[kAqCache];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kAqCache; ++i) {
+      const int64_t c = threadIdx.x + static_cast<int64_t>(i) * kAqThreads;
+      if (c < nchunk) {
+        cache[i] = __ldg(row + c);
+        amax = fmaxf(amax, absmax8(cache[i]));
+      }
+    }
+    for (int64_t c = threadIdx.x + static_cast<int64_t>(kAqCache) * kAqThreads; c < nchunk;
+         c += kAqThreads)
+      amax = fmaxf(amax, absmax8(__ldg(row + c)));
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < kAqThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+    const float scale = __fdiv_rn(amax, 448.0f);
+    if (threadIdx.x == 0) scales[t] = scale;
+    uint2* out = reinterpret_cast<uint2*>(codes + t * H);
+#pragma unroll
+    for (int i = 0; i < kAqCache; ++i) {
+      const int64_t c = threadIdx.x + static_cast<int64_t>(i) * kAqThreads;
+      if (c < nchunk) {
+        float v[8];
+        unpack8(cache[i], v);
+        out[c] = quant8(v, scale);
+      }
+    }
+    for (int64_t c = threadIdx.x + static_cast<int64_t>(kAqCache) * kAqThreads; c < nchunk;
+         c += kAqThreads) {
+      float v[8];
+      unpack8(__ldg(row + c), v);
+      out[c] = quant8(v, scale);
+    }
+    __syncthreads();  // red[] is reused by the next row
+  }
+}
+
+// ---------------------------------------------------------------- INT4 pack
+// One warp per group of 128 weights (grid-stride).  Lane l holds elements
+// 4l..4l+3; the group scale is bf16(absmax / 7); q = clamp(rint(w / s), -8, 7);
+// lanes 2i and 2i+1 form word i (nibbles little-endian along K).
+__global__ void __launch_bounds__(256) pack_int4_kernel(const __nv_bfloat16* __restrict__ w,
+                                                        int64_t R, int64_t K,
+                                                        int32_t* __restrict__ packed,
+                                                        __nv_bfloat16* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t groups_per_row = K / kGroup;
+  const int64_t ngroups = R * groups_per_row;
+  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t g = warp_global; g < ngroups; g += nwarps) {
+    const int64_t r = g / groups_per_row, gi = g - r * groups_per_row;
+    const __nv_bfloat16* src = w + r * K + gi * kGroup + lane * 4;
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
+    float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    amax = warp_max(amax);
+    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
+    const float s = __bfloat162float(sb);
+    uint32_t nib = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int q = 0;
+      if (s != 0.0f) q = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -8.0f), 7.0f));
+      nib |= static_cast<uint32_t>(q + 8) << (4 * i);
+    }
+    const uint32_t hi = __shfl_down_sync(kFull, nib, 1);
+    if ((lane & 1) == 0)
+      packed[r * (K / 8) + gi * (kGroup / 8) + (lane >> 1)] = static_cast<int32_t>(nib | (hi << 16));
+    if (lane == 0) scales[r * groups_per_row + gi] = sb;
+  }
+}
+
+// ---------------------------------------------------------------- routing
+// Top-k per token: each warp takes 32 consecutive tokens of the block, one at
+// a time; lane l holds the logits of experts l, l+32, ...  k rounds of a warp
+// arg-max under the order (larger logit, then lower id).  Weights: softmax of
+// the selected logits in float32.  Also counts the block's tokens per expert.
+template <int NV>  // logits per lane (E <= 32 * NV)
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int64_t T,
+                                                         int E, int k, int32_t* __restrict__ topk_ids,
+                                                         float* __restrict__ topk_w,
+                                                         int32_t* __restrict__ block_counts) {
+  __shared__ int cnt[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * kRouteTok + warp * 32;
+  for (int i = 0; i < 32; ++i) {
+    const int64_t t = t_begin + i;
+    if (t >= T) break;
+    const float* lt = logits + t * E;
+    float v[NV];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int e = lane + 32 * q;
+      if (e < E) v[q] = __ldg(lt + e);
+      else { v[q] = -INFINITY; taken |= 1u << q; }
+    }
+    float myv = 0.0f, v0 = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = INT_MAX;
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        const int e = lane + 32 * q;
+        if (!((taken >> q) & 1u) && (v[q] > bv || (v[q] == bv && e < bi))) { bv = v[q]; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(kFull, bv, o);
+        const int oi = __shfl_xor_sync(kFull, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == j) myv = bv;
+      if (j == 0) v0 = bv;
+      if (lane == 0) {
+        topk_ids[t * k + j] = bi;
+        atomicAdd(&cnt[bi], 1);
+      }
+    }
+    const float ex = (lane < k) ? expf(myv - v0) : 0.0f;
+    const float sum = warp_sum(ex);
+    if (lane < k) topk_w[t * k + lane] = __fdiv_rn(ex, sum);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = cnt[e];
+}
+
+// Exclusive scan over the experts (one CTA of 1024 threads, thread = expert):
+// per-block bases within each expert, expert offsets, GEMM tile prefix.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* sh /*[32]*/, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = (lane < static_cast<int>(blockDim.x >> 5)) ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, s, o);
+      if (lane >= o) s += y;
+    }
+    sh[lane] = s;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? sh[warp - 1] : 0);
+  *total = sh[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return excl;
+}
+
+__global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ block_counts,
+                                                          int64_t nblk, int E,
+                                                          int32_t* __restrict__ block_base,
+                                                          int32_t* __restrict__ expert_offsets,
+                                                          int32_t* __restrict__ tile_prefix) {
+  __shared__ int sh[32];
+  const int e = threadIdx.x;
+  int running = 0;
+  if (e < E) {
+    int64_t b = 0;
+    for (; b + 8 <= nblk; b += 8) {
+      int c[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) c[u] = __ldg(block_counts + (b + u) * E + e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { block_base[(b + u) * E + e] = running; running += c[u]; }
+    }
+    for (; b < nblk; ++b) {
+      const int c = __ldg(block_counts + b * E + e);
+      block_base[b * E + e] = running;
+      running += c;
+    }
+  }
+  int total = 0, total_tiles = 0;
+  const int off = block_exclusive_scan(e < E ? running : 0, sh, &total);
+  const int tiles = (e < E) ? (running + kTileN - 1) / kTileN : 0;
+  const int toff = block_exclusive_scan(tiles, sh, &total_tiles);
+  if (e < E) {
+    expert_offsets[e] = off;
+    tile_prefix[e] = toff;
+    for (int64_t b = 0; b < nblk; ++b) block_base[b * E + e] += off;
+  }
+  if (e == 0) {
+    expert_offsets[E] = total;
+    tile_prefix[E] = total_tiles;
+  }
+}
+
+// Stable scatter: one warp per routing block walks its 256 tokens in chunks
+// of 32 (lane = token).  A per-expert bitmask of the chunk's tokens gives the
+// rank of a token among earlier tokens of the chunk; a per-expert running
+// count carries the rank across chunks.
+__global__ void __launch_bounds__(32) route_scatter_kernel(const int32_t* __restrict__ topk_ids,
+                                                           int64_t T, int E, int k,
+                                                           const int32_t* __restrict__ block_base,
+                                                           int32_t* __restrict__ sorted_token_ids,
+                                                           int32_t* __restrict__ row_of,
+                                                           uint32_t* __restrict__ row_amax) {
+  __shared__ uint32_t mask[kMaxExperts];
+  __shared__ int running[kMaxExperts];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) { mask[e] = 0u; running[e] = 0; }
+  __syncwarp();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTok;
+  const int32_t* base = block_base + static_cast<int64_t>(blockIdx.x) * E;
+  for (int c = 0; c < kRouteTok / 32; ++c) {
+    const int64_t t = t0 + c * 32 + lane;
+    const bool valid = t < T;
+    int ids[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) ids[j] = (valid && j < k) ? __ldg(topk_ids + t * k + j) : 0;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (valid && j < k) atomicOr(&mask[ids[j]], 1u << lane);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (valid && j < k) {
+        const uint32_t m = mask[ids[j]];
+        const int row = base[ids[j]] + running[ids[j]] + __popc(m & lt_mask);
+        row_of[t * k + j] = row;
+        sorted_token_ids[row] = static_cast<int32_t>(t);
+        if (row_amax) row_amax[row] = 0u;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (valid && j < k) {
+        const uint32_t m = mask[ids[j]];
+        if ((m & lt_mask) == 0u) running[ids[j]] += __popc(m);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (valid && j < k) mask[ids[j]] = 0u;
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------- intermediate requant
+// 16 consecutive values of one segment row per thread: scale = amax_r / 448,
+// codes = E4M3(h / scale).
+__global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restrict__ h,
+                                                          const uint32_t* __restrict__ row_amax,
+                                                          int64_t A, int64_t I,
+                                                          uint8_t* __restrict__ codes,
+                                                          float* __restrict__ scales) {
+  const int64_t per_row = I / 16;
+  const int64_t n = A * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / per_row, c = i - r * per_row;
+    const float amax = __uint_as_float(__ldg(row_amax + r));
+    const float scale = __fdiv_rn(amax, 448.0f);
+    if (c == 0) scales[r] = scale;
+    const float4* src = reinterpret_cast<const float4*>(h + r * I + c * 16);
+    uint2 out[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const float4 a = __ldg(src + 2 * half), b = __ldg(src + 2 * half + 1);
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      out[half] = quant8(v, scale);
+    }
+    *reinterpret_cast<uint4*>(codes + r * I + c * 16) =
+        make_uint4(out[0].x, out[0].y, out[1].x, out[1].y);
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// out[t, c..c+7] = bf16(sum_j w[t, j] * Y[row_of[t, j], c..c+7]) in slot order.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y,
+                                                      const int32_t* __restrict__ row_of,
+                                                      const float* __restrict__ topk_w, int64_t T,
+                                                      int64_t H, int k,
+                                                      __nv_bfloat16* __restrict__ out) {
+  const int64_t per_row = H / 8;
+  const int64_t n = T * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / per_row, c = i - t * per_row;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int64_t r = __ldg(row_of + t * k + j);
+      const float wj = __ldg(topk_w + t * k + j);
+      const float4* src = reinterpret_cast<const float4*>(y + r * H + c * 8);
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      acc[0] = fmaf(wj, a.x, acc[0]); acc[1] = fmaf(wj, a.y, acc[1]);
+      acc[2] = fmaf(wj, a.z, acc[2]); acc[3] = fmaf(wj, a.w, acc[3]);
+      acc[4] = fmaf(wj, b.x, acc[4]); acc[5] = fmaf(wj, b.y, acc[5]);
+      acc[6] = fmaf(wj, b.z, acc[6]); acc[7] = fmaf(wj, b.w, acc[7]);
+    }
+    uint32_t p[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+      p[q] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(out + t * H + c * 8) = make_uint4(p[0], p[1], p[2], p[3]);
+  }
+}
+
+inline int grid_for(int64_t work_items, int threads, int num_sms, int per_sm = 8) {
+  int64_t g = (work_items + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
+  if (g > cap) g = cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
+                             int num_sms, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  const int grid = static_cast<int>(T < cap ? T : cap);
+  act_quant_kernel<<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, codes,
+                                               scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
+                             int num_sms, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  const int64_t ngroups = R * (K / kGroup);
+  const int grid = grid_for(ngroups * 32, 256, num_sms, 16);
+  pack_int4_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), R, K, packed,
+                                        static_cast<__nv_bfloat16*>(scales));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
+                         float* topk_w, int32_t* expert_offsets, int32_t* sorted_token_ids,
+                         int32_t* row_of, int32_t* block_counts, int32_t* block_base,
+                         int32_t* tile_prefix, uint32_t* row_amax_to_zero, cudaStream_t s) {
+  const int64_t nblk = route_blocks(T);
+  if (nblk > 0) {
+    const int nv = (E + 31) / 32;
+    if (nv <= 1)
+      route_topk_kernel<1><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    else if (nv <= 2)
+      route_topk_kernel<2><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    else if (nv <= 4)
+      route_topk_kernel<4><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    else if (nv <= 8)
+      route_topk_kernel<8><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    else if (nv <= 16)
+      route_topk_kernel<16><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    else
+      route_topk_kernel<32><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, block_base, expert_offsets,
+                                       tile_prefix);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || nblk == 0) return err;
+  route_scatter_kernel<<<nblk, 32, 0, s>>>(topk_ids, T, E, k, block_base, sorted_token_ids, row_of,
+                                           row_amax_to_zero);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
+                               uint8_t* codes, float* scales, int num_sms, cudaStream_t s) {
+  if (A == 0) return cudaSuccess;
+  const int grid = grid_for(A * (I / 16), 256, num_sms);
+  inter_quant_kernel<<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
+                           int64_t H, int k, void* out, int num_sms, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int grid = grid_for(T * (H / 8), 256, num_sms);
+  combine_kernel<<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k,
+                                      static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace w4a8
