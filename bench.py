@@ -204,11 +204,17 @@ def main():
                     help="tokens in the oracle sample of cpu_baseline (0: skip)")
     ap.add_argument("--ref-tokens", type=int, default=1,
                     help="tokens per step of the --impl reference arm")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="run the workload with this many experts instead (a smaller case for "
+                         "profiler captures; recorded in config)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     cfg = workloads.config_by_name(args.config)
+    if args.experts:
+        cfg = cfg.with_(name=f"{cfg.name}_E{args.experts}", E=args.experts,
+                        forced_empty=min(cfg.forced_empty, args.experts // 16))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

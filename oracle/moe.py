@@ -108,14 +108,15 @@ def _silu(x):
 
 
 def moe_forward(hidden, logits, experts: Sequence, k: int,
-                tokens: Optional[np.ndarray] = None):
+                tokens: Optional[np.ndarray] = None, hidden_of_tokens=None):
     """The whole layer for all tokens, or for the token subset ``tokens``.
 
     ``hidden``: float64 [T, H] (bf16 values); ``logits``: float32 [T, E];
     ``experts[e]`` = ``(w13_packed, s13, w2_packed, s2)``.  Routing and the
     permutation always cover all T tokens (they are cheap); the expert GEMMs
     and the combine run only for the assignments of ``tokens`` (all tokens by
-    default).
+    default).  ``hidden`` may be None when ``hidden_of_tokens`` (float64
+    [len(tokens), H], the rows of ``tokens``) is given instead.
 
     Returns a dict with ``topk_ids``, ``topk_w``, ``expert_offsets``,
     ``sorted_token_ids``, ``row_of``, ``act_codes`` / ``act_scales`` (rows of
@@ -123,15 +124,19 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
     (keyed by segment row, for the rows computed), ``out`` float64
     [len(tokens), H] bf16 values and ``tokens``.
     """
-    hidden = np.asarray(hidden, dtype=np.float64)
-    T, H = hidden.shape
-    E = logits.shape[1]
+    T, E = logits.shape
+    if hidden_of_tokens is None:
+        hidden = np.asarray(hidden, dtype=np.float64)
+
     ids, w = route_topk(logits, k)
     offsets, sorted_tok, row_of = permute_by_expert(ids, E)
     tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     pos = {int(t): i for i, t in enumerate(tokens)}
+    x_rows = hidden[tokens] if hidden_of_tokens is None else np.asarray(hidden_of_tokens,
+                                                                         dtype=np.float64)
+    H = x_rows.shape[1]
 
-    codes, a_scale = quant_act_fp8_per_token(hidden[tokens])
+    codes, a_scale = quant_act_fp8_per_token(x_rows)
     x_deq = a_scale[:, None] * e4m3_decode(codes)          # exact: 24-bit x 4-bit significands
 
     need_rows = np.sort(row_of[tokens].reshape(-1))
