@@ -242,6 +242,11 @@ def main():
     stream = torch.cuda.current_stream(device)
 
     def step(events=None):
+        if events:
+            # torch only reports elapsed time for events it recorded itself; the
+            # library re-records each one at its stage boundary later in the stream
+            for e in events:
+                e.record(stream)
         layer(hidden, logits, out=out, aux={"expert_offsets": offsets}, stage_events=events)
 
     for _ in range(args.warmup):

@@ -12,16 +12,18 @@
 // rows of one expert (the MMA N side).  For gate/up the 128 weight rows are
 // 64 gate rows and the 64 matching up rows, so SwiGLU finishes inside the
 // tile.  Per 128-wide K group:
-//   warp 8 (TMA)      packed INT4 box [128 rows x 64 B] (64-byte swizzle) and
-//                     the activation codes [n rows x 128 B] (128-byte swizzle,
-//                     rows gathered four at a time) into a 6-stage ring;
+//   warp 12 (TMA W)   packed INT4 box [128 rows x 64 B] (64-byte swizzle)
+//                     into a 12-stage ring (96 KB in flight for decode);
+//   warp 14 (TMA B)   the activation codes [n rows x 128 B] (128-byte
+//                     swizzle, rows gathered four at a time) into a 4-stage ring;
 //   warps 0-3 (cvt)   each thread owns one weight row: 64 B of nibbles ->
 //                     128 E4M3 bytes with byte permutes, stored straight into
 //                     a TMEM A slot (tcgen05.st), 4 slots;
-//   warp 9 (MMA)      4 x tcgen05.mma kind::f8f6f4 (K = 32 each), A from
+//   warp 13 (MMA)     4 x tcgen05.mma kind::f8f6f4 (K = 32 each), A from
 //                     TMEM, B from shared memory, into one of two TMEM
 //                     accumulators (FP32, fresh per group);
-//   warps 4-7 (epi)   tcgen05.ld the group's partial sums, multiply by the
+//   warps 4-11 (epi)  two warps per TMEM lane quadrant, 64 columns each:
+//                     tcgen05.ld the group's partial sums, multiply by the
 //                     row's group scale and add into FP32 registers.
 // After the last group the epilogue applies the token (or row) scale and
 // writes h (plus the SwiGLU and absmax) or Y.
@@ -42,23 +44,28 @@ namespace w4a8 {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kThreads = 320;  // warps 0-3 convert, 4-7 epilogue, 8 TMA, 9 MMA
-constexpr int kStages = 6;
+constexpr int kThreads = 512;      // 16 warps, see the role map above
+constexpr int kWarpW = 12, kWarpMma = 13, kWarpB = 14;
+constexpr int kEpiWarps = 8;
+constexpr int kWStages = 12;
+constexpr int kBStages = 4;
 constexpr int kASlots = 4;
 constexpr int kBM = 128;
-constexpr int kWStageBytes = kBM * kGroup / 2;  // 8 KB of packed INT4
-constexpr int kBStageBytes = kTileN * kGroup;   // 16 KB of E4M3 codes
-constexpr int kUpBytes = 64 * kTileN * 4;       // up-projection exchange for SwiGLU
+constexpr int kHalfN = kTileN / 2;                  // columns per epilogue warp
+constexpr int kWStageBytes = kBM * kGroup / 2;      // 8 KB of packed INT4
+constexpr int kBStageBytes = kTileN * kGroup;       // 16 KB of E4M3 codes
+constexpr int kUpBytes = 64 * kTileN * 4;           // up-projection exchange for SwiGLU
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemA = 0;    // A slots: 32 columns (128 E4M3 per lane) each
 constexpr uint32_t kTmemD = 128;  // two accumulators of kTileN columns
-constexpr int kNumBars = 2 * kStages + 2 * kASlots + 4 + 3;
+constexpr int kNumBars = 2 * kWStages + 2 * kBStages + 2 * kASlots + 4 + 3;
 
 static_assert(kTmemA + kASlots * 32 <= kTmemD, "TMEM A slots overlap the accumulators");
 static_assert(kTmemD + 2 * kTileN <= kTmemCols, "TMEM accumulators exceed the allocation");
+static_assert(kHalfN % 32 == 0, "epilogue column halves are whole 32-column loads");
 
 __host__ __device__ constexpr int smem_bytes(bool gate_up) {
-  return 1024 /* alignment slack */ + kStages * (kWStageBytes + kBStageBytes) +
+  return 1024 /* alignment slack */ + kWStages * kWStageBytes + kBStages * kBStageBytes +
          (gate_up ? kUpBytes : 0) + kNumBars * 8 + 16;
 }
 
@@ -131,19 +138,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sW = smem;
-  uint8_t* sB = sW + kStages * kWStageBytes;
-  float* sU = reinterpret_cast<float*>(sB + kStages * kBStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * kBStageBytes +
+  uint8_t* sB = sW + kWStages * kWStageBytes;
+  float* sU = reinterpret_cast<float*>(sB + kBStages * kBStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kBStages * kBStageBytes +
                                                (kGateUp ? kUpBytes : 0));
-  uint64_t* full = bars;                 // [kStages]  TMA bytes landed
-  uint64_t* empty = full + kStages;      // [kStages]  4 converter warps + MMA done
-  uint64_t* afull = empty + kStages;     // [kASlots]  converted A in TMEM
-  uint64_t* aempty = afull + kASlots;    // [kASlots]  MMAs reading the slot done
-  uint64_t* dfull = aempty + kASlots;    // [2]        group partial sums ready
-  uint64_t* dempty = dfull + 2;          // [2]        epilogue read them
-  uint64_t* upfull = dempty + 2;         // up rows staged in sU
-  uint64_t* upempty = upfull + 1;        // sU consumed
-  uint64_t* drain = upempty + 1;         // all MMAs of this CTA complete
+  uint64_t* wfull = bars;                 // [kWStages] packed weights landed
+  uint64_t* wempty = wfull + kWStages;    // [kWStages] 4 converter warps read them
+  uint64_t* bfull = wempty + kWStages;    // [kBStages] activation rows landed
+  uint64_t* bempty = bfull + kBStages;    // [kBStages] MMAs reading them done
+  uint64_t* afull = bempty + kBStages;    // [kASlots]  converted A in TMEM
+  uint64_t* aempty = afull + kASlots;     // [kASlots]  MMAs reading the slot done
+  uint64_t* dfull = aempty + kASlots;     // [2]        group partial sums ready
+  uint64_t* dempty = dfull + 2;           // [2]        8 epilogue warps read them
+  uint64_t* upfull = dempty + 2;          // up rows staged in sU
+  uint64_t* upempty = upfull + 1;         // sU consumed
+  uint64_t* drain = upempty + 1;          // all MMAs of this CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -153,9 +162,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t tmo = a.timeout_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 5);
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 4);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
     }
     for (int s = 0; s < kASlots; ++s) {
       mbar_init(&afull[s], 4);
@@ -163,18 +176,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int d = 0; d < 2; ++d) {
       mbar_init(&dfull[d], 1);
-      mbar_init(&dempty[d], 4);
+      mbar_init(&dempty[d], kEpiWarps);
     }
-    mbar_init(upfull, 2);
-    mbar_init(upempty, 2);
+    mbar_init(upfull, kEpiWarps / 2);
+    mbar_init(upempty, kEpiWarps / 2);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8 && lane == 0) {
-    prefetch_tmap(&tmap_w);
-    prefetch_tmap(&tmap_act);
-  }
+  if (warp == kWarpW && lane == 0) prefetch_tmap(&tmap_w);
+  if (warp == kWarpB && lane == 0) prefetch_tmap(&tmap_act);
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -185,8 +196,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int total = __ldg(a.tile_prefix + a.E) * mb_count;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == kWarpW) {
+    // ------------------------------------------------------------ TMA: packed weights
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const Tile t = decode_tile(a, mb_count, tile);
+        const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
+        const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
+        for (int g = 0; g < G; ++g) {
+          const int s = it % kWStages;
+          const uint32_t ph = (it / kWStages) & 1;
+          if (!mbar_wait(&wempty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
+          const uint32_t dW = smem_u32(sW + s * kWStageBytes);
+          mbar_arrive_expect_tx(&wfull[s], kWStageBytes);
+          if (kGateUp) {
+            tma_load_2d(dW, &tmap_w, &wfull[s], g * 64, wy0);
+            tma_load_2d(dW + kWStageBytes / 2, &tmap_w, &wfull[s], g * 64, wy1);
+          } else {
+            tma_load_2d(dW, &tmap_w, &wfull[s], g * 64, wy0);
+          }
+          ++it;
+        }
+      }
+      // The latest fill of every stage must have landed before the CTA exits.
+      for (int i = (it > kWStages ? it - kWStages : 0); i < it; ++i)
+        mbar_wait_drain(&wfull[i % kWStages], (i / kWStages) & 1, tmo);
+    }
+    __syncwarp();
+  } else if (warp == kWarpB) {
+    // ------------------------------------------------------------ TMA: activation rows
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
@@ -198,35 +238,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ry[q] = kGateUp ? __ldg(a.row_tokens + r) : static_cast<int32_t>(r);
       }
       const int n_ops = t.n_mma >> 2;
-      const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
-      const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
-      const uint32_t tx = kWStageBytes + t.n_mma * kGroup;
+      const uint32_t tx = t.n_mma * kGroup;
       for (int g = 0; g < G; ++g) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
-        const uint32_t dW = smem_u32(sW + s * kWStageBytes);
+        const int s = it % kBStages;
+        const uint32_t ph = (it / kBStages) & 1;
+        if (!mbar_wait(&bempty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
         const uint32_t dB = smem_u32(sB + s * kBStageBytes);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], tx);
-          if (kGateUp) {
-            tma_load_2d(dW, &tmap_w, &full[s], g * 64, wy0);
-            tma_load_2d(dW + kWStageBytes / 2, &tmap_w, &full[s], g * 64, wy1);
-          } else {
-            tma_load_2d(dW, &tmap_w, &full[s], g * 64, wy0);
-          }
-        }
+        if (lane == 0) mbar_arrive_expect_tx(&bfull[s], tx);
         __syncwarp();
         if (lane < n_ops)
-          tma_gather4(dB + lane * 4 * kGroup, &tmap_act, &full[s], g * kGroup, ry[0], ry[1], ry[2],
-                      ry[3]);
+          tma_gather4(dB + lane * 4 * kGroup, &tmap_act, &bfull[s], g * kGroup, ry[0], ry[1],
+                      ry[2], ry[3]);
         ++it;
       }
     }
-    // The latest fill of every stage must have landed before the CTA exits.
-    for (int i = (it > kStages ? it - kStages : 0); i < it; ++i)
-      mbar_wait_drain(&full[i % kStages], (i / kStages) & 1, tmo);
-  } else if (warp == 9) {
+    if (lane == 0)
+      for (int i = (it > kBStages ? it - kBStages : 0); i < it; ++i)
+        mbar_wait_drain(&bfull[i % kBStages], (i / kBStages) & 1, tmo);
+    __syncwarp();
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0;
@@ -235,20 +265,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = decode_tile(a, mb_count, tile);
         const uint32_t idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
         for (int g = 0; g < G; ++g) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
+          const int sb = it % kBStages;
+          const uint32_t phb = (it / kBStages) & 1;
           const int as = it % kASlots;
           const uint32_t pha = (it / kASlots) & 1;
           const int d = it & 1;
           const uint32_t phd = (it >> 1) & 1;
           if (!mbar_wait(&dempty[d], phd ^ 1, abort_flag, tmo) ||
-              !mbar_wait(&full[s], ph, abort_flag, tmo) ||
+              !mbar_wait(&bfull[sb], phb, abort_flag, tmo) ||
               !mbar_wait(&afull[as], pha, abort_flag, tmo)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * kBStageBytes));
+          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + sb * kBStageBytes));
           const uint32_t dt = tmem + kTmemD + d * kTileN;
           const uint32_t at = tmem + kTmemA + as * 32;
 #pragma unroll
@@ -257,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       kk > 0 ? 1u : 0u);
           tc_commit(&dfull[d]);
           tc_commit(&aempty[as]);
-          tc_commit(&empty[s]);
+          tc_commit(&bempty[sb]);
           ++it;
         }
       }
@@ -274,11 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
       for (int g = 0; g < G; ++g) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
+        const int s = it % kWStages;
+        const uint32_t ph = (it / kWStages) & 1;
         const int as = it % kASlots;
         const uint32_t pha = (it / kASlots) & 1;
-        if (!mbar_wait(&full[s], ph, abort_flag, tmo) ||
+        if (!mbar_wait(&wfull[s], ph, abort_flag, tmo) ||
             !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo)) {
           ok = false;
           break;
@@ -294,20 +324,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           cvt8_uint4b8_e4m3(v.z, r[8 * c + 4], r[8 * c + 5]);
           cvt8_uint4b8_e4m3(v.w, r[8 * c + 6], r[8 * c + 7]);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wempty[s]);     // the stage's bytes are in registers
         tmem_st_32x32b_x32(tmem + lane_base + kTmemA + as * 32, r);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&afull[as]);
-          mbar_arrive(&empty[s]);
-        }
+        if (lane == 0) mbar_arrive(&afull[as]);
         ++it;
       }
     }
-  } else {
+  } else if (warp < 4 + kEpiWarps) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                         // TMEM lane quadrant
+    const int half = (warp - 4) >> 2;               // column half of the tile
     const int m = q * 32 + lane;                    // weight row of the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const __nv_bfloat16* wscale = static_cast<const __nv_bfloat16*>(a.wscale);
@@ -319,10 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                : t.mb * kBM + m;
       const __nv_bfloat16* srow =
           wscale + (static_cast<int64_t>(t.e) * a.n_rows + wrow) * static_cast<int64_t>(G);
-      float ts[kTileN / 32];  // token (gate/up) or row (down) scales, lane-strided
+      const int j0 = half * kHalfN;                 // first column (segment row) of this warp
+      float ts[kHalfN / 32];  // token (gate/up) or row (down) scales, lane-strided
 #pragma unroll
-      for (int i = 0; i < kTileN / 32; ++i) {
-        const int j = lane + 32 * i;
+      for (int i = 0; i < kHalfN / 32; ++i) {
+        const int j = j0 + lane + 32 * i;
         float v = 0.0f;
         if (j < t.n_valid) {
           const int64_t r = t.row0 + j;
@@ -330,9 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ts[i] = v;
       }
-      float acc[kTileN];
+      float acc[kHalfN];
 #pragma unroll
-      for (int j = 0; j < kTileN; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < kHalfN; ++j) acc[j] = 0.0f;
       float s_next = __bfloat162float(srow[0]);
       for (int g = 0; g < G; ++g) {
         const float sg = s_next;
@@ -341,10 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t phd = (it >> 1) & 1;
         if (!mbar_wait(&dfull[d], phd, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t taddr = tmem + lane_base + kTmemD + d * kTileN;
+        const uint32_t taddr = tmem + lane_base + kTmemD + d * kTileN + j0;
 #pragma unroll
-        for (int c = 0; c < kTileN / 32; ++c) {
-          if (c * 32 < t.n_mma) {
+        for (int c = 0; c < kHalfN / 32; ++c) {
+          if (j0 + c * 32 < t.n_mma) {
             uint32_t v[32];
             tmem_ld_32x32b_x32(taddr + c * 32, v);
             tmem_wait_ld();
@@ -365,10 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (q >= 2) {  // up rows: stage u = acc * token scale for the gate warps
           if (!mbar_wait(upempty, phu ^ 1, abort_flag, tmo)) break;
 #pragma unroll
-          for (int j = 0; j < kTileN; ++j) {
-            if (j < t.n_valid) {
-              const float tsj = __shfl_sync(kFull, ts[j >> 5], j & 31);
-              sU[j * 64 + (m - 64)] = acc[j] * tsj;
+          for (int jj = 0; jj < kHalfN; ++jj) {
+            if (j0 + jj < t.n_valid) {
+              const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
+              sU[(j0 + jj) * 64 + (m - 64)] = acc[jj] * tsj;
             }
           }
           __syncwarp();
@@ -376,13 +407,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {  // gate rows: h = silu(gate) * up, store, row absmax
           if (!mbar_wait(upfull, phu, abort_flag, tmo)) break;
 #pragma unroll
-          for (int j = 0; j < kTileN; ++j) {
-            if (j < t.n_valid) {
-              const float tsj = __shfl_sync(kFull, ts[j >> 5], j & 31);
-              const float gt = acc[j] * tsj;
-              const float u = sU[j * 64 + m];
+          for (int jj = 0; jj < kHalfN; ++jj) {
+            if (j0 + jj < t.n_valid) {
+              const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
+              const float gt = acc[jj] * tsj;
+              const float u = sU[(j0 + jj) * 64 + m];
               const float h = __fdiv_rn(gt, 1.0f + expf(-gt)) * u;
-              const int64_t r = t.row0 + j;
+              const int64_t r = t.row0 + j0 + jj;
               a.out[r * a.out_ld + t.mb * 64 + m] = h;
               const float hm = warp_max(fabsf(h));
               if (lane == 0) atomicMax(a.row_amax + r, __float_as_uint(hm));
@@ -393,15 +424,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < kTileN; ++j) {
-          if (j < t.n_valid) {
-            const float tsj = __shfl_sync(kFull, ts[j >> 5], j & 31);
-            a.out[(t.row0 + j) * a.out_ld + t.mb * kBM + m] = acc[j] * tsj;
+        for (int jj = 0; jj < kHalfN; ++jj) {
+          if (j0 + jj < t.n_valid) {
+            const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
+            a.out[(t.row0 + j0 + jj) * a.out_ld + t.mb * kBM + m] = acc[jj] * tsj;
           }
         }
       }
     }
   }
+  // warp 15 has no role
 
   tc_fence_before();
   __syncthreads();

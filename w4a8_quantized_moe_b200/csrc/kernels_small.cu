@@ -155,62 +155,55 @@ __global__ void __launch_bounds__(256) pack_int4_kernel(const __nv_bfloat16* __r
 }
 
 // ---------------------------------------------------------------- routing
-// Top-k per token: each warp takes 32 consecutive tokens of the block, one at
-// a time; lane l holds the logits of experts l, l+32, ...  k rounds of a warp
-// arg-max under the order (larger logit, then lower id).  Weights: softmax of
-// the selected logits in float32.  Also counts the block's tokens per expert.
+// Top-k per token, one warp per token: lane l holds the logits of experts
+// l, l+32, ...; k rounds of a warp arg-max under the order (larger logit, then
+// lower id).  Weights: softmax of the selected logits in float32.  Each
+// selection also counts into block_counts[token / kRouteTok][expert] (global
+// atomics; the launcher zeroes the counts first).
 template <int NV>  // logits per lane (E <= 32 * NV)
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int64_t T,
                                                          int E, int k, int32_t* __restrict__ topk_ids,
                                                          float* __restrict__ topk_w,
                                                          int32_t* __restrict__ block_counts) {
-  __shared__ int cnt[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * kRouteTok + warp * 32;
-  for (int i = 0; i < 32; ++i) {
-    const int64_t t = t_begin + i;
-    if (t >= T) break;
-    const float* lt = logits + t * E;
-    float v[NV];
-    uint32_t taken = 0;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;  // warp-uniform
+  const float* lt = logits + t * E;
+  int32_t* counts = block_counts + (t / kRouteTok) * E;
+  float v[NV];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    const int e = lane + 32 * q;
+    if (e < E) v[q] = __ldg(lt + e);
+    else { v[q] = -INFINITY; taken |= 1u << q; }
+  }
+  float myv = 0.0f, v0 = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = INT_MAX;
 #pragma unroll
     for (int q = 0; q < NV; ++q) {
       const int e = lane + 32 * q;
-      if (e < E) v[q] = __ldg(lt + e);
-      else { v[q] = -INFINITY; taken |= 1u << q; }
+      if (!((taken >> q) & 1u) && (v[q] > bv || (v[q] == bv && e < bi))) { bv = v[q]; bi = e; }
     }
-    float myv = 0.0f, v0 = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = INT_MAX;
 #pragma unroll
-      for (int q = 0; q < NV; ++q) {
-        const int e = lane + 32 * q;
-        if (!((taken >> q) & 1u) && (v[q] > bv || (v[q] == bv && e < bi))) { bv = v[q]; bi = e; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(kFull, bv, o);
-        const int oi = __shfl_xor_sync(kFull, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == j) myv = bv;
-      if (j == 0) v0 = bv;
-      if (lane == 0) {
-        topk_ids[t * k + j] = bi;
-        atomicAdd(&cnt[bi], 1);
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(kFull, bv, o);
+      const int oi = __shfl_xor_sync(kFull, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    const float ex = (lane < k) ? expf(myv - v0) : 0.0f;
-    const float sum = warp_sum(ex);
-    if (lane < k) topk_w[t * k + lane] = __fdiv_rn(ex, sum);
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) {
+      myv = bv;
+      topk_ids[t * k + j] = bi;
+      atomicAdd(counts + bi, 1);
+    }
+    if (j == 0) v0 = bv;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = cnt[e];
+  const float ex = (lane < k) ? expf(myv - v0) : 0.0f;
+  const float sum = warp_sum(ex);
+  if (lane < k) topk_w[t * k + lane] = __fdiv_rn(ex, sum);
 }
 
 // Exclusive scan over the experts (one CTA of 1024 threads, thread = expert):
@@ -279,57 +272,43 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   }
 }
 
-// Stable scatter: one warp per routing block walks its 256 tokens in chunks
-// of 32 (lane = token).  A per-expert bitmask of the chunk's tokens gives the
-// rank of a token among earlier tokens of the chunk; a per-expert running
-// count carries the rank across chunks.
-__global__ void __launch_bounds__(32) route_scatter_kernel(const int32_t* __restrict__ topk_ids,
-                                                           int64_t T, int E, int k,
-                                                           const int32_t* __restrict__ block_base,
-                                                           int32_t* __restrict__ sorted_token_ids,
-                                                           int32_t* __restrict__ row_of,
-                                                           uint32_t* __restrict__ row_amax) {
-  __shared__ uint32_t mask[kMaxExperts];
-  __shared__ int running[kMaxExperts];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) { mask[e] = 0u; running[e] = 0; }
-  __syncwarp();
+// Stable scatter: one CTA per routing block of 256 tokens, warp w owns tokens
+// 32w..32w+31 of the block (lane = token).  mask[w][e] has bit l set when
+// token l of chunk w chose expert e; the rank of a token among the block's
+// tokens of expert e is the popcount of the earlier chunks' masks plus the
+// bits below it in its own chunk's mask.
+constexpr int kScatterWarps = kRouteTok / 32;
+
+__global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
+    const int32_t* __restrict__ topk_ids, int64_t T, int E, int k,
+    const int32_t* __restrict__ block_base, int32_t* __restrict__ sorted_token_ids,
+    int32_t* __restrict__ row_of, uint32_t* __restrict__ row_amax) {
+  extern __shared__ uint32_t mask[];  // [kScatterWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteTok + threadIdx.x;
+  const bool valid = t < T;
+  int ids[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) ids[j] = (valid && j < k) ? __ldg(topk_ids + t * k + j) : 0;
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (valid && j < k) atomicOr(&mask[warp * E + ids[j]], 1u << lane);
+  __syncthreads();
   const uint32_t lt_mask = (1u << lane) - 1u;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteTok;
   const int32_t* base = block_base + static_cast<int64_t>(blockIdx.x) * E;
-  for (int c = 0; c < kRouteTok / 32; ++c) {
-    const int64_t t = t0 + c * 32 + lane;
-    const bool valid = t < T;
-    int ids[kMaxTopK];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) ids[j] = (valid && j < k) ? __ldg(topk_ids + t * k + j) : 0;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (valid && j < k) atomicOr(&mask[ids[j]], 1u << lane);
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (valid && j < k) {
-        const uint32_t m = mask[ids[j]];
-        const int row = base[ids[j]] + running[ids[j]] + __popc(m & lt_mask);
-        row_of[t * k + j] = row;
-        sorted_token_ids[row] = static_cast<int32_t>(t);
-        if (row_amax) row_amax[row] = 0u;
-      }
+  for (int j = 0; j < kMaxTopK; ++j) {
+    if (valid && j < k) {
+      const int e = ids[j];
+      int rank = __popc(mask[warp * E + e] & lt_mask);
+      for (int w = 0; w < warp; ++w) rank += __popc(mask[w * E + e]);
+      const int row = base[e] + rank;
+      row_of[t * k + j] = row;
+      sorted_token_ids[row] = static_cast<int32_t>(t);
+      if (row_amax) row_amax[row] = 0u;
     }
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (valid && j < k) {
-        const uint32_t m = mask[ids[j]];
-        if ((m & lt_mask) == 0u) running[ids[j]] += __popc(m);
-      }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (valid && j < k) mask[ids[j]] = 0u;
-    __syncwarp();
   }
 }
 
@@ -430,28 +409,33 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          int32_t* tile_prefix, uint32_t* row_amax_to_zero, cudaStream_t s) {
   const int64_t nblk = route_blocks(T);
   if (nblk > 0) {
+    cudaError_t err = cudaMemsetAsync(block_counts, 0,
+                                      static_cast<size_t>(nblk) * E * sizeof(int32_t), s);
+    if (err != cudaSuccess) return err;
+    const int64_t grid = (T + 7) / 8;  // one warp per token, 8 per CTA
     const int nv = (E + 31) / 32;
     if (nv <= 1)
-      route_topk_kernel<1><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+      route_topk_kernel<1><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
     else if (nv <= 2)
-      route_topk_kernel<2><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+      route_topk_kernel<2><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
     else if (nv <= 4)
-      route_topk_kernel<4><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+      route_topk_kernel<4><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
     else if (nv <= 8)
-      route_topk_kernel<8><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+      route_topk_kernel<8><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
     else if (nv <= 16)
-      route_topk_kernel<16><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+      route_topk_kernel<16><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
     else
-      route_topk_kernel<32><<<nblk, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
-    cudaError_t err = cudaGetLastError();
+      route_topk_kernel<32><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, block_counts);
+    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
   route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, block_base, expert_offsets,
                                        tile_prefix);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || nblk == 0) return err;
-  route_scatter_kernel<<<nblk, 32, 0, s>>>(topk_ids, T, E, k, block_base, sorted_token_ids, row_of,
-                                           row_amax_to_zero);
+  const size_t smem = static_cast<size_t>(kScatterWarps) * E * sizeof(uint32_t);
+  route_scatter_kernel<<<nblk, kRouteTok, smem, s>>>(topk_ids, T, E, k, block_base,
+                                                     sorted_token_ids, row_of, row_amax_to_zero);
   return cudaGetLastError();
 }
 
