@@ -142,6 +142,41 @@ W4A8_API w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int3
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * w4a8_moe_route_permute_noalloc - the same routing and permutation as
+ * w4a8_moe_route_permute, for callers that cannot allocate device memory.
+ * (The pages have no counterpart: this is a calling convention of this
+ * library, not a step of the method.)
+ *
+ * Why: some callers may not call cudaMalloc where they route tokens - code
+ * running while a CUDA graph is being captured (an allocation there breaks
+ * the capture or is not replayed), runtimes and plugin interfaces that give a
+ * kernel only its planned inputs and outputs and no scratch, and paths whose
+ * device memory budget is fixed in advance.  This call takes no workspace and
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Scratch: a file-scope device array of 528,388 bytes (2 * 65536 + 1025
+ * int32) that every device which loads the library holds until the process
+ * exits.  Limit: ceil(T / 256) * E <= 65536 (for example T <= 65536 with
+ * E = 256, or T <= 16384 with E = 1024); larger problems get
+ * W4A8_ERR_UNSUPPORTED_SHAPE and should use w4a8_moe_route_permute.
+ * Set-up: the first call on each device looks up the array's device address
+ * with that device current; make that first call before any stream capture.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents.  The histogram part is zeroed by each call on `stream`
+ * and the rest is rewritten before it is read, but calls that overlap on the
+ * GPU (different streams at the same time) race on it and must be ordered by
+ * the caller.
+ *
+ * Arguments, outputs and errors are those of w4a8_moe_route_permute without
+ * the workspace.
+ */
+W4A8_API w4a8_status w4a8_moe_route_permute_noalloc(const float* logits, int64_t T, int32_t E,
+                                                    int32_t k, int32_t* topk_ids, float* topk_w,
+                                                    int32_t* expert_offsets,
+                                                    int32_t* sorted_token_ids, int32_t* row_of,
+                                                    void* stream);
+
+/*
  * Optional outputs and instrumentation of w4a8_moe_forward.  Every member may
  * be NULL.  A non-NULL buffer replaces the workspace region of the same
  * intermediate, so it receives exactly what the layer computed.  Shapes use

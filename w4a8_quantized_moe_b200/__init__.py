@@ -16,7 +16,8 @@ import torch
 
 __all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_abi_version",
            "w4a8_status_string", "w4a8_pack_int4", "w4a8_quant_act_fp8_per_token",
-           "w4a8_moe_route_workspace_size", "w4a8_moe_route_permute", "w4a8_moe_workspace_size",
+           "w4a8_moe_route_workspace_size", "w4a8_moe_route_permute",
+           "w4a8_moe_route_permute_noalloc", "w4a8_moe_workspace_size",
            "w4a8_moe_forward", "w4a8_check_device_error", "W4A8MoELayer"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a8.so")
@@ -55,6 +56,7 @@ def _declare(L):
         "w4a8_quant_act_fp8_per_token": (i32, [vp, i64, i64, vp, vp, vp]),
         "w4a8_moe_route_workspace_size": (sz, [i64, i32]),
         "w4a8_moe_route_permute": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "w4a8_moe_route_permute_noalloc": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]),
         "w4a8_moe_workspace_size": (sz, [i64, i64, i64, i32, i32]),
         "w4a8_moe_forward": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, sz,
                                    vp, vp]),
@@ -184,6 +186,30 @@ def w4a8_moe_route_permute(logits: torch.Tensor, k: int,
                                         _p(out["topk_w"]), _p(out["expert_offsets"]),
                                         _p(out["sorted_token_ids"]), _p(out["row_of"]),
                                         _p(workspace), workspace.numel(), _stream(dev)))
+    return out
+
+
+def w4a8_moe_route_permute_noalloc(logits: torch.Tensor, k: int,
+                                   out: Optional[Dict[str, torch.Tensor]] = None
+                                   ) -> Dict[str, torch.Tensor]:
+    """Routing + permutation without a workspace, for callers that cannot
+    allocate device memory at call time (see include/w4a8.h).  The library
+    allocates nothing; pass ``out`` (the five output tensors) to allocate
+    nothing here either."""
+    _need(logits, "logits", torch.float32, 2)
+    T, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = dict(topk_ids=torch.empty(T, k, dtype=torch.int32, device=dev),
+                   topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+                   expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                   sorted_token_ids=torch.empty(T * k, dtype=torch.int32, device=dev),
+                   row_of=torch.empty(T, k, dtype=torch.int32, device=dev))
+    _check("w4a8_moe_route_permute_noalloc",
+           lib().w4a8_moe_route_permute_noalloc(_p(logits), T, E, k, _p(out["topk_ids"]),
+                                                _p(out["topk_w"]), _p(out["expert_offsets"]),
+                                                _p(out["sorted_token_ids"]), _p(out["row_of"]),
+                                                _stream(dev)))
     return out
 
 

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libw4a8.so")
-SOURCES = ["kernels_small.cu", "grouped_gemm.cu", "capi.cu"]
+SOURCES = ["kernels_small.cu", "grouped_gemm.cu", "capi.cu", "route_static.cu"]
 HEADERS = ["internal.h", "ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

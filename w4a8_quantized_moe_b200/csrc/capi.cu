@@ -17,6 +17,7 @@
 
 namespace w4a8 {
 cudaError_t read_and_clear_device_error(int* value);
+const char* set_last_error(const char* msg);
 }
 
 using namespace w4a8;
@@ -199,6 +200,14 @@ w4a8_status check_route_args(const void* logits, int64_t T, int32_t E, int32_t k
 }
 
 }  // namespace
+
+namespace w4a8 {
+// Records the message w4a8_last_error() returns on this thread.
+const char* set_last_error(const char* msg) {
+  g_last_error = msg;
+  return g_last_error.c_str();
+}
+}  // namespace w4a8
 
 extern "C" {
 
