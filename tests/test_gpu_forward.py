@@ -92,6 +92,10 @@ def test_forward_tiny_workload():
                         forced_empty=5),
     workloads.MoEConfig("outliers_wide", T=24, H=1024, I=512, E=8, k=2, seed=16,
                         outlier_frac=0.01),
+    # few tokens per expert on average (the narrow-tile shape) but skewed, so
+    # the busiest experts span several 32-token tiles
+    workloads.MoEConfig("decode_shape_multi_block", T=96, H=256, I=128, E=8, k=2, seed=17,
+                        zipf_s=1.1),
 ], ids=lambda c: c.name)
 def test_forward_edge_cases(cfg):
     run_and_compare(cfg, *small_case(cfg))

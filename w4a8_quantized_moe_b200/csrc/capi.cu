@@ -176,6 +176,9 @@ w4a8_status encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uin
   return W4A8_OK;
 }
 
+// Average tokens per expert up to which w4a8_moe_forward uses the decode shape.
+constexpr int kDecodeTokensPerExpert = 32;
+
 uint64_t wait_timeout_ns() {
   static uint64_t v = [] {
     const char* s = std::getenv("W4A8_WAIT_TIMEOUT_MS");
@@ -304,7 +307,8 @@ w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int32_t E, in
   RouteBufs rb = carve_route(c, T, E);
   cudaError_t err = launch_route(logits, T, E, k, topk_ids, topk_w, expert_offsets,
                                  sorted_token_ids, row_of, rb.block_counts, rb.block_base,
-                                 rb.tile_prefix, nullptr, static_cast<cudaStream_t>(stream));
+                                 rb.tile_prefix, kTileNPrefill, nullptr,
+                                 static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "route launch");
 }
 
@@ -368,6 +372,10 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
     ev = aux->stage_events;
   }
   const int64_t A = T * k;
+  // Few tokens per expert (decode): narrow tiles with a deep pipeline; many
+  // (prefill): wide tiles that feed each converted weight tile to more tokens.
+  const bool decode = A <= static_cast<int64_t>(kDecodeTokensPerExpert) * E;
+  const int tile_n = grouped_gemm_tile_n(decode);
 
   // TMA descriptors: packed weights [E * rows, K / 2] bytes, 64-byte swizzle;
   // activation codes [rows, K] bytes, 128-byte swizzle, one-row boxes for gather4.
@@ -404,7 +412,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   W4A8_STEP(record(2), "cudaEventRecord");
   W4A8_STEP(launch_route(logits, T, E, k, b.topk_ids, b.topk_w, b.expert_offsets,
                          b.sorted_token_ids, b.row_of, b.route.block_counts, b.route.block_base,
-                         b.route.tile_prefix, b.row_amax, s),
+                         b.route.tile_prefix, tile_n, b.row_amax, s),
             "route launch");
   W4A8_STEP(record(3), "cudaEventRecord");
 
@@ -424,7 +432,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
   W4A8_STEP(record(4), "cudaEventRecord");
-  W4A8_STEP(launch_grouped_gemm(true, tw1, ta1, g1, di.sms, s), "gate/up GEMM launch");
+  W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, g1, di.sms, s), "gate/up GEMM launch");
   W4A8_STEP(record(5), "cudaEventRecord");
 
   W4A8_STEP(record(6), "cudaEventRecord");
@@ -448,7 +456,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g2.act_rows = A;
   g2.timeout_ns = wait_timeout_ns();
   W4A8_STEP(record(8), "cudaEventRecord");
-  W4A8_STEP(launch_grouped_gemm(false, tw2, ta2, g2, di.sms, s), "down GEMM launch");
+  W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, g2, di.sms, s), "down GEMM launch");
   W4A8_STEP(record(9), "cudaEventRecord");
 
   W4A8_STEP(record(10), "cudaEventRecord");

@@ -10,7 +10,8 @@ namespace w4a8 {
 
 constexpr int kGroup = 128;        // INT4 group size along K
 constexpr int kRouteTok = 256;     // tokens per routing block
-constexpr int kTileN = 128;        // max tokens per grouped-GEMM tile
+constexpr int kTileNDecode = 32;   // tokens per grouped-GEMM tile, decode shape
+constexpr int kTileNPrefill = 128; // tokens per grouped-GEMM tile, prefill shape
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 
@@ -22,10 +23,12 @@ cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
                              int num_sms, cudaStream_t s);
 // routing: top-k + per-block expert histogram; scan; stable scatter.
+// tile_prefix[e] = sum over experts e' < e of ceil(count[e'] / tile_n).
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
                          float* topk_w, int32_t* expert_offsets, int32_t* sorted_token_ids,
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
-                         int32_t* tile_prefix, uint32_t* row_amax_to_zero, cudaStream_t s);
+                         int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
+                         cudaStream_t s);
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
@@ -38,7 +41,7 @@ struct GemmArgs {
   int half_rows;                  // gate/up: I (first up row); down: 0
   int E;
   const int32_t* expert_offsets;  // [E + 1]
-  const int32_t* tile_prefix;     // [E + 1] prefix of ceil(count / kTileN)
+  const int32_t* tile_prefix;     // [E + 1] prefix of ceil(count / tile width of the shape)
   const int32_t* row_tokens;      // gate/up: sorted_token_ids (gather rows); down: nullptr
   const float* act_scale;         // gate/up: per token [T]; down: per segment row [A]
   const void* wscale;             // bf16 [E, n_rows, K / 128]
@@ -48,9 +51,10 @@ struct GemmArgs {
   int64_t act_rows;               // rows of the activation tensor (T or A)
   uint64_t timeout_ns;
 };
-cudaError_t launch_grouped_gemm(bool gate_up, const CUtensorMap& tmap_w,
+// decode = the shape for few tokens per expert (see grouped_gemm.cu).
+cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
                                 cudaStream_t s);
-size_t grouped_gemm_smem_bytes(bool gate_up);
+int grouped_gemm_tile_n(bool decode);
 
 }  // namespace w4a8

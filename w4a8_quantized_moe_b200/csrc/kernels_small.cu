@@ -235,7 +235,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh /*[32]*/, int
 }
 
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ block_counts,
-                                                          int64_t nblk, int E,
+                                                          int64_t nblk, int E, int tile_n,
                                                           int32_t* __restrict__ block_base,
                                                           int32_t* __restrict__ expert_offsets,
                                                           int32_t* __restrict__ tile_prefix) {
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   }
   int total = 0, total_tiles = 0;
   const int off = block_exclusive_scan(e < E ? running : 0, sh, &total);
-  const int tiles = (e < E) ? (running + kTileN - 1) / kTileN : 0;
+  const int tiles = (e < E) ? (running + tile_n - 1) / tile_n : 0;
   const int toff = block_exclusive_scan(tiles, sh, &total_tiles);
   if (e < E) {
     expert_offsets[e] = off;
@@ -406,7 +406,8 @@ cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packe
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
                          float* topk_w, int32_t* expert_offsets, int32_t* sorted_token_ids,
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
-                         int32_t* tile_prefix, uint32_t* row_amax_to_zero, cudaStream_t s) {
+                         int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
+                         cudaStream_t s) {
   const int64_t nblk = route_blocks(T);
   if (nblk > 0) {
     cudaError_t err = cudaMemsetAsync(block_counts, 0,
@@ -429,8 +430,8 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
-  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, block_base, expert_offsets,
-                                       tile_prefix);
+  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, tile_n, block_base,
+                                       expert_offsets, tile_prefix);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || nblk == 0) return err;
   const size_t smem = static_cast<size_t>(kScatterWarps) * E * sizeof(uint32_t);

@@ -120,8 +120,8 @@ extern "C" W4A8_API w4a8_status w4a8_moe_route_permute_noalloc(
   // the tile prefix are fully rewritten before they are read.
   cudaError_t err = w4a8::launch_route(logits, T, E, k, topk_ids, topk_w, expert_offsets,
                                        sorted_token_ids, row_of, scratch, scratch + kTableEntries,
-                                       scratch + 2 * kTableEntries, nullptr,
-                                       static_cast<cudaStream_t>(stream));
+                                       scratch + 2 * kTableEntries, w4a8::kTileNPrefill,
+                                       nullptr, static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) {
     w4a8::set_last_error(cudaGetErrorString(err));
     return W4A8_ERR_CUDA;
