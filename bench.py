@@ -95,7 +95,7 @@ class ClockSampler:
 
 
 def build_layer(cfg, device, w4):
-    """Pack every expert's seeded bf16 weights on the device (not timed)."""
+    """Pack every expert's seeded bf16 weights on the device and lay them out for the GEMMs (not timed)."""
     E, H, I = cfg.E, cfg.H, cfg.I
     p13 = torch.empty(E, 2 * I, H // 8, dtype=torch.int32, device=device)
     s13 = torch.empty(E, 2 * I, H // 128, dtype=torch.bfloat16, device=device)
@@ -105,8 +105,11 @@ def build_layer(cfg, device, w4):
         w13, w2 = workloads.gen_expert_weights(cfg, e, device=device)
         w4.w4a8_pack_int4(w13, packed=p13[e], scales=s13[e])
         w4.w4a8_pack_int4(w2, packed=p2[e], scales=s2[e])
+    p13, s13g = w4.w4a8_prepare_experts_b200(p13, s13, packed_out=p13)
+    p2, s2g = w4.w4a8_prepare_experts_b200(p2, s2, packed_out=p2)
     torch.cuda.synchronize(device)
-    return w4.W4A8MoELayer(p13, s13, p2, s2, cfg.k)
+    del s13, s2
+    return w4.W4A8MoELayer(p13, s13g, p2, s2g, cfg.k)
 
 
 def algorithmic_work(cfg, counts):

@@ -93,6 +93,34 @@ W4A8_API w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, in
                            int32_t* packed, void* scales_bf16, void* stream);
 
 /*
+ * w4a8_prepare_experts_b200 - lay out one projection's quantised experts the
+ * way w4a8_moe_forward reads them.  The codes and scale values are those of
+ * w4a8_pack_int4 (the pages fix the uint4b8 codes and the group-128 bf16
+ * scales); only their placement in memory is this library's own.
+ *
+ * Words: inside every int32 word the nibble of element j (0..7) moves from
+ * bits 4j..4j+3 to bits 8j..8j+3 for j < 4 and to bits 8(j-4)+4..8(j-4)+7 for
+ * j >= 4.  Then (w & 0x0F0F0F0F) holds elements 0..3, one per byte, and
+ * ((w >> 4) & 0x0F0F0F0F) elements 4..7; the grouped GEMM turns each such
+ * byte u straight into the E4M3 value u * 2^-9 (exact for u = 0..15).  Word
+ * order is unchanged, so the map is a bijection on words.
+ * Scales: [E, rows, K / 128] -> group-major [E, K / 128, rows], so that the
+ * scales of consecutive rows for one group are contiguous.
+ *
+ *   packed       [E, rows, K / 8] int32 from w4a8_pack_int4
+ *   scales_bf16  [E, rows, K / 128] bf16 from w4a8_pack_int4
+ *   E, rows, K   >= 0, >= 0, > 0 with K % 128 == 0 (E * rows == 0: no-op)
+ *   packed_out   [E, rows, K / 8] int32, written; may be `packed` itself
+ *                (in place) but must not partly overlap it
+ *   scales_out   [E, K / 128, rows] bf16, written; must not overlap
+ *                `scales_bf16`
+ */
+W4A8_API w4a8_status w4a8_prepare_experts_b200(const int32_t* packed, const void* scales_bf16,
+                                               int64_t E, int64_t rows, int64_t K,
+                                               int32_t* packed_out, void* scales_out,
+                                               void* stream);
+
+/*
  * w4a8_quant_act_fp8_per_token - dynamic per-token FP8 E4M3 quantisation.
  * (Model card, "quantisation method" and the table above: FP8 per-token
  * dynamic activations.)
@@ -220,16 +248,23 @@ W4A8_API size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t
  *   5. down grouped GEMM: Y[r, n] = h_s[r] * sum_g s2[e, n, g] * sum e4m3 * q2;
  *   6. combine: out[t] = bf16(sum_j topk_w[t, j] * Y[row_of[t, j]]), slot order.
  *
+ * The GEMMs multiply E4M3 activations by the stored nibbles u = q + 8 (each
+ * turned into the exact E4M3 value u * 2^-9) and remove the offset per group:
+ * sum a * q = 512 * sum a * (u * 2^-9) - 8 * sum a, where sum a is the group
+ * sum of the E4M3 activation values, which steps 1 and 4 also write.
+ *
  *   hidden_bf16   [T, H] bf16
  *   logits        [T, E] float32 router logits
- *   w13_packed    [E, 2I, H / 8] int32 (w4a8_pack_int4 of the [E*2I, H]
- *                 gate/up weight; rows [0, I) of each expert are the gate
- *                 projection, rows [I, 2I) the up projection)
- *   w13_scales    [E, 2I, H / 128] bf16
- *   w2_packed     [E, H, I / 8] int32
- *   w2_scales     [E, H, I / 128] bf16
- *   T, H, I, E, k T >= 0 (0: no-op); H % 128 == 0, I % 128 == 0, both > 0;
- *                 1 <= E <= 1024; 1 <= k <= min(E, 32)
+ *   w13_packed    [E, 2I, H / 8] int32: w4a8_pack_int4 of the [E*2I, H]
+ *                 gate/up weight, then w4a8_prepare_experts_b200; rows
+ *                 [0, I) of each expert are the gate projection, rows
+ *                 [I, 2I) the up projection
+ *   w13_scales    [E, H / 128, 2I] bf16 (group-major, from
+ *                 w4a8_prepare_experts_b200)
+ *   w2_packed     [E, H, I / 8] int32, packed then prepared the same way
+ *   w2_scales     [E, I / 128, H] bf16 (group-major)
+ *   T, H, I, E, k T >= 0 (0: no-op); H and I positive multiples of 128, at
+ *                 most 8192 each; 1 <= E <= 1024; 1 <= k <= min(E, 32)
  *   out_bf16      [T, H] bf16, written
  *   workspace     scratch of >= w4a8_moe_workspace_size(T, H, I, E, k) bytes
  *   aux           optional, see w4a8_moe_aux (NULL for none)

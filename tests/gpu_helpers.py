@@ -22,6 +22,17 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
 
 
+def repack_b200(packed: np.ndarray) -> np.ndarray:
+    """Expected word layout of w4a8_prepare_experts_b200, from the header's definition:
+    nibble j of each word moves to nibble 2j (j < 4) or 2(j - 4) + 1 (j >= 4)."""
+    w = np.asarray(packed).view(np.uint32).astype(np.uint64)
+    r = np.zeros_like(w)
+    for j in range(8):
+        dst = 2 * j if j < 4 else 2 * (j - 4) + 1
+        r |= ((w >> np.uint64(4 * j)) & np.uint64(0xF)) << np.uint64(4 * dst)
+    return r.astype(np.uint32).view(np.int32).reshape(np.shape(packed))
+
+
 def e4m3_ordinal(codes: np.ndarray) -> np.ndarray:
     """Position of each E4M3 code on the number line (+0 and -0 both 0)."""
     c = codes.astype(np.int64)

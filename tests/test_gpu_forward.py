@@ -15,7 +15,7 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
-from gpu_helpers import aux_buffers, bf16_bits, codes_agree, f64, rel_fro, small_case
+from gpu_helpers import aux_buffers, bf16_bits, codes_agree, f64, rel_fro, small_case, repack_b200
 
 pytestmark = pytest.mark.gpu
 
@@ -41,10 +41,10 @@ def run_and_compare(cfg, hidden, logits, w13, w2, check_rows=None):
     # packed weights (bit-exact)
     for e in range(E):
         p13, s13, p2, s2 = store[e]
-        assert np.array_equal(layer.w13_packed[e].cpu().numpy(), p13)
-        assert np.array_equal(bf16_bits(layer.w13_scales[e]), oracle.f64_to_bf16_bits(s13))
-        assert np.array_equal(layer.w2_packed[e].cpu().numpy(), p2)
-        assert np.array_equal(bf16_bits(layer.w2_scales[e]), oracle.f64_to_bf16_bits(s2))
+        assert np.array_equal(layer.w13_packed[e].cpu().numpy(), repack_b200(p13))
+        assert np.array_equal(bf16_bits(layer.w13_scales[e].t()), oracle.f64_to_bf16_bits(s13))
+        assert np.array_equal(layer.w2_packed[e].cpu().numpy(), repack_b200(p2))
+        assert np.array_equal(bf16_bits(layer.w2_scales[e].t()), oracle.f64_to_bf16_bits(s2))
     # routing + permutation (bit-exact), weights (1e-6)
     assert np.array_equal(aux["topk_ids"].cpu().numpy(), res["topk_ids"])
     assert np.array_equal(aux["expert_offsets"].cpu().numpy(), res["expert_offsets"])

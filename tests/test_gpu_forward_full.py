@@ -14,7 +14,7 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
-from gpu_helpers import bf16_bits, codes_agree, f64, rel_fro
+from gpu_helpers import bf16_bits, codes_agree, f64, rel_fro, repack_b200
 
 pytestmark = pytest.mark.gpu
 
@@ -78,10 +78,10 @@ def test_forward_full_size_sampled(ci):
     # packed weights of the touched experts (bit-exact)
     for e in sorted(set(res["topk_ids"][toks].reshape(-1).tolist())):
         p13, s13, p2, s2 = store[e]
-        assert np.array_equal(layer.w13_packed[e].cpu().numpy(), p13)
-        assert np.array_equal(bf16_bits(layer.w13_scales[e]), oracle.f64_to_bf16_bits(s13))
-        assert np.array_equal(layer.w2_packed[e].cpu().numpy(), p2)
-        assert np.array_equal(bf16_bits(layer.w2_scales[e]), oracle.f64_to_bf16_bits(s2))
+        assert np.array_equal(layer.w13_packed[e].cpu().numpy(), repack_b200(p13))
+        assert np.array_equal(bf16_bits(layer.w13_scales[e].t()), oracle.f64_to_bf16_bits(s13))
+        assert np.array_equal(layer.w2_packed[e].cpu().numpy(), repack_b200(p2))
+        assert np.array_equal(bf16_bits(layer.w2_scales[e].t()), oracle.f64_to_bf16_bits(s2))
     e_out = rel_fro(f64(out[torch.as_tensor(toks, device=dev)]), res["out"])
     counts = np.diff(res["expert_offsets"].astype(np.int64))
     print(f"\n[{cfg.name}] sampled tokens {toks.tolist()} out rel-Frobenius {e_out:.2e}; "

@@ -9,7 +9,7 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
-from gpu_helpers import bf16_bits, f64
+from gpu_helpers import bf16_bits, f64, repack_b200
 
 pytestmark = pytest.mark.gpu
 
@@ -46,6 +46,33 @@ def test_pack_int4_3d_and_empty():
     assert np.array_equal(packed.reshape(128, 32).cpu().numpy(), oracle.pack_uint4b8(q))
     p0, s0 = w4.w4a8_pack_int4(torch.zeros(0, 256, dtype=torch.bfloat16, device="cuda"))
     assert p0.shape == (0, 32)
+
+
+@pytest.mark.parametrize("E,rows,K", [(1, 1, 128), (3, 5, 384), (4, 256, 2048), (2, 4096, 6144)])
+def test_prepare_experts_bit_exact(E, rows, K):
+    g = torch.Generator().manual_seed(E * 7 + rows + K)
+    words = torch.randint(-2**31, 2**31, (E, rows, K // 8), generator=g, dtype=torch.int64)
+    src = words.to(torch.int32).cuda()
+    sc = torch.randn(E, rows, K // 128, generator=g).to(torch.bfloat16).cuda()
+    p_out, s_out = w4.w4a8_prepare_experts_b200(src, sc)
+    assert np.array_equal(p_out.cpu().numpy(), repack_b200(src.cpu().numpy()))
+    assert np.array_equal(bf16_bits(s_out), bf16_bits(sc.transpose(1, 2)))
+    expect = p_out.cpu().numpy()
+    w4.w4a8_prepare_experts_b200(src, sc, packed_out=src)   # in place gives the same words
+    assert np.array_equal(src.cpu().numpy(), expect)
+
+
+def test_prepare_experts_empty_and_overlap_rejected():
+    w4.w4a8_prepare_experts_b200(torch.zeros(0, 4, 16, dtype=torch.int32, device="cuda"),
+                                 torch.zeros(0, 4, 1, dtype=torch.bfloat16, device="cuda"))
+    buf = torch.zeros(2, 4, 32, dtype=torch.int32, device="cuda")
+    sc = torch.zeros(1, 4, 2, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(w4.W4A8Error):   # words partly overlapping
+        w4.w4a8_prepare_experts_b200(buf[0:1], sc, packed_out=buf.view(-1)[8:136].view(1, 4, 32))
+    scales_buf = torch.zeros(8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(w4.W4A8Error):   # scales_out on top of scales
+        w4.w4a8_prepare_experts_b200(buf[0:1], scales_buf.view(1, 4, 2),
+                                     scales_out=scales_buf.view(1, 2, 4))
 
 
 def _acts(T, H, seed):

@@ -53,6 +53,7 @@ def _declare(L):
         "w4a8_last_error": (ctypes.c_char_p, []),
         "w4a8_check_device_error": (i32, [vp]),
         "w4a8_pack_int4": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+        "w4a8_prepare_experts_b200": (i32, [vp, vp, i64, i64, i64, vp, vp, vp]),
         "w4a8_quant_act_fp8_per_token": (i32, [vp, i64, i64, vp, vp, vp]),
         "w4a8_moe_route_workspace_size": (sz, [i64, i32]),
         "w4a8_moe_route_permute": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -146,6 +147,36 @@ def w4a8_pack_int4(w: torch.Tensor, group: int = 128, packed: Optional[torch.Ten
     _check("w4a8_pack_int4", lib().w4a8_pack_int4(_p(w2), R, K, group, _p(packed), _p(scales),
                                                   _stream(w.device)))
     return packed, scales
+
+
+def w4a8_prepare_experts_b200(packed: torch.Tensor, scales: torch.Tensor,
+                              packed_out: Optional[torch.Tensor] = None,
+                              scales_out: Optional[torch.Tensor] = None):
+    """Lay out ``w4a8_pack_int4`` output the way ``w4a8_moe_forward`` reads it.
+
+    ``packed`` int32 [E, rows, K/8] and ``scales`` bf16 [E, rows, K/128] ->
+    ``(packed_out [E, rows, K/8], scales_out [E, K/128, rows])``: nibbles
+    interleaved inside each word, scales group-major.  ``packed_out`` may be
+    ``packed`` itself (in place).
+    """
+    _need(packed, "packed", torch.int32, 3)
+    _need(scales, "scales", torch.bfloat16, 3)
+    E, rows, k8 = packed.shape
+    K = k8 * 8
+    if scales.shape != (E, rows, K // 128):
+        raise ValueError("scales must be [E, rows, K/128] for packed [E, rows, K/8]")
+    if packed_out is None:
+        packed_out = torch.empty_like(packed)
+    if scales_out is None:
+        scales_out = torch.empty(E, K // 128, rows, dtype=torch.bfloat16, device=packed.device)
+    _need(packed_out, "packed_out", torch.int32, 3)
+    _need(scales_out, "scales_out", torch.bfloat16, 3)
+    if packed_out.shape != packed.shape or scales_out.shape != (E, K // 128, rows):
+        raise ValueError("packed_out must match packed; scales_out must be [E, K/128, rows]")
+    _check("w4a8_prepare_experts_b200",
+           lib().w4a8_prepare_experts_b200(_p(packed), _p(scales), E, rows, K, _p(packed_out),
+                                           _p(scales_out), _stream(packed.device)))
+    return packed_out, scales_out
 
 
 def w4a8_quant_act_fp8_per_token(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
@@ -243,9 +274,10 @@ def w4a8_moe_forward(hidden: torch.Tensor, logits: torch.Tensor, w13_packed: tor
     E = logits.shape[1]
     I = w2_packed.shape[2] * 8
     if logits.shape[0] != T or w13_packed.shape != (E, 2 * I, H // 8) or \
-            w2_packed.shape != (E, H, I // 8):
+            w2_packed.shape != (E, H, I // 8) or w13_scales.shape != (E, H // 128, 2 * I) or \
+            w2_scales.shape != (E, I // 128, H):
         raise ValueError("inconsistent shapes: hidden [T,H], logits [T,E], w13 [E,2I,H/8], "
-                         "w2 [E,H,I/8]")
+                         "w2 [E,H,I/8], w13_scales [E,H/128,2I], w2_scales [E,I/128,H]")
     dev = hidden.device
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
@@ -281,8 +313,9 @@ class W4A8MoELayer:
     """A layer with packed experts resident on the device and a reusable workspace.
 
     ``W4A8MoELayer.from_bf16(w13, w2, k)`` packs bf16 ``w13`` [E, 2I, H] and
-    ``w2`` [E, H, I] with ``w4a8_pack_int4``; calling the layer runs
-    ``w4a8_moe_forward``.
+    ``w2`` [E, H, I] with ``w4a8_pack_int4`` and lays them out with
+    ``w4a8_prepare_experts_b200``; the ``w13_*`` / ``w2_*`` attributes hold
+    that layout.  Calling the layer runs ``w4a8_moe_forward``.
     """
 
     def __init__(self, w13_packed, w13_scales, w2_packed, w2_scales, k: int):
@@ -297,6 +330,8 @@ class W4A8MoELayer:
     def from_bf16(cls, w13: torch.Tensor, w2: torch.Tensor, k: int) -> "W4A8MoELayer":
         p13, s13 = w4a8_pack_int4(w13)
         p2, s2 = w4a8_pack_int4(w2)
+        p13, s13 = w4a8_prepare_experts_b200(p13, s13, packed_out=p13)
+        p2, s2 = w4a8_prepare_experts_b200(p2, s2, packed_out=p2)
         return cls(p13, s13, p2, s2, k)
 
     def workspace(self, T: int) -> torch.Tensor:

@@ -117,10 +117,12 @@ struct ForwardBufs {
   RouteBufs route;
   uint8_t* act_codes;
   float* act_scales;
+  float* act_gsum;
   float* h;
   uint32_t* row_amax;
   uint8_t* inter_codes;
   float* inter_scales;
+  float* inter_gsum;
   float* y;
 };
 
@@ -135,10 +137,12 @@ ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int
   b.route = carve_route(c, T, E);
   b.act_codes = c.take<uint8_t>(static_cast<size_t>(T) * static_cast<size_t>(H));
   b.act_scales = c.take<float>(static_cast<size_t>(T));
+  b.act_gsum = c.take<float>(static_cast<size_t>(T) * static_cast<size_t>(H / kGroup));
   b.h = c.take<float>(A * static_cast<size_t>(I));
   b.row_amax = c.take<uint32_t>(A);
   b.inter_codes = c.take<uint8_t>(A * static_cast<size_t>(I));
   b.inter_scales = c.take<float>(A);
+  b.inter_gsum = c.take<float>(A * static_cast<size_t>(I / kGroup));
   b.y = c.take<float>(A * static_cast<size_t>(H));
   return b;
 }
@@ -272,9 +276,40 @@ w4a8_status w4a8_quant_act_fp8_per_token(const void* x_bf16, int64_t T, int64_t 
     return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   DeviceInfo di;
   if (w4a8_status st = device_info(&di)) return st;
-  cudaError_t err = launch_act_quant(x_bf16, T, H, codes_e4m3, scales, di.sms,
+  cudaError_t err = launch_act_quant(x_bf16, T, H, codes_e4m3, scales, nullptr, di.sms,
                                      static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "act_quant launch");
+}
+
+w4a8_status w4a8_prepare_experts_b200(const int32_t* packed, const void* scales_bf16, int64_t E,
+                                      int64_t rows, int64_t K, int32_t* packed_out,
+                                      void* scales_out, void* stream) {
+  if (E < 0 || rows < 0 || K <= 0)
+    return fail(W4A8_ERR_INVALID_ARG, "E = %lld, rows = %lld, K = %lld", static_cast<long long>(E),
+                static_cast<long long>(rows), static_cast<long long>(K));
+  if (K % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "K = %lld is not a multiple of 128",
+                              static_cast<long long>(K));
+  const int64_t nwords = E * rows * (K / 8);
+  const int64_t nscales = E * rows * (K / kGroup);
+  if (nwords == 0) return W4A8_OK;
+  if (!packed || !scales_bf16 || !packed_out || !scales_out)
+    return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  for (const void* p : {static_cast<const void*>(packed), scales_bf16,
+                        static_cast<const void*>(packed_out), static_cast<const void*>(scales_out)})
+    if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (packed != packed_out && packed < packed_out + nwords && packed_out < packed + nwords)
+    return fail(W4A8_ERR_INVALID_ARG, "packed and packed_out overlap without being the same buffer");
+  const uint8_t* si = static_cast<const uint8_t*>(scales_bf16);
+  const uint8_t* so = static_cast<const uint8_t*>(scales_out);
+  if (si < so + 2 * nscales && so < si + 2 * nscales)
+    return fail(W4A8_ERR_INVALID_ARG, "scales and scales_out overlap");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_repack_int4_b200(packed, nwords, packed_out, di.sms, s);
+  if (err == cudaSuccess)
+    err = launch_transpose_scales(scales_bf16, E, rows, K / kGroup, scales_out, di.sms, s);
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "prepare_experts launch");
 }
 
 size_t w4a8_moe_route_workspace_size(int64_t T, int32_t E) {
@@ -329,6 +364,9 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   if (H <= 0 || I <= 0 || H % kGroup || I % kGroup)
     return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld and I = %lld must be positive multiples of 128",
                 static_cast<long long>(H), static_cast<long long>(I));
+  if (H / kGroup > kMaxGroups || I / kGroup > kMaxGroups)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld, I = %lld: at most %d groups of 128 per row",
+                static_cast<long long>(H), static_cast<long long>(I), kMaxGroups);
   if (static_cast<int64_t>(E) * 2 * I > INT32_MAX || static_cast<int64_t>(E) * H > INT32_MAX)
     return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "E * rows exceeds 2^31 - 1");
   if (T == 0) return W4A8_OK;
@@ -379,7 +417,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
 
   // TMA descriptors: packed weights [E * rows, K / 2] bytes, 64-byte swizzle;
   // activation codes [rows, K] bytes, 128-byte swizzle, one-row boxes for gather4.
-  CUtensorMap tw1, ta1, tw2, ta2;
+  CUtensorMap tw1, ta1, tw2, ta2, ts1, ts2;
   if (w4a8_status st = encode_u8_2d(&tw1, w13_packed, static_cast<uint64_t>(H / 2),
                                     static_cast<uint64_t>(E) * 2 * I, 64, 64,
                                     CU_TENSOR_MAP_SWIZZLE_64B))
@@ -394,6 +432,15 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   if (w4a8_status st = encode_u8_2d(&ta2, b.inter_codes, static_cast<uint64_t>(I),
                                     static_cast<uint64_t>(A), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
+  // group-major scales as bytes: [E * G, 2 * rows]; one box = one tile's scales
+  if (w4a8_status st = encode_u8_2d(&ts1, w13_scales, static_cast<uint64_t>(2 * I) * 2,
+                                    static_cast<uint64_t>(E) * (H / kGroup), 128,
+                                    static_cast<uint32_t>(H / kGroup), CU_TENSOR_MAP_SWIZZLE_NONE))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ts2, w2_scales, static_cast<uint64_t>(H) * 2,
+                                    static_cast<uint64_t>(E) * (I / kGroup), 256,
+                                    static_cast<uint32_t>(I / kGroup), CU_TENSOR_MAP_SWIZZLE_NONE))
+    return st;
 
   auto record = [&](int i) -> cudaError_t {
     return ev && ev[i] ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
@@ -406,7 +453,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   } while (0)
 
   W4A8_STEP(record(0), "cudaEventRecord");
-  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, di.sms, s),
+  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, b.act_gsum, di.sms, s),
             "act_quant launch");
   W4A8_STEP(record(1), "cudaEventRecord");
   W4A8_STEP(record(2), "cudaEventRecord");
@@ -425,6 +472,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g1.tile_prefix = b.route.tile_prefix;
   g1.row_tokens = b.sorted_token_ids;
   g1.act_scale = b.act_scales;
+  g1.act_gsum = b.act_gsum;
   g1.wscale = w13_scales;
   g1.out = b.h;
   g1.out_ld = I;
@@ -432,11 +480,12 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
   W4A8_STEP(record(4), "cudaEventRecord");
-  W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, g1, di.sms, s), "gate/up GEMM launch");
+  W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, g1, di.sms, s), "gate/up GEMM launch");
   W4A8_STEP(record(5), "cudaEventRecord");
 
   W4A8_STEP(record(6), "cudaEventRecord");
-  W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales, di.sms, s),
+  W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales, b.inter_gsum,
+                                di.sms, s),
             "intermediate quant launch");
   W4A8_STEP(record(7), "cudaEventRecord");
 
@@ -449,6 +498,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g2.tile_prefix = b.route.tile_prefix;
   g2.row_tokens = nullptr;
   g2.act_scale = b.inter_scales;
+  g2.act_gsum = b.inter_gsum;
   g2.wscale = w2_scales;
   g2.out = b.y;
   g2.out_ld = H;
@@ -456,7 +506,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g2.act_rows = A;
   g2.timeout_ns = wait_timeout_ns();
   W4A8_STEP(record(8), "cudaEventRecord");
-  W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, g2, di.sms, s), "down GEMM launch");
+  W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, ts2, g2, di.sms, s), "down GEMM launch");
   W4A8_STEP(record(9), "cudaEventRecord");
 
   W4A8_STEP(record(10), "cudaEventRecord");

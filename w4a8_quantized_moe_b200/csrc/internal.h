@@ -14,12 +14,14 @@ constexpr int kTileNDecode = 32;   // tokens per grouped-GEMM tile, decode shape
 constexpr int kTileNPrefill = 128; // tokens per grouped-GEMM tile, prefill shape
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
+constexpr int kMaxGroups = 64;     // K / 128 per GEMM (K <= 8192)
 
 inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok; }
 
 // ---- kernels_small.cu
+// gsum (nullable): [T, H / 128] sums of the E4M3 values of each 128-wide group.
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
-                             int num_sms, cudaStream_t s);
+                             float* gsum, int num_sms, cudaStream_t s);
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
                              int num_sms, cudaStream_t s);
 // routing: top-k + per-block expert histogram; scan; stable scatter.
@@ -30,7 +32,14 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
                          cudaStream_t s);
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
-                               uint8_t* codes, float* scales, int num_sms, cudaStream_t s);
+                               uint8_t* codes, float* scales, float* gsum, int num_sms,
+                               cudaStream_t s);
+// packed uint4b8 words -> the word-local nibble interleave the grouped GEMM reads.
+cudaError_t launch_repack_int4_b200(const int32_t* in, int64_t nwords, int32_t* out, int num_sms,
+                                    cudaStream_t s);
+// bf16 weight scales [E, rows, G] -> group-major [E, G, rows].
+cudaError_t launch_transpose_scales(const void* in, int64_t E, int64_t rows, int64_t G, void* out,
+                                    int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
                            int64_t H, int k, void* out, int num_sms, cudaStream_t s);
 
@@ -44,7 +53,8 @@ struct GemmArgs {
   const int32_t* tile_prefix;     // [E + 1] prefix of ceil(count / tile width of the shape)
   const int32_t* row_tokens;      // gate/up: sorted_token_ids (gather rows); down: nullptr
   const float* act_scale;         // gate/up: per token [T]; down: per segment row [A]
-  const void* wscale;             // bf16 [E, n_rows, K / 128]
+  const float* act_gsum;          // [rows, K / 128] E4M3 group sums (by token / segment row)
+  const void* wscale;             // bf16 [E, K / 128, n_rows] (group-major)
   float* out;                     // gate/up: h [A, I]; down: Y [A, H]
   int64_t out_ld;
   uint32_t* row_amax;             // gate/up only: float bits of max |h| per segment row
@@ -52,9 +62,11 @@ struct GemmArgs {
   uint64_t timeout_ns;
 };
 // decode = the shape for few tokens per expert (see grouped_gemm.cu).
+// tmap_sc: the group-major weight scales as bytes [E * K / 128, 2 * n_rows],
+// box [K / 128 rows, 128 bytes (gate/up) or 256 bytes (down)].
 cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tmap_w,
-                                const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
-                                cudaStream_t s);
+                                const CUtensorMap& tmap_act, const CUtensorMap& tmap_sc,
+                                const GemmArgs& a, int num_ctas, cudaStream_t s);
 int grouped_gemm_tile_n(bool decode);
 
 }  // namespace w4a8

@@ -2,6 +2,7 @@
 // per-token FP8 activation quantisation, INT4 RTN packing, top-k routing and
 // the expert permutation, the intermediate requantisation, the combine.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -44,6 +45,20 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float scale) {
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
+// Sum of the E4M3 values of the eight codes in c (low byte first).
+__device__ __forceinline__ float sum8_e4m3(uint2 c) {
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t pair = static_cast<uint16_t>(((i < 2 ? c.x : c.y) >> (16 * (i & 1))) & 0xffffu);
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    s += f.x;
+    s += f.y;
+  }
+  return s;
+}
+
 __device__ __forceinline__ void unpack8(uint4 c, float (&v)[8]) {
   v[0] = bf16_lo(c.x); v[1] = bf16_hi(c.x); v[2] = bf16_lo(c.y); v[3] = bf16_hi(c.y);
   v[4] = bf16_lo(c.z); v[5] = bf16_hi(c.z); v[6] = bf16_lo(c.w); v[7] = bf16_hi(c.w);
@@ -65,13 +80,18 @@ __device__ __forceinline__ float warp_sum(float v) {
 // One CTA per token row (grid-stride): absmax over the row, scale = absmax/448,
 // codes = E4M3(x / scale).  Up to kAqCache 16-byte chunks per thread stay in
 // registers between the two passes; longer rows are re-read (L1/L2 hits).
+// Optionally also the sum of the E4M3 values (codes decoded, without the
+// scale) of every 128-wide group, which the grouped GEMM needs because it
+// feeds the weights to the MMA as q + 8 (see grouped_gemm.cu): 16 chunks of 8
+// make a group, held by 16 consecutive threads.
 constexpr int kAqThreads = 256;
 constexpr int kAqCache = 4;
 
 __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat16* __restrict__ x,
                                                                int64_t T, int64_t H,
                                                                uint8_t* __restrict__ codes,
-                                                               float* __restrict__ scales) {
+                                                               float* __restrict__ scales,
+                                                               float* __restrict__ gsum) {
   __shared__ float red[kAqThreads / 32];
   const int64_t nchunk = H / 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,20 +119,35 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
     const float scale = __fdiv_rn(amax, 448.0f);
     if (threadIdx.x == 0) scales[t] = scale;
     uint2* out = reinterpret_cast<uint2*>(codes + t * H);
-#pragma unroll
-    for (int i = 0; i < kAqCache; ++i) {
-      const int64_t c = threadIdx.x + static_cast<int64_t>(i) * kAqThreads;
+    float* gs = gsum ? gsum + t * (H / kGroup) : nullptr;
+    // Every thread runs every chunk slot (the slot bounds are uniform) so that
+    // the 16-lane group reductions see full warps.
+    auto emit = [&](int64_t c, const uint4& raw) {
+      float part = 0.0f;
       if (c < nchunk) {
         float v[8];
-        unpack8(cache[i], v);
-        out[c] = quant8(v, scale);
+        unpack8(raw, v);
+        const uint2 q = quant8(v, scale);
+        out[c] = q;
+        if (gs) part = sum8_e4m3(q);
       }
+      if (gs) {
+        part += __shfl_xor_sync(kFull, part, 8);
+        part += __shfl_xor_sync(kFull, part, 4);
+        part += __shfl_xor_sync(kFull, part, 2);
+        part += __shfl_xor_sync(kFull, part, 1);
+        if (c < nchunk && (c & 15) == 0) gs[c >> 4] = part;
+      }
+    };
+#pragma unroll
+    for (int i = 0; i < kAqCache; ++i) {
+      if (static_cast<int64_t>(i) * kAqThreads >= nchunk) break;
+      emit(threadIdx.x + static_cast<int64_t>(i) * kAqThreads, cache[i]);
     }
-    for (int64_t c = threadIdx.x + static_cast<int64_t>(kAqCache) * kAqThreads; c < nchunk;
-         c += kAqThreads) {
-      float v[8];
-      unpack8(__ldg(row + c), v);
-      out[c] = quant8(v, scale);
+    for (int64_t base = static_cast<int64_t>(kAqCache) * kAqThreads; base < nchunk;
+         base += kAqThreads) {
+      const int64_t c = base + threadIdx.x;
+      emit(c, c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u));
     }
     __syncthreads();  // red[] is reused by the next row
   }
@@ -314,30 +349,83 @@ __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
 
 // ---------------------------------------------------------------- intermediate requant
 // 16 consecutive values of one segment row per thread: scale = amax_r / 448,
-// codes = E4M3(h / scale).
+// codes = E4M3(h / scale), and the sum of the E4M3 values of each 128-wide
+// group (8 consecutive threads).  Whole warps run every iteration so that
+// the group reduction can use shuffles.
 __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restrict__ h,
                                                           const uint32_t* __restrict__ row_amax,
                                                           int64_t A, int64_t I,
                                                           uint8_t* __restrict__ codes,
-                                                          float* __restrict__ scales) {
+                                                          float* __restrict__ scales,
+                                                          float* __restrict__ gsum) {
   const int64_t per_row = I / 16;
   const int64_t n = A * per_row;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t n_iter = (n + stride - 1) / stride;
+  for (int64_t k = 0; k < n_iter; ++k) {
+    const int64_t i = k * stride + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const bool active = i < n;
+    float part = 0.0f;
+    int64_t r = 0, c = 0;
+    if (active) {
+      r = i / per_row;
+      c = i - r * per_row;
+      const float amax = __uint_as_float(__ldg(row_amax + r));
+      const float scale = __fdiv_rn(amax, 448.0f);
+      if (c == 0) scales[r] = scale;
+      const float4* src = reinterpret_cast<const float4*>(h + r * I + c * 16);
+      uint2 out[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const float4 a = __ldg(src + 2 * half), b = __ldg(src + 2 * half + 1);
+        const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        out[half] = quant8(v, scale);
+      }
+      *reinterpret_cast<uint4*>(codes + r * I + c * 16) =
+          make_uint4(out[0].x, out[0].y, out[1].x, out[1].y);
+      if (gsum) part = sum8_e4m3(out[0]) + sum8_e4m3(out[1]);
+    }
+    if (gsum) {
+      part += __shfl_xor_sync(kFull, part, 4);
+      part += __shfl_xor_sync(kFull, part, 2);
+      part += __shfl_xor_sync(kFull, part, 1);
+      if (active && (c & 7) == 0) gsum[r * (I / kGroup) + (c >> 3)] = part;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- B200 weight layout
+// Word-local nibble interleave: element j of each group of 8 moves from
+// nibble j to nibble 2j (j < 4) or 2(j - 4) + 1 (j >= 4), so that w & 0x0F0F0F0F
+// holds elements 0..3 one per byte and (w >> 4) & 0x0F0F0F0F elements 4..7.
+// `in` may equal `out` (each thread reads its word before writing it).
+__global__ void __launch_bounds__(256) repack_int4_b200_kernel(const uint32_t* in, int64_t nwords,
+                                                               uint32_t* out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t w = in[i];
+    uint32_t r = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t nib = (w >> (4 * j)) & 0xFu;
+      const int p = j < 4 ? 2 * j : 2 * (j - 4) + 1;
+      r |= nib << (4 * p);
+    }
+    out[i] = r;
+  }
+}
+
+// [E, rows, G] -> [E, G, rows] (group-major weight scales).
+__global__ void __launch_bounds__(256) transpose_scales_kernel(const uint16_t* __restrict__ in,
+                                                               int64_t E, int64_t rows, int64_t G,
+                                                               uint16_t* __restrict__ out) {
+  const int64_t n = E * G * rows;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / per_row, c = i - r * per_row;
-    const float amax = __uint_as_float(__ldg(row_amax + r));
-    const float scale = __fdiv_rn(amax, 448.0f);
-    if (c == 0) scales[r] = scale;
-    const float4* src = reinterpret_cast<const float4*>(h + r * I + c * 16);
-    uint2 out[2];
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const float4 a = __ldg(src + 2 * half), b = __ldg(src + 2 * half + 1);
-      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      out[half] = quant8(v, scale);
-    }
-    *reinterpret_cast<uint4*>(codes + r * I + c * 16) =
-        make_uint4(out[0].x, out[0].y, out[1].x, out[1].y);
+    const int64_t e = i / (G * rows);
+    const int64_t rem = i - e * G * rows;
+    const int64_t g = rem / rows, r = rem - g * rows;
+    out[i] = __ldg(in + (e * rows + r) * G + g);
   }
 }
 
@@ -384,12 +472,12 @@ inline int grid_for(int64_t work_items, int threads, int num_sms, int per_sm = 8
 }  // namespace
 
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
-                             int num_sms, cudaStream_t s) {
+                             float* gsum, int num_sms, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(T < cap ? T : cap);
   act_quant_kernel<<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, codes,
-                                               scales);
+                                               scales, gsum);
   return cudaGetLastError();
 }
 
@@ -441,10 +529,30 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
 }
 
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
-                               uint8_t* codes, float* scales, int num_sms, cudaStream_t s) {
+                               uint8_t* codes, float* scales, float* gsum, int num_sms,
+                               cudaStream_t s) {
   if (A == 0) return cudaSuccess;
   const int grid = grid_for(A * (I / 16), 256, num_sms);
-  inter_quant_kernel<<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales);
+  inter_quant_kernel<<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, gsum);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_int4_b200(const int32_t* in, int64_t nwords, int32_t* out, int num_sms,
+                                    cudaStream_t s) {
+  if (nwords == 0) return cudaSuccess;
+  const int grid = grid_for(nwords, 256, num_sms, 16);
+  repack_int4_b200_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(in), nwords,
+                                               reinterpret_cast<uint32_t*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_scales(const void* in, int64_t E, int64_t rows, int64_t G, void* out,
+                                    int num_sms, cudaStream_t s) {
+  const int64_t n = E * rows * G;
+  if (n == 0) return cudaSuccess;
+  const int grid = grid_for(n, 256, num_sms, 16);
+  transpose_scales_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(in), E, rows, G,
+                                               static_cast<uint16_t*>(out));
   return cudaGetLastError();
 }
 
