@@ -31,6 +31,8 @@ def _pack_all(cfg, device):
         w13, w2 = workloads.gen_expert_weights(cfg, e, device=device)
         w4.w4a8_pack_int4(w13, packed=p13[e], scales=s13[e])
         w4.w4a8_pack_int4(w2, packed=p2[e], scales=s2[e])
+    p13, s13 = w4.w4a8_prepare_experts_b200(p13, s13, packed_out=p13)
+    p2, s2 = w4.w4a8_prepare_experts_b200(p2, s2, packed_out=p2)
     return w4.W4A8MoELayer(p13, s13, p2, s2, cfg.k)
 
 

@@ -116,6 +116,7 @@ struct ForwardBufs {
   int32_t* row_of;
   RouteBufs route;
   uint8_t* act_codes;
+  uint8_t* perm_codes;
   float* act_scales;
   float* act_gsum;
   float* h;
@@ -136,6 +137,7 @@ ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int
   b.row_of = c.take<int32_t>(A);
   b.route = carve_route(c, T, E);
   b.act_codes = c.take<uint8_t>(static_cast<size_t>(T) * static_cast<size_t>(H));
+  b.perm_codes = c.take<uint8_t>(A * static_cast<size_t>(H));
   b.act_scales = c.take<float>(static_cast<size_t>(T));
   b.act_gsum = c.take<float>(static_cast<size_t>(T) * static_cast<size_t>(H / kGroup));
   b.h = c.take<float>(A * static_cast<size_t>(I));
@@ -276,7 +278,7 @@ w4a8_status w4a8_quant_act_fp8_per_token(const void* x_bf16, int64_t T, int64_t 
     return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   DeviceInfo di;
   if (w4a8_status st = device_info(&di)) return st;
-  cudaError_t err = launch_act_quant(x_bf16, T, H, codes_e4m3, scales, nullptr, di.sms,
+  cudaError_t err = launch_act_quant(x_bf16, T, H, codes_e4m3, scales, nullptr, nullptr, 0, nullptr, di.sms,
                                      static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "act_quant launch");
 }
@@ -416,21 +418,21 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   const int tile_n = grouped_gemm_tile_n(decode);
 
   // TMA descriptors: packed weights [E * rows, K / 2] bytes, 64-byte swizzle;
-  // activation codes [rows, K] bytes, 128-byte swizzle, one-row boxes for gather4.
+  // activation codes in segment order [A, K] bytes, 128-byte swizzle, 16-row boxes.
   CUtensorMap tw1, ta1, tw2, ta2, ts1, ts2;
   if (w4a8_status st = encode_u8_2d(&tw1, w13_packed, static_cast<uint64_t>(H / 2),
                                     static_cast<uint64_t>(E) * 2 * I, 64, 64,
                                     CU_TENSOR_MAP_SWIZZLE_64B))
     return st;
-  if (w4a8_status st = encode_u8_2d(&ta1, b.act_codes, static_cast<uint64_t>(H),
-                                    static_cast<uint64_t>(T), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (w4a8_status st = encode_u8_2d(&ta1, b.perm_codes, static_cast<uint64_t>(H),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
   if (w4a8_status st = encode_u8_2d(&tw2, w2_packed, static_cast<uint64_t>(I / 2),
                                     static_cast<uint64_t>(E) * H, 64, 128,
                                     CU_TENSOR_MAP_SWIZZLE_64B))
     return st;
   if (w4a8_status st = encode_u8_2d(&ta2, b.inter_codes, static_cast<uint64_t>(I),
-                                    static_cast<uint64_t>(A), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
   // group-major scales as bytes: [E * G, 2 * rows]; one box = one tile's scales
   if (w4a8_status st = encode_u8_2d(&ts1, w13_scales, static_cast<uint64_t>(2 * I) * 2,
@@ -452,16 +454,19 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
     if (err != cudaSuccess) return cuda_fail(err, what); \
   } while (0)
 
-  W4A8_STEP(record(0), "cudaEventRecord");
-  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, b.act_gsum, di.sms, s),
-            "act_quant launch");
-  W4A8_STEP(record(1), "cudaEventRecord");
+  // routing first: the activation quantiser writes each token's codes to its
+  // segment rows as well, so both GEMMs read contiguous activation tiles
   W4A8_STEP(record(2), "cudaEventRecord");
   W4A8_STEP(launch_route(logits, T, E, k, b.topk_ids, b.topk_w, b.expert_offsets,
                          b.sorted_token_ids, b.row_of, b.route.block_counts, b.route.block_base,
                          b.route.tile_prefix, tile_n, b.row_amax, s),
             "route launch");
   W4A8_STEP(record(3), "cudaEventRecord");
+  W4A8_STEP(record(0), "cudaEventRecord");
+  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, b.act_gsum, b.row_of, k,
+                             b.perm_codes, di.sms, s),
+            "act_quant launch");
+  W4A8_STEP(record(1), "cudaEventRecord");
 
   GemmArgs g1{};
   g1.K = static_cast<int>(H);

@@ -26,7 +26,9 @@
 //   TMA W warp        packed INT4 box [128 rows x 64 B] (64-byte swizzle)
 //                     into a kWStages ring;
 //   TMA B warp        the activation codes [n rows x 128 B] (128-byte
-//                     swizzle, rows gathered four at a time) into a kBStages ring;
+//                     swizzle) into a kBStages ring; the codes are stored in
+//                     expert-segment order, so a tile's rows are contiguous
+//                     and come as 16-row boxes;
 //   converter warps   each thread owns one weight row: 64 B of nibbles ->
 //                     128 E4M3 bytes, stored straight into a TMEM A slot
 //                     (tcgen05.st); kConvSets sets of 4 warps take turns;
@@ -73,7 +75,7 @@ constexpr int kWStageBytes = kBM * kGroup / 2;      // 8 KB of packed INT4
 constexpr uint32_t kTmemCols = 512;
 
 template <int TileN, int WStages, int BStages, int ASlots, int DBufs, int ConvSets,
-          int EpiPerQuad, int LdCols, int MmaWarps>
+          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets>
 struct Shape {
   static constexpr int kTileN = TileN;
   static constexpr int kWStages = WStages;
@@ -85,7 +87,9 @@ struct Shape {
   static constexpr int kLdCols = LdCols;                  // TMEM columns per tcgen05.ld
   static constexpr int kMmaWarps = MmaWarps;
   static constexpr int kConvWarps = 4 * ConvSets;
-  static constexpr int kEpiWarps = 4 * EpiPerQuad;
+  static constexpr int kEpiSets = EpiSets;                // epilogue sets taking turns by tile
+  static constexpr int kEpiPerSet = 4 * EpiPerQuad;
+  static constexpr int kEpiWarps = kEpiPerSet * EpiSets;
   static constexpr int kWarpW = kConvWarps + kEpiWarps;   // TMA: packed weights
   static constexpr int kWarpMma = kWarpW + 1;             // first MMA issuer
   static constexpr int kWarpB = kWarpMma + MmaWarps;      // TMA: activation rows
@@ -100,14 +104,15 @@ struct Shape {
   static constexpr uint32_t kTmemA = 0;                   // A slots: 32 columns each
   static constexpr uint32_t kTmemD = ASlots * 32;         // accumulators: TileN columns each
   static constexpr int kNumBars = 2 * WStages + 2 * BStages + 2 * ASlots + 2 * DBufs + 3 +
-                                  2 * EpiPerQuad + 2 * kTileScBufs;
+                                  2 * EpiSets * (1 + EpiPerQuad) + 2 * kTileScBufs + 1;
   static_assert(kTmemD + DBufs * TileN <= kTmemCols, "TMEM budget exceeded");
   static_assert(kEpiN % 32 == 0 && kEpiN % LdCols == 0 && (LdCols == 16 || LdCols == 32),
                 "epilogue load width");
   static_assert(TileN % 16 == 0 && TileN <= 256, "MMA N");
   static_assert(MmaWarps == 1 || MmaWarps == 2, "MMA issuers");
-  // Runtime-sized regions (G = K / 128 groups): staged S_g, [kEpiPerQuad][G][kSumLd]
-  // floats, and the tile scales, [kTileScBufs][G][128] bf16.
+  static_assert(EpiSets == 1 || EpiSets == kTileScBufs, "one tile-scale buffer per epilogue set");
+  // Runtime-sized regions (G = K / 128 groups): staged S_g, per set
+  // [kEpiPerQuad][G][kSumLd] floats, and the tile scales, [kTileScBufs][G][128] bf16.
   static constexpr __host__ __device__ int sum_bytes(int G) {
     return (EpiPerQuad * G * kSumLd * 4 + 127) & ~127;
   }
@@ -115,17 +120,20 @@ struct Shape {
   // tile_prefix and expert_offsets, [E + 1] int32 each
   static constexpr __host__ __device__ int table_bytes(int E) { return (8 * (E + 1) + 15) & ~15; }
   static constexpr int smem_bytes(bool gate_up, int G, int E) {
-    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes + (gate_up ? kUpBytes : 0) +
-           sum_bytes(G) + kTileScBufs * tile_sc_bytes(G) + table_bytes(E) + kNumBars * 8 + 16;
+    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes +
+           EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G)) + kTileScBufs * tile_sc_bytes(G) +
+           table_bytes(E) + kNumBars * 8 + 16;
   }
 };
 
 // Shapes, selectable for tuning (W4A8_GEMM_DECODE_SHAPE / W4A8_GEMM_PREFILL_SHAPE).
-//                          TileN        W   B  A  D cvt epi/q ld mma
-using DecodeShape0 = Shape<kTileNDecode, 16, 8, 8, 8, 2, 1, 32, 2>;
-using DecodeShape1 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2>;
-using PrefillShape0 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2>;
-using PrefillShape1 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 32, 2>;
+//                          TileN        W   B  A  D cvt epi/q ld mma sets
+using DecodeShape0 = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2>;
+using DecodeShape1 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1>;
+using DecodeShape2 = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2>;
+using PrefillShape0 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2, 1>;
+using PrefillShape1 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 32, 2, 1>;
+using PrefillShape2 = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1>;
 
 struct Tile {
   int e, mb, n_valid, n_mma;
@@ -207,10 +215,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sW = smem;
   uint8_t* sB = sW + kWStages * kWStageBytes;
-  float* sU = reinterpret_cast<float*>(sB + kBStages * kBStageBytes);
   const int G = a.K / kGroup;
-  float* sS = reinterpret_cast<float*>(sB + kBStages * kBStageBytes + (kGateUp ? kUpBytes : 0));
-  uint8_t* sT = reinterpret_cast<uint8_t*>(sS) + S::sum_bytes(G);
+  // per epilogue set: [sU (gate/up only)][sS]
+  constexpr int kUpPerSet = kGateUp ? kUpBytes : 0;
+  const int set_bytes = kUpPerSet + S::sum_bytes(G);
+  uint8_t* sSet = sB + kBStages * kBStageBytes;
+  uint8_t* sT = sSet + S::kEpiSets * set_bytes;
   int* sTP = reinterpret_cast<int*>(sT + S::kTileScBufs * S::tile_sc_bytes(G));
   int* sEO = sTP + (a.E + 1);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sTP) + S::table_bytes(a.E));
@@ -222,18 +232,21 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   uint64_t* aempty = afull + kASlots;     // [kASlots]  MMAs reading the slot done
   uint64_t* dfull = aempty + kASlots;     // [kDBufs]   group partial sums ready
   uint64_t* dempty = dfull + kDBufs;      // [kDBufs]   epilogue warps read them
-  uint64_t* upfull = dempty + kDBufs;     // up rows staged in sU
-  uint64_t* upempty = upfull + 1;         // sU consumed
-  uint64_t* drain = upempty + 1;          // all MMAs of this CTA complete
-  uint64_t* sfull = drain + 1;            // [kEpiPerQuad] a slice's S_g staged in sS
-  uint64_t* sempty = sfull + S::kEpiPerQuad;  // [kEpiPerQuad] the slice's warps are done
+  uint64_t* upfull = dempty + kDBufs;     // [kEpiSets] up rows staged in the set's sU
+  uint64_t* upempty = upfull + S::kEpiSets;  // [kEpiSets] sU consumed
+  uint64_t* drain = upempty + S::kEpiSets;   // all MMAs of this CTA complete
+  uint64_t* sfull = drain + 1;            // [kEpiSets][kEpiPerQuad] a slice's S_g staged
+  uint64_t* sempty = sfull + S::kEpiSets * S::kEpiPerQuad;  // [..] the slice's warps are done
   if constexpr (S::kUnified) {            // one "group's MMAs done" barrier per slot
     bempty = aempty;
     dfull = aempty;
   }
-  uint64_t* tfull = sempty + S::kEpiPerQuad;   // [kTileScBufs] a tile's weight scales landed
+  uint64_t* tfull = sempty + S::kEpiSets * S::kEpiPerQuad;  // [kTileScBufs] tile scales landed
   uint64_t* tempty = tfull + S::kTileScBufs;    // [kTileScBufs] epilogue warps are done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + S::kTileScBufs);
+  // Group loops run in tile order, one set at a time (completion n = tile n's loop
+  // done), so every wait on the shared accumulator ring stays within one phase.
+  uint64_t* loopdone = tempty + S::kTileScBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(loopdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -255,19 +268,22 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     }
     for (int d = 0; d < kDBufs; ++d) {
       if (!S::kUnified) mbar_init(&dfull[d], 1);
-      mbar_init(&dempty[d], S::kEpiWarps);
+      mbar_init(&dempty[d], S::kEpiPerSet);   // each group is read by one set
     }
-    mbar_init(upfull, S::kEpiWarps / 2);
-    mbar_init(upempty, S::kEpiWarps / 2);
+    for (int i = 0; i < S::kEpiSets; ++i) {
+      mbar_init(&upfull[i], S::kEpiPerSet / 2);
+      mbar_init(&upempty[i], S::kEpiPerSet / 2);
+    }
     mbar_init(drain, S::kMmaWarps);
-    for (int i = 0; i < S::kEpiPerQuad; ++i) {
+    for (int i = 0; i < S::kEpiSets * S::kEpiPerQuad; ++i) {
       mbar_init(&sfull[i], 4);
       mbar_init(&sempty[i], 4);
     }
     for (int i = 0; i < S::kTileScBufs; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], S::kEpiWarps);
+      mbar_init(&tempty[i], S::kEpiPerSet);  // a tile's scales are read by one set
     }
+    mbar_init(loopdone, S::kEpiPerSet);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -343,14 +359,11 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
       const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, tile);
-      int32_t ry[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int64_t r = t.row0 + min(4 * lane + q, t.n_valid - 1);
-        ry[q] = kGateUp ? __ldg(a.row_tokens + r) : static_cast<int32_t>(r);
-      }
-      const int n_ops = t.n_mma >> 2;
+      // the activations are in segment order: the tile's rows are contiguous,
+      // loaded as 16-row boxes (rows past the tensor's end read as zero)
+      const int n_ops = t.n_mma >> 4;
       const uint32_t tx = t.n_mma * kGroup;
+      const int32_t y0 = static_cast<int32_t>(t.row0) + 16 * lane;
       for (int g = 0; g < G; ++g) {
         const int s = it % kBStages;
         const uint32_t ph = (it / kBStages) & 1;
@@ -358,9 +371,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const uint32_t dB = smem_u32(sB + s * kBStageBytes);
         if (lane == 0) mbar_arrive_expect_tx(&bfull[s], tx);
         __syncwarp();
-        if (lane < n_ops)
-          tma_gather4(dB + lane * 4 * kGroup, &tmap_act, &bfull[s], g * kGroup, ry[0], ry[1],
-                      ry[2], ry[3]);
+        if (lane < n_ops) tma_load_2d(dB + lane * 16 * kGroup, &tmap_act, &bfull[s], g * kGroup, y0);
         ++it;
       }
     }
@@ -428,8 +439,10 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       const uint32_t ph = (it / kWStages) & 1;
       const int as = it % kASlots;
       const uint32_t pha = (it / kASlots) & 1;
-      if (!mbar_wait(&wfull[s], ph, abort_flag, tmo) ||
-          !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo))
+      const bool rw = mbar_try_wait(&wfull[s], ph);   // both polls in flight at once
+      const bool ra = mbar_try_wait(&aempty[as], pha ^ 1);
+      if (!(rw && ra) && (!mbar_wait(&wfull[s], ph, abort_flag, tmo) ||
+                          !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo)))
         break;
       tc_fence_after();
       const uint32_t row = smem_u32(sW + s * kWStageBytes) + m * 64;
@@ -455,20 +468,29 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   } else if (warp < S::kWarpW) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - S::kConvWarps;
+    const int set = e / S::kEpiPerSet;              // takes this CTA's tiles set, set + sets, ...
     const int q = warp & 3;                         // TMEM lane quadrant
-    const int slice = e >> 2;                       // column slice of the tile
+    const int slice = (e % S::kEpiPerSet) >> 2;     // column slice of the tile
     const int m = q * 32 + lane;                    // weight row of the tile
     const int j0 = slice * kEpiN;                   // first column (segment row) of this warp
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    float* sSl = sS + slice * G * kSumLd;           // [g][jj] activation group sums of the slice
+    float* sU = reinterpret_cast<float*>(sSet + set * set_bytes);
+    float* sSl = reinterpret_cast<float*>(sSet + set * set_bytes + kUpPerSet) +
+                 slice * G * kSumLd;                // [g][jj] activation group sums of the slice
+    uint64_t* my_sfull = &sfull[set * S::kEpiPerQuad + slice];
+    uint64_t* my_sempty = &sempty[set * S::kEpiPerQuad + slice];
+    uint64_t* my_upfull = &upfull[set];
+    uint64_t* my_upempty = &upempty[set];
     // this row's scale of group g in a tile-scale buffer: [G][64] gate rows
     // then [G][64] up rows (gate/up), or [G][128] rows (down)
     const int sc_off = kGateUp ? (m < 64 ? m : 64 * G + (m - 64)) : m;
     constexpr int kScStride = kGateUp ? 64 : 128;
-    int it = 0, ntile = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++ntile) {
+    for (int tile = blockIdx.x + set * gridDim.x, ntile = set; ok && tile < total;
+         tile += S::kEpiSets * gridDim.x, ntile += S::kEpiSets) {
       const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, tile);
+      int it = ntile * G;                           // CTA-wide index of the tile's first group
+      const uint32_t lt = ntile / S::kEpiSets;      // this set's tile count: barrier phases
       // token (gate/up) or row (down) scales of this warp's columns, lane-strided;
       // loaded now so their latency hides behind the group loop
       float ts[kEpiN / 32];
@@ -482,10 +504,10 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         }
         ts[i] = v;
       }
-      const uint32_t phs = ntile & 1;
+      const uint32_t phs = lt & 1;
       {  // stage S_g of this warp's quarter of the slice's columns: sSl[g][jj]
         constexpr int kTok = kEpiN / 4;
-        if (!mbar_wait(&sempty[slice], phs ^ 1, abort_flag, tmo)) break;
+        if (!mbar_wait(my_sempty, phs ^ 1, abort_flag, tmo)) break;
         constexpr int kBatch = kTok < 8 ? kTok : 8;   // loads in flight per lane
 #pragma unroll
         for (int b0 = 0; b0 < kTok; b0 += kBatch) {
@@ -512,19 +534,23 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sfull[slice]);
+        if (lane == 0) mbar_arrive(my_sfull);
       }
-      if (!mbar_wait(&sfull[slice], phs, abort_flag, tmo)) break;
+      if (!mbar_wait(my_sfull, phs, abort_flag, tmo)) break;
       const int tb = ntile % S::kTileScBufs;
       if (!mbar_wait(&tfull[tb], (ntile / S::kTileScBufs) & 1, abort_flag, tmo)) break;
       const __nv_bfloat16* sTm =
           reinterpret_cast<const __nv_bfloat16*>(sT + tb * S::tile_sc_bytes(G)) + sc_off;
+      if (S::kEpiSets > 1 && ntile > 0 &&
+          !mbar_wait(loopdone, static_cast<uint32_t>(ntile - 1) & 1, abort_flag, tmo))
+        break;
       float acc[kEpiN];
 #pragma unroll
       for (int j = 0; j < kEpiN; ++j) acc[j] = 0.0f;
       for (int g = 0; g < G; ++g) {
         const float sg = __bfloat162float(sTm[g * kScStride]);
-        const float s512 = sg * 512.0f, sm8 = -8.0f * sg;
+        const float2 s512x2 = make_float2(sg * 512.0f, sg * 512.0f);
+        const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
         const float* sg_row = sSl + g * kSumLd;
         const int d = it % kDBufs;
         const uint32_t phd = (it / kDBufs) & 1;
@@ -541,13 +567,18 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < kLdCols; i += 4) {
               const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
-              const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                float x = acc[c * kLdCols + i + u];
-                x = fmaf(s512, __uint_as_float(v[i + u]), x);
-                acc[c * kLdCols + i + u] = fmaf(sm8, sv[u], x);
-              }
+              const int o = c * kLdCols + i;
+              float2 x0 = make_float2(acc[o], acc[o + 1]);
+              float2 x1 = make_float2(acc[o + 2], acc[o + 3]);
+              x0 = ffma2(s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), x0);
+              x1 = ffma2(s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
+                         x1);
+              x0 = ffma2(sm8x2, make_float2(s4.x, s4.y), x0);
+              x1 = ffma2(sm8x2, make_float2(s4.z, s4.w), x1);
+              acc[o] = x0.x;
+              acc[o + 1] = x0.y;
+              acc[o + 2] = x1.x;
+              acc[o + 3] = x1.y;
             }
           }
         }
@@ -559,41 +590,46 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       if (!ok) break;
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sempty[slice]);
+        mbar_arrive(my_sempty);
         mbar_arrive(&tempty[tb]);
+        if (S::kEpiSets > 1) mbar_arrive(loopdone);
       }
       if constexpr (kGateUp) {
-        const uint32_t phu = ntile & 1;
+        const uint32_t phu = lt & 1;
         if (q >= 2) {  // up rows: stage u = acc * token scale for the gate warps
-          if (!mbar_wait(upempty, phu ^ 1, abort_flag, tmo)) break;
+          if (!mbar_wait(my_upempty, phu ^ 1, abort_flag, tmo)) break;
+          // every column, valid or not, so the loop has no branches; the gate
+          // warps ignore the padding columns
 #pragma unroll
           for (int jj = 0; jj < kEpiN; ++jj) {
-            if (j0 + jj < t.n_valid) {
-              const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
-              sU[(j0 + jj) * 64 + (m - 64)] = acc[jj] * tsj;
-            }
+            const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
+            sU[(j0 + jj) * 64 + (m - 64)] = acc[jj] * tsj;
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(upfull);
+          if (lane == 0) mbar_arrive(my_upfull);
         } else {  // gate rows: h = silu(gate) * up, store, row absmax
-          if (!mbar_wait(upfull, phu, abort_flag, tmo)) break;
+          if (!mbar_wait(my_upfull, phu, abort_flag, tmo)) break;
+          // branch-free over the columns (stores predicated) so that the
+          // shuffles, exp and divide of different columns overlap
+          const int n_here = t.n_valid - j0;
 #pragma unroll
           for (int jj = 0; jj < kEpiN; ++jj) {
-            float hm = 0.0f;
-            if (j0 + jj < t.n_valid) {
-              const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
-              const float gt = acc[jj] * tsj;
-              const float u = sU[(j0 + jj) * 64 + m];
-              // silu(g) * u with the fast exp and divide: relative error ~1e-6,
-              // far inside what the FP8 requantisation of h rounds away
-              const float h = __fdividef(gt, 1.0f + __expf(-gt)) * u;
-              a.out[(t.row0 + j0 + jj) * a.out_ld + t.mb * 64 + m] = h;
-              hm = fabsf(h);
-            }
-            acc[jj] = hm;
+            const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
+            const float gt = acc[jj] * tsj;
+            const float u = sU[(j0 + jj) * 64 + m];
+            // silu(g) * u with the fast exp and divide: relative error ~1e-6,
+            // far inside what the FP8 requantisation of h rounds away
+            acc[jj] = __fdividef(gt, 1.0f + __expf(-gt)) * u;
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(upempty);
+          if (lane == 0) mbar_arrive(my_upempty);
+          float* hout = a.out + (t.row0 + j0) * a.out_ld + t.mb * 64 + m;
+#pragma unroll
+          for (int jj = 0; jj < kEpiN; ++jj) {
+            const bool valid = jj < n_here;
+            if (valid) hout[jj * a.out_ld] = acc[jj];
+            acc[jj] = valid ? fabsf(acc[jj]) : 0.0f;
+          }
           // per-column max over this warp's 32 rows: lane l ends with column l
 #pragma unroll
           for (int b = 0; b < kEpiN / 32; ++b) {
@@ -603,12 +639,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           }
         }
       } else {
+        float* yout = a.out + (t.row0 + j0) * a.out_ld + t.mb * kBM + m;
+        const int n_here = t.n_valid - j0;
 #pragma unroll
         for (int jj = 0; jj < kEpiN; ++jj) {
-          if (j0 + jj < t.n_valid) {
-            const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
-            a.out[(t.row0 + j0 + jj) * a.out_ld + t.mb * kBM + m] = acc[jj] * tsj;
-          }
+          const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
+          if (jj < n_here) yout[jj * a.out_ld] = acc[jj] * tsj;
         }
       }
     }
@@ -673,10 +709,14 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
   if (decode) {
     if (dshape == 1)
       return launch_either<DecodeShape1>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    if (dshape == 2)
+      return launch_either<DecodeShape2>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
     return launch_either<DecodeShape0>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
   }
   if (pshape == 1)
     return launch_either<PrefillShape1>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+  if (pshape == 2)
+    return launch_either<PrefillShape2>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
   return launch_either<PrefillShape0>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
 }
 

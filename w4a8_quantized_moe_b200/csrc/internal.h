@@ -20,8 +20,11 @@ inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok;
 
 // ---- kernels_small.cu
 // gsum (nullable): [T, H / 128] sums of the E4M3 values of each 128-wide group.
+// perm (nullable): [T * k, H] codes in expert-segment order; row r = row_of[t, j]
+// receives token t's codes for every slot j.
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
-                             float* gsum, int num_sms, cudaStream_t s);
+                             float* gsum, const int32_t* row_of, int k, uint8_t* perm,
+                             int num_sms, cudaStream_t s);
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
                              int num_sms, cudaStream_t s);
 // routing: top-k + per-block expert histogram; scan; stable scatter.
@@ -51,7 +54,7 @@ struct GemmArgs {
   int E;
   const int32_t* expert_offsets;  // [E + 1]
   const int32_t* tile_prefix;     // [E + 1] prefix of ceil(count / tile width of the shape)
-  const int32_t* row_tokens;      // gate/up: sorted_token_ids (gather rows); down: nullptr
+  const int32_t* row_tokens;      // gate/up: sorted_token_ids (token of each row); down: nullptr
   const float* act_scale;         // gate/up: per token [T]; down: per segment row [A]
   const float* act_gsum;          // [rows, K / 128] E4M3 group sums (by token / segment row)
   const void* wscale;             // bf16 [E, K / 128, n_rows] (group-major)

@@ -91,8 +91,12 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
                                                                int64_t T, int64_t H,
                                                                uint8_t* __restrict__ codes,
                                                                float* __restrict__ scales,
-                                                               float* __restrict__ gsum) {
+                                                               float* __restrict__ gsum,
+                                                               const int32_t* __restrict__ row_of,
+                                                               int k,
+                                                               uint8_t* __restrict__ perm) {
   __shared__ float red[kAqThreads / 32];
+  __shared__ int64_t dst_rows[kMaxTopK];
   const int64_t nchunk = H / 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
@@ -112,6 +116,7 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
       amax = fmaxf(amax, absmax8(__ldg(row + c)));
     amax = warp_max(amax);
     if (lane == 0) red[warp] = amax;
+    if (perm && threadIdx.x < k) dst_rows[threadIdx.x] = __ldg(row_of + t * k + threadIdx.x);
     __syncthreads();
     amax = red[0];
 #pragma unroll
@@ -129,6 +134,8 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
         unpack8(raw, v);
         const uint2 q = quant8(v, scale);
         out[c] = q;
+        if (perm)  // the token's codes again at each of its k segment rows
+          for (int j = 0; j < k; ++j) reinterpret_cast<uint2*>(perm + dst_rows[j] * H)[c] = q;
         if (gs) part = sum8_e4m3(q);
       }
       if (gs) {
@@ -472,12 +479,14 @@ inline int grid_for(int64_t work_items, int threads, int num_sms, int per_sm = 8
 }  // namespace
 
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
-                             float* gsum, int num_sms, cudaStream_t s) {
+                             float* gsum, const int32_t* row_of, int k, uint8_t* perm, int num_sms,
+                             cudaStream_t s) {
   if (T == 0) return cudaSuccess;
+  if (perm && (!row_of || k < 1 || k > kMaxTopK)) return cudaErrorInvalidValue;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(T < cap ? T : cap);
   act_quant_kernel<<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, codes,
-                                               scales, gsum);
+                                               scales, gsum, row_of, k, perm);
   return cudaGetLastError();
 }
 
