@@ -210,6 +210,9 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="run the workload with this many experts instead (a smaller case for "
                          "profiler captures; recorded in config)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with this many tokens instead (a smaller case for "
+                         "profiler captures; recorded in config)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -218,6 +221,8 @@ def main():
     if args.experts:
         cfg = cfg.with_(name=f"{cfg.name}_E{args.experts}", E=args.experts,
                         forced_empty=min(cfg.forced_empty, args.experts // 16))
+    if args.tokens:
+        cfg = cfg.with_(name=f"{cfg.name}_T{args.tokens}", T=args.tokens)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -126,14 +126,15 @@ struct Shape {
   }
 };
 
-// Shapes, selectable for tuning (W4A8_GEMM_DECODE_SHAPE / W4A8_GEMM_PREFILL_SHAPE).
-//                          TileN        W   B  A  D cvt epi/q ld mma sets
-using DecodeShape0 = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2>;
-using DecodeShape1 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1>;
-using DecodeShape2 = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2>;
-using PrefillShape0 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2, 1>;
-using PrefillShape1 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 32, 2, 1>;
-using PrefillShape2 = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1>;
+// Shapes.  By default each projection takes the shape measured fastest for it;
+// W4A8_GEMM_DECODE_SHAPE / W4A8_GEMM_PREFILL_SHAPE = 1, 2, 3 force one for both.
+//                            TileN        W   B  A  D cvt epi/q ld mma sets
+using DecodeOneSet  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1>;
+using DecodeTwoSets = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2>;
+using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2>;
+using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1>;
+using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2, 1>;
+using Prefill8EpiLd32 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 32, 2, 1>;
 
 struct Tile {
   int e, mb, n_valid, n_mma;
@@ -399,9 +400,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const int d = it % kDBufs;
         const uint32_t phd = (it / kDBufs) & 1;
         // poll all three at once (each poll is a ~100-cycle round trip)
-        const bool rd = mbar_try_wait(&dempty[d], phd ^ 1);
-        const bool rb = mbar_try_wait(&bfull[sb], phb);
-        const bool ra = mbar_try_wait(&afull[as], pha);
+        const bool rd = mbar_test_wait(&dempty[d], phd ^ 1);
+        const bool rb = mbar_test_wait(&bfull[sb], phb);
+        const bool ra = mbar_test_wait(&afull[as], pha);
         if (!(rd && rb && ra) &&
             (!mbar_wait(&dempty[d], phd ^ 1, abort_flag, tmo) ||
              !mbar_wait(&bfull[sb], phb, abort_flag, tmo) ||
@@ -439,8 +440,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       const uint32_t ph = (it / kWStages) & 1;
       const int as = it % kASlots;
       const uint32_t pha = (it / kASlots) & 1;
-      const bool rw = mbar_try_wait(&wfull[s], ph);   // both polls in flight at once
-      const bool ra = mbar_try_wait(&aempty[as], pha ^ 1);
+      const bool rw = mbar_test_wait(&wfull[s], ph);   // both polls in flight at once
+      const bool ra = mbar_test_wait(&aempty[as], pha ^ 1);
       if (!(rw && ra) && (!mbar_wait(&wfull[s], ph, abort_flag, tmo) ||
                           !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo)))
         break;
@@ -544,16 +545,16 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       if (S::kEpiSets > 1 && ntile > 0 &&
           !mbar_wait(loopdone, static_cast<uint32_t>(ntile - 1) & 1, abort_flag, tmo))
         break;
-      float acc[kEpiN];
+      float2 acc2[kEpiN / 2];  // column pairs, for the packed two-lane FMA
 #pragma unroll
-      for (int j = 0; j < kEpiN; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < kEpiN / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
+      int d = it % kDBufs;
+      uint32_t phd = (it / kDBufs) & 1;
       for (int g = 0; g < G; ++g) {
         const float sg = __bfloat162float(sTm[g * kScStride]);
         const float2 s512x2 = make_float2(sg * 512.0f, sg * 512.0f);
         const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
         const float* sg_row = sSl + g * kSumLd;
-        const int d = it % kDBufs;
-        const uint32_t phd = (it / kDBufs) & 1;
         if (!mbar_wait(&dfull[d], phd, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr = tmem + lane_base + kTmemD + d * kTileN + j0;
@@ -567,18 +568,14 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < kLdCols; i += 4) {
               const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
-              const int o = c * kLdCols + i;
-              float2 x0 = make_float2(acc[o], acc[o + 1]);
-              float2 x1 = make_float2(acc[o + 2], acc[o + 3]);
-              x0 = ffma2(s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), x0);
-              x1 = ffma2(s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
-                         x1);
-              x0 = ffma2(sm8x2, make_float2(s4.x, s4.y), x0);
-              x1 = ffma2(sm8x2, make_float2(s4.z, s4.w), x1);
-              acc[o] = x0.x;
-              acc[o + 1] = x0.y;
-              acc[o + 2] = x1.x;
-              acc[o + 3] = x1.y;
+              const int o = (c * kLdCols + i) / 2;
+              acc2[o] = __ffma2_rn(
+                  s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
+              acc2[o + 1] = __ffma2_rn(
+                  s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
+                  acc2[o + 1]);
+              acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
+              acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
             }
           }
         }
@@ -586,8 +583,18 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&dempty[d]);
         ++it;
+        if (++d == kDBufs) {  // accumulator ring position, kept incrementally
+          d = 0;
+          phd ^= 1;
+        }
       }
       if (!ok) break;
+      float acc[kEpiN];
+#pragma unroll
+      for (int j = 0; j < kEpiN / 2; ++j) {
+        acc[2 * j] = acc2[j].x;
+        acc[2 * j + 1] = acc2[j].y;
+      }
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(my_sempty);
@@ -620,16 +627,22 @@ __global__ void __launch_bounds__(S::kThreads, 1)
             // silu(g) * u with the fast exp and divide: relative error ~1e-6,
             // far inside what the FP8 requantisation of h rounds away
             acc[jj] = __fdividef(gt, 1.0f + __expf(-gt)) * u;
+            sU[(j0 + jj) * 64 + m] = acc[jj];      // h in place of the u this lane read
           }
+          // h of this warp's 32 rows is 128 contiguous bytes per segment row, in
+          // shared memory and in h: the TMA engine copies them (lane jj: row jj)
+          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(my_upempty);
-          float* hout = a.out + (t.row0 + j0) * a.out_ld + t.mb * 64 + m;
 #pragma unroll
-          for (int jj = 0; jj < kEpiN; ++jj) {
-            const bool valid = jj < n_here;
-            if (valid) hout[jj * a.out_ld] = acc[jj];
-            acc[jj] = valid ? fabsf(acc[jj]) : 0.0f;
+          for (int i = 0; i < kEpiN / 32; ++i) {
+            const int jj = lane + 32 * i;
+            if (jj < n_here)
+              bulk_store_s2g(a.out + (t.row0 + j0 + jj) * a.out_ld + t.mb * 64 + q * 32,
+                             smem_u32(sU + (j0 + jj) * 64 + q * 32), 128);
           }
+          bulk_commit();
+#pragma unroll
+          for (int jj = 0; jj < kEpiN; ++jj) acc[jj] = jj < n_here ? fabsf(acc[jj]) : 0.0f;
           // per-column max over this warp's 32 rows: lane l ends with column l
 #pragma unroll
           for (int b = 0; b < kEpiN / 32; ++b) {
@@ -637,6 +650,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
             const int j = j0 + b * 32 + lane;
             if (j < t.n_valid) atomicMax(a.row_amax + t.row0 + j, __float_as_uint(hm));
           }
+          bulk_wait_read_all();                     // sU may be refilled after this
+          __syncwarp();
+          if (lane == 0) mbar_arrive(my_upempty);
         }
       } else {
         float* yout = a.out + (t.row0 + j0) * a.out_ld + t.mb * kBM + m;
@@ -648,6 +664,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         }
       }
     }
+    if constexpr (kGateUp) bulk_wait_all();       // h copies complete before the CTA exits
   }
   // the remaining warps have no role
 
@@ -707,17 +724,19 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
   static const int pshape = shape_choice("W4A8_GEMM_PREFILL_SHAPE");
   if (a.K % kGroup || a.K / kGroup > kMaxGroups || a.K <= 0) return cudaErrorInvalidValue;
   if (decode) {
-    if (dshape == 1)
-      return launch_either<DecodeShape1>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
-    if (dshape == 2)
-      return launch_either<DecodeShape2>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
-    return launch_either<DecodeShape0>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    // gate/up (48 groups per tile at H = 6144) runs best with one epilogue set
+    // and a deep weight ring; down (16 groups per tile) with two epilogue sets,
+    // whose tile finalize then overlaps the other set's groups
+    const int d = dshape != 0 ? dshape : (gate_up ? 1 : 2);
+    if (d == 1) return launch_either<DecodeOneSet>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    if (d == 3) return launch_either<DecodeTwoCvt>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    return launch_either<DecodeTwoSets>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
   }
-  if (pshape == 1)
-    return launch_either<PrefillShape1>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
-  if (pshape == 2)
-    return launch_either<PrefillShape2>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
-  return launch_either<PrefillShape0>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+  const int p = pshape != 0 ? pshape : 1;
+  if (p == 2) return launch_either<Prefill8Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+  if (p == 3)
+    return launch_either<Prefill8EpiLd32>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+  return launch_either<Prefill16Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
 }
 
 cudaError_t read_and_clear_device_error(int* value) {
