@@ -17,7 +17,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
+import hashlib
 import sys
 import time
 
@@ -44,54 +44,69 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples during the timed region."""
+    """SM clock and clock-event reasons sampled during the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NVML is polled from a thread every ~2 ms (the timed region of a short run is
+    only tens of milliseconds); the device is found by its PCI bus id, so the
+    sample is of the GPU this process runs on whatever CUDA_VISIBLE_DEVICES is.
+    """
 
-    def __init__(self, gpu_index: int):
-        self.gpu_index = gpu_index
-        self.proc = None
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device: torch.device, period_s: float = 0.002):
+        self.device, self.period_s = device, period_s
+        self.samples, self.max_mhz, self.reasons, self.err = [], None, set(), None
+        self._stop = None
+
+    def _handle(self, nv):
+        try:
+            p = torch.cuda.get_device_properties(self.device)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.device.index or 0)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report no samples rather than guess
+            self.err = f"{type(e).__name__}: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while True:
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.reasons.update(n for n, b in self.REASONS.items() if r & b)
+                except Exception as e:
+                    self.err = f"{type(e).__name__}: {e}"
+                    return
+                if self._stop.wait(self.period_s):
+                    return
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+               "samples": len(self.samples), "source": "nvml"}
+        if self.err:
+            out["error"] = self.err
+        return out
 
 
 def build_layer(cfg, device, w4):
@@ -110,6 +125,28 @@ def build_layer(cfg, device, w4):
     torch.cuda.synchronize(device)
     del s13, s2
     return w4.W4A8MoELayer(p13, s13g, p2, s2g, cfg.k)
+
+
+def kernel_source_id() -> str:
+    """Git blob id of the grouped GEMM source, which keys the DRAM traffic records."""
+    path = os.path.join(ROOT, "w4a8_quantized_moe_b200", "csrc", "grouped_gemm.cu")
+    data = open(path, "rb").read()
+    return hashlib.sha1(b"blob %d\0" % len(data) + data).hexdigest()
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch from the ncu record in
+    profiles/dram_traffic.txt, or None when there is none for this workload and
+    kernel or the kernel source has changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sid = kernel_source_id()
+    for ln in open(path):
+        f = ln.split()
+        if len(f) == 4 and not ln.startswith("#") and f[0] == workload and f[1] == kernel:
+            return float(f[2]) if f[3] == sid else None
+    return None
 
 
 def algorithmic_work(cfg, counts):
@@ -269,7 +306,7 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
-    with ClockSampler(local) as clk:
+    with ClockSampler(device) as clk:
         t_start.record(stream)
         for i in range(args.steps):
             step(ev[i])
@@ -328,13 +365,14 @@ def main():
         achieved = work["flops"] / (stage_ms[gi] / 1e3) / 1e12
         peak = 2.0 * pk["bf16_sus"]                     # FP8 = 2 x bf16 (nominal ratio)
         roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
-                    frac=achieved / peak, traffic=None, kernel=kname,
+                    frac=achieved / peak, traffic=recorded_traffic(cfg.name, kname), kernel=kname,
                     peak_source=f"{pk['src']} sustained bf16 x 2")
     else:
         achieved = work["bytes"] / (stage_ms[gi] / 1e3) / 1e9
         peak = pk["hbm"]
         roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
-                    traffic=None, kernel=kname, peak_source=f"{pk['src']} HBM copy")
+                    traffic=recorded_traffic(cfg.name, kname), kernel=kname,
+                    peak_source=f"{pk['src']} HBM copy")
 
     line = dict(
         metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,

@@ -182,6 +182,17 @@ w4a8_status encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uin
   return W4A8_OK;
 }
 
+// Tile order within an expert: token blocks fastest for the wide (prefill)
+// tiles, where several token blocks share each weight-row block;
+// W4A8_TILE_ORDER = 0 / 1 forces weight-block-major / token-block-fastest.
+int tile_order_nb_fastest(bool decode) {
+  static const int forced = [] {
+    const char* s = std::getenv("W4A8_TILE_ORDER");
+    return s ? std::atoi(s) : -1;
+  }();
+  return forced >= 0 ? (forced != 0) : (decode ? 0 : 1);
+}
+
 // Average tokens per expert up to which w4a8_moe_forward uses the decode shape.
 constexpr int kDecodeTokensPerExpert = 32;
 
@@ -484,6 +495,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g1.row_amax = b.row_amax;
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
+  g1.nb_fastest = tile_order_nb_fastest(decode);
   W4A8_STEP(record(4), "cudaEventRecord");
   W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, g1, di.sms, s), "gate/up GEMM launch");
   W4A8_STEP(record(5), "cudaEventRecord");
@@ -510,6 +522,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g2.row_amax = nullptr;
   g2.act_rows = A;
   g2.timeout_ns = wait_timeout_ns();
+  g2.nb_fastest = tile_order_nb_fastest(decode);
   W4A8_STEP(record(8), "cudaEventRecord");
   W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, ts2, g2, di.sms, s), "down GEMM launch");
   W4A8_STEP(record(9), "cudaEventRecord");

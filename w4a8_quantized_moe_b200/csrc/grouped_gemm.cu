@@ -141,17 +141,19 @@ struct Tile {
   int64_t row0;
 };
 
-// Linear tile index -> (expert, weight-row block, segment rows).  Tiles are
-// ordered by global token block, then weight-row block, so CTAs running at
-// the same time share one activation block through L2.  tile_prefix and
-// expert_offsets are read from the CTA's shared copies (sTP, sEO): the
-// binary search is a chain of dependent loads.
+// Linear tile index -> (expert, weight-row block, segment rows).  An expert's
+// tiles are consecutive.  Within an expert they run weight-row block major
+// (nb_fastest = 0: the weight-row blocks that share one token block are
+// neighbours) or token block fastest (nb_fastest = 1: the token blocks that
+// share one weight-row block are neighbours), so that CTAs running at the
+// same time share operands through L2.  tile_prefix and expert_offsets are
+// read from the CTA's shared copies (sTP, sEO): the binary search is a chain of
+// dependent loads.
 template <int TileN>
 __device__ __forceinline__ Tile decode_tile(const int* sTP, const int* sEO, int E, int mb_count,
-                                            int idx) {
-  const int nbg = idx / mb_count;
+                                            int nb_fastest, int idx) {
+  const int nbg = idx / mb_count;  // global token block of the idx's expert range
   Tile t;
-  t.mb = idx - nbg * mb_count;
   int lo = 0, hi = E;  // tile_prefix[lo] <= nbg < tile_prefix[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -159,7 +161,16 @@ __device__ __forceinline__ Tile decode_tile(const int* sTP, const int* sEO, int 
     else hi = mid;
   }
   t.e = lo;
-  const int nb = nbg - sTP[lo];
+  const int local = idx - sTP[lo] * mb_count;
+  int nb;
+  if (nb_fastest) {
+    const int ne = sTP[lo + 1] - sTP[lo];
+    t.mb = local / ne;
+    nb = local - t.mb * ne;
+  } else {
+    nb = local / mb_count;
+    t.mb = local - nb * mb_count;
+  }
   const int seg0 = sEO[lo];
   const int cnt = sEO[lo + 1] - seg0;
   t.row0 = static_cast<int64_t>(seg0) + static_cast<int64_t>(nb) * TileN;
@@ -315,7 +326,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       int it = 0, nt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++nt) {
-        const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, tile);
+        const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
         const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
         const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
         {  // the tile's weight scales: box [G groups x 128 (or 2 x 64) rows] of bf16
@@ -359,7 +370,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, tile);
+      const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
       // the activations are in segment order: the tile's rows are contiguous,
       // loaded as 16-row boxes (rows past the tensor's end read as zero)
       const int n_ops = t.n_mma >> 4;
@@ -390,7 +401,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const int tl = it / G;
         if (tl != cur) {
           cur = tl;
-          const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, blockIdx.x + tl * gridDim.x);
+          const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, blockIdx.x + tl * gridDim.x);
           idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
         }
         const int sb = it % kBStages;
@@ -489,7 +500,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x + set * gridDim.x, ntile = set; ok && tile < total;
          tile += S::kEpiSets * gridDim.x, ntile += S::kEpiSets) {
-      const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, tile);
+      const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
       int it = ntile * G;                           // CTA-wide index of the tile's first group
       const uint32_t lt = ntile / S::kEpiSets;      // this set's tile count: barrier phases
       // token (gate/up) or row (down) scales of this warp's columns, lane-strided;

@@ -62,6 +62,7 @@ struct GemmArgs {
   int64_t out_ld;
   uint32_t* row_amax;             // gate/up only: float bits of max |h| per segment row
   int64_t act_rows;               // rows of the activation tensor (T or A)
+  int nb_fastest;                 // tile order within an expert (see grouped_gemm.cu)
   uint64_t timeout_ns;
 };
 // decode = the shape for few tokens per expert (see grouped_gemm.cu).
