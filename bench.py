@@ -127,6 +127,19 @@ def build_layer(cfg, device, w4):
     return w4.W4A8MoELayer(p13, s13g, p2, s2g, cfg.k)
 
 
+def max_over_ranks(dist, values, device):
+    """Element-wise max over all ranks of a list of timings (every rank calls it,
+    at the same point): the job is as slow as its slowest rank."""
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def whole_job_throughput(tokens_per_rank: int, world: int, steps: int, ms: float) -> float:
+    """Tokens of all ranks over all timed steps per second of the (max-over-ranks) time."""
+    return tokens_per_rank * world * steps / (ms / 1e3)
+
+
 def kernel_source_id() -> str:
     """Git blob id of the grouped GEMM source, which keys the DRAM traffic records."""
     path = os.path.join(ROOT, "w4a8_quantized_moe_b200", "csrc", "grouped_gemm.cu")
@@ -346,14 +359,10 @@ def main():
     e2e_ms = e_start.elapsed_time(e_end)
 
     if dist:
-        t = torch.tensor([ms, e2e_ms] + stage_ms, device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-        stage_ms = [float(x) for x in t[2:]]
+        ms, e2e_ms, *stage_ms = max_over_ranks(dist, [ms, e2e_ms] + stage_ms, device)
 
-    tokens = cfg.T * world * args.steps
-    value = tokens / (ms / 1e3)
-    e2e_value = tokens / (e2e_ms / 1e3)
+    value = whole_job_throughput(cfg.T, world, args.steps, ms)
+    e2e_value = whole_job_throughput(cfg.T, world, args.steps, e2e_ms)
 
     pk = peaks()
     g1, g2, active = algorithmic_work(cfg, counts)

@@ -73,6 +73,18 @@ W4A8_API const char* w4a8_last_error(void);
 W4A8_API w4a8_status w4a8_check_device_error(void* stream);
 
 /*
+ * w4a8_selftest_wait_timeout - exercise the failure-detection path.  Launches
+ * one thread that waits, with the bounded wait every grouped-GEMM role uses,
+ * on a barrier that nothing ever arrives on.  After timeout_ns the wait gives
+ * up and raises the device latch, so the next w4a8_check_device_error on the
+ * stream returns W4A8_ERR_DEVICE_TIMEOUT (and clears the latch).  Nothing
+ * traps or faults; the context stays usable.  No counterpart on the pages.
+ *
+ *   timeout_ns  0 < timeout_ns <= 10 s (else W4A8_ERR_INVALID_ARG)
+ */
+W4A8_API w4a8_status w4a8_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/*
  * w4a8_pack_int4 - symmetric INT4 round-to-nearest weight quantisation with
  * one bf16 scale per group of `group` weights along K, packed as uint4b8.
  * (GLM-5.3-W4A8 model card, "quantisation method": symmetric INT4, group

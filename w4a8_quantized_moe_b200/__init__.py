@@ -52,6 +52,7 @@ def _declare(L):
         "w4a8_status_string": (ctypes.c_char_p, [i32]),
         "w4a8_last_error": (ctypes.c_char_p, []),
         "w4a8_check_device_error": (i32, [vp]),
+        "w4a8_selftest_wait_timeout": (i32, [ctypes.c_uint64, vp]),
         "w4a8_pack_int4": (i32, [vp, i64, i64, i32, vp, vp, vp]),
         "w4a8_prepare_experts_b200": (i32, [vp, vp, i64, i64, i64, vp, vp, vp]),
         "w4a8_quant_act_fp8_per_token": (i32, [vp, i64, i64, vp, vp, vp]),
@@ -126,6 +127,14 @@ def w4a8_check_device_error(device=None):
     """Synchronise the current stream and raise if a bounded in-kernel wait ran out."""
     dev = torch.device("cuda") if device is None else torch.device(device)
     _check("w4a8_check_device_error", lib().w4a8_check_device_error(_stream(dev)))
+
+
+def w4a8_selftest_wait_timeout(timeout_s: float = 0.05, device=None):
+    """Launch a bounded wait that nothing satisfies; the next
+    ``w4a8_check_device_error`` then raises W4A8_ERR_DEVICE_TIMEOUT."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check("w4a8_selftest_wait_timeout",
+           lib().w4a8_selftest_wait_timeout(int(timeout_s * 1e9), _stream(dev)))
 
 
 def w4a8_pack_int4(w: torch.Tensor, group: int = 128, packed: Optional[torch.Tensor] = None,

@@ -259,6 +259,16 @@ w4a8_status w4a8_check_device_error(void* stream) {
   return W4A8_OK;
 }
 
+w4a8_status w4a8_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+    return fail(W4A8_ERR_INVALID_ARG, "timeout_ns = %llu; need 0 < timeout_ns <= 10 s",
+                static_cast<unsigned long long>(timeout_ns));
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_wait_timeout_selftest(timeout_ns, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "self-test launch");
+}
+
 w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, int32_t group,
                            int32_t* packed, void* scales_bf16, void* stream) {
   if (group != kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "group = %d; only 128", group);

@@ -750,6 +750,30 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
   return launch_either<Prefill16Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
 }
 
+namespace {
+
+// Failure-detection self-test: one thread waits, with the same bounded wait
+// the GEMM roles use, on an mbarrier that nothing ever arrives on.  The wait
+// gives up after timeout_ns, raising the device latch; nothing faults or hangs.
+__global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_ns);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, cudaStream_t s) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(timeout_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_device_error(int* value) {
   int v = 0;
   cudaError_t err = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));

@@ -72,5 +72,7 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
                                 const CUtensorMap& tmap_act, const CUtensorMap& tmap_sc,
                                 const GemmArgs& a, int num_ctas, cudaStream_t s);
 int grouped_gemm_tile_n(bool decode);
+// One bounded wait on an mbarrier nothing arrives on (failure-detection self-test).
+cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
 
 }  // namespace w4a8
