@@ -75,7 +75,7 @@ constexpr int kWStageBytes = kBM * kGroup / 2;      // 8 KB of packed INT4
 constexpr uint32_t kTmemCols = 512;
 
 template <int TileN, int WStages, int BStages, int ASlots, int DBufs, int ConvSets,
-          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets>
+          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetInMma>
 struct Shape {
   static constexpr int kTileN = TileN;
   static constexpr int kWStages = WStages;
@@ -88,6 +88,10 @@ struct Shape {
   static constexpr int kMmaWarps = MmaWarps;
   static constexpr int kConvWarps = 4 * ConvSets;
   static constexpr int kEpiSets = EpiSets;                // epilogue sets taking turns by tile
+  // The +8 offset of the stored nibbles is removed by the tensor core (four more
+  // MMAs per group against a constant -2^-6 operand) instead of by the epilogue.
+  static constexpr bool kOffsetInMma = OffsetInMma != 0;
+  static constexpr int kConstABytes = kOffsetInMma ? 128 * 128 : 0;  // 128 rows x 128 B
   static constexpr int kEpiPerSet = 4 * EpiPerQuad;
   static constexpr int kEpiWarps = kEpiPerSet * EpiSets;
   static constexpr int kWarpW = kConvWarps + kEpiWarps;   // TMA: packed weights
@@ -114,13 +118,13 @@ struct Shape {
   // Runtime-sized regions (G = K / 128 groups): staged S_g, per set
   // [kEpiPerQuad][G][kSumLd] floats, and the tile scales, [kTileScBufs][G][128] bf16.
   static constexpr __host__ __device__ int sum_bytes(int G) {
-    return (EpiPerQuad * G * kSumLd * 4 + 127) & ~127;
+    return kOffsetInMma ? 0 : (EpiPerQuad * G * kSumLd * 4 + 127) & ~127;
   }
   static constexpr __host__ __device__ int tile_sc_bytes(int G) { return 256 * G; }
   // tile_prefix and expert_offsets, [E + 1] int32 each
   static constexpr __host__ __device__ int table_bytes(int E) { return (8 * (E + 1) + 15) & ~15; }
   static constexpr int smem_bytes(bool gate_up, int G, int E) {
-    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes +
+    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes + kConstABytes +
            EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G)) + kTileScBufs * tile_sc_bytes(G) +
            table_bytes(E) + kNumBars * 8 + 16;
   }
@@ -128,13 +132,13 @@ struct Shape {
 
 // Shapes.  By default each projection takes the shape measured fastest for it;
 // W4A8_GEMM_DECODE_SHAPE / W4A8_GEMM_PREFILL_SHAPE = 1, 2, 3 force one for both.
-//                            TileN        W   B  A  D cvt epi/q ld mma sets
-using DecodeOneSet  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1>;
-using DecodeTwoSets = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2>;
-using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2>;
-using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1>;
-using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2, 1>;
-using Prefill8EpiLd32 = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 32, 2, 1>;
+//                            TileN        W   B  A  D cvt epi/q ld mma sets offset-in-MMA
+using DecodeOneSet  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;
+using DecodeTwoSets = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2, 0>;
+using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2, 0>;
+using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 1>;
+using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2, 1, 1>;
+using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
 
 struct Tile {
   int e, mb, n_valid, n_mma;
@@ -231,7 +235,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   // per epilogue set: [sU (gate/up only)][sS]
   constexpr int kUpPerSet = kGateUp ? kUpBytes : 0;
   const int set_bytes = kUpPerSet + S::sum_bytes(G);
-  uint8_t* sSet = sB + kBStages * kBStageBytes;
+  uint8_t* sConstA = sB + kBStages * kBStageBytes;  // 1024-aligned; bytes 0x88 = E4M3 -2^-6
+  uint8_t* sSet = sConstA + S::kConstABytes;
   uint8_t* sT = sSet + S::kEpiSets * set_bytes;
   int* sTP = reinterpret_cast<int*>(sT + S::kTileScBufs * S::tile_sc_bytes(G));
   int* sEO = sTP + (a.E + 1);
@@ -311,6 +316,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
     sTP[i] = __ldg(a.tile_prefix + i);
     sEO[i] = __ldg(a.expert_offsets + i);
+  }
+  if constexpr (S::kOffsetInMma) {
+    for (int i = threadIdx.x; i < S::kConstABytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(sConstA)[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u,
+                                                        0x88888888u);
+    fence_proxy_async_smem();  // the MMA reads it through the async proxy
   }
   tc_fence_before();
   __syncthreads();
@@ -424,9 +435,17 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const uint32_t dt = tmem + kTmemD + d * kTileN;
         const uint32_t at = tmem + kTmemA + as * 32;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // K = 32 E4M3 per MMA: 8 TMEM columns, 32 B of smem
+        for (int kk = 0; kk < 4; ++kk) {  // K = 32 E4M3 per MMA: 8 TMEM columns, 32 B of smem
           mma_f8_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
                     kk > 0 ? 1u : 0u);
+          if constexpr (S::kOffsetInMma) {
+            // D += sum_k a_k * (-2^-6) over the same 32 k: after each pair D holds
+            // 2^-9 * sum a * q of the slices so far, so the offset cancels at the
+            // magnitude of a 32-element partial sum, not of the whole group
+            mma_f8_ss(dt, sdesc_kmajor_sw128(smem_u32(sConstA)) + static_cast<uint64_t>(kk * 2),
+                      bdesc + static_cast<uint64_t>(kk * 2), idesc, 1u);
+          }
+        }
         if constexpr (S::kUnified) {
           tc_commit(&aempty[as]);               // A slot, B stage and accumulator at once
         } else {
@@ -517,7 +536,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         ts[i] = v;
       }
       const uint32_t phs = lt & 1;
-      {  // stage S_g of this warp's quarter of the slice's columns: sSl[g][jj]
+      if constexpr (!S::kOffsetInMma) {  // stage S_g of this warp's quarter of the slice's columns
         constexpr int kTok = kEpiN / 4;
         if (!mbar_wait(my_sempty, phs ^ 1, abort_flag, tmo)) break;
         constexpr int kBatch = kTok < 8 ? kTok : 8;   // loads in flight per lane
@@ -548,7 +567,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(my_sfull);
       }
-      if (!mbar_wait(my_sfull, phs, abort_flag, tmo)) break;
+      if (!S::kOffsetInMma && !mbar_wait(my_sfull, phs, abort_flag, tmo)) break;
       const int tb = ntile % S::kTileScBufs;
       if (!mbar_wait(&tfull[tb], (ntile / S::kTileScBufs) & 1, abort_flag, tmo)) break;
       const __nv_bfloat16* sTm =
@@ -578,15 +597,17 @@ __global__ void __launch_bounds__(S::kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < kLdCols; i += 4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
               const int o = (c * kLdCols + i) / 2;
               acc2[o] = __ffma2_rn(
                   s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
               acc2[o + 1] = __ffma2_rn(
                   s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
                   acc2[o + 1]);
-              acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
-              acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
+              if constexpr (!S::kOffsetInMma) {  // remove the +8 offset: - 8 s_g S_g
+                const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
+                acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
+                acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
+              }
             }
           }
         }
@@ -608,7 +629,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(my_sempty);
+        if (!S::kOffsetInMma) mbar_arrive(my_sempty);
         mbar_arrive(&tempty[tb]);
         if (S::kEpiSets > 1) mbar_arrive(loopdone);
       }
@@ -746,7 +767,8 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
   const int p = pshape != 0 ? pshape : 1;
   if (p == 2) return launch_either<Prefill8Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
   if (p == 3)
-    return launch_either<Prefill8EpiLd32>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    return launch_either<Prefill16EpiEpilogueOffset>(gate_up, tmap_w, tmap_act, tmap_sc, a,
+                                                     num_ctas, s);
   return launch_either<Prefill16Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
 }
 
