@@ -91,7 +91,6 @@ struct Shape {
   // The +8 offset of the stored nibbles is removed by the tensor core (four more
   // MMAs per group against a constant -2^-6 operand) instead of by the epilogue.
   static constexpr bool kOffsetInMma = OffsetInMma != 0;
-  static constexpr int kConstABytes = kOffsetInMma ? 128 * 128 : 0;  // 128 rows x 128 B
   static constexpr int kEpiPerSet = 4 * EpiPerQuad;
   static constexpr int kEpiWarps = kEpiPerSet * EpiSets;
   static constexpr int kWarpW = kConvWarps + kEpiWarps;   // TMA: packed weights
@@ -106,7 +105,8 @@ struct Shape {
   static constexpr int kSumLd = kEpiN + 4;                // padded: 4-way bank spread on stores
   static constexpr int kTileScBufs = 2;                   // tile weight-scale buffers
   static constexpr uint32_t kTmemA = 0;                   // A slots: 32 columns each
-  static constexpr uint32_t kTmemD = ASlots * 32;         // accumulators: TileN columns each
+  static constexpr uint32_t kTmemConst = ASlots * 32;     // E4M3 -2^-6 in every byte (offset MMAs)
+  static constexpr uint32_t kTmemD = kTmemConst + (OffsetInMma ? 32 : 0);  // TileN columns each
   static constexpr int kNumBars = 2 * WStages + 2 * BStages + 2 * ASlots + 2 * DBufs + 3 +
                                   2 * EpiSets * (1 + EpiPerQuad) + 2 * kTileScBufs + 1;
   static_assert(kTmemD + DBufs * TileN <= kTmemCols, "TMEM budget exceeded");
@@ -124,7 +124,7 @@ struct Shape {
   // tile_prefix and expert_offsets, [E + 1] int32 each
   static constexpr __host__ __device__ int table_bytes(int E) { return (8 * (E + 1) + 15) & ~15; }
   static constexpr int smem_bytes(bool gate_up, int G, int E) {
-    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes + kConstABytes +
+    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes +
            EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G)) + kTileScBufs * tile_sc_bytes(G) +
            table_bytes(E) + kNumBars * 8 + 16;
   }
@@ -136,8 +136,8 @@ struct Shape {
 using DecodeOneSet  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;
 using DecodeTwoSets = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2, 0>;
 using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2, 0>;
-using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 1>;
-using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 4, 2, 1, 2, 16, 2, 1, 1>;
+using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 3, 3, 1, 4, 16, 2, 1, 1>;
+using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 3, 2, 1, 2, 16, 2, 1, 1>;
 using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
 
 struct Tile {
@@ -235,8 +235,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   // per epilogue set: [sU (gate/up only)][sS]
   constexpr int kUpPerSet = kGateUp ? kUpBytes : 0;
   const int set_bytes = kUpPerSet + S::sum_bytes(G);
-  uint8_t* sConstA = sB + kBStages * kBStageBytes;  // 1024-aligned; bytes 0x88 = E4M3 -2^-6
-  uint8_t* sSet = sConstA + S::kConstABytes;
+  uint8_t* sSet = sB + kBStages * kBStageBytes;
   uint8_t* sT = sSet + S::kEpiSets * set_bytes;
   int* sTP = reinterpret_cast<int*>(sT + S::kTileScBufs * S::tile_sc_bytes(G));
   int* sEO = sTP + (a.E + 1);
@@ -316,12 +315,6 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
     sTP[i] = __ldg(a.tile_prefix + i);
     sEO[i] = __ldg(a.expert_offsets + i);
-  }
-  if constexpr (S::kOffsetInMma) {
-    for (int i = threadIdx.x; i < S::kConstABytes / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(sConstA)[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u,
-                                                        0x88888888u);
-    fence_proxy_async_smem();  // the MMA reads it through the async proxy
   }
   tc_fence_before();
   __syncthreads();
@@ -439,11 +432,11 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           mma_f8_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
                     kk > 0 ? 1u : 0u);
           if constexpr (S::kOffsetInMma) {
-            // D += sum_k a_k * (-2^-6) over the same 32 k: after each pair D holds
-            // 2^-9 * sum a * q of the slices so far, so the offset cancels at the
-            // magnitude of a 32-element partial sum, not of the whole group
-            mma_f8_ss(dt, sdesc_kmajor_sw128(smem_u32(sConstA)) + static_cast<uint64_t>(kk * 2),
-                      bdesc + static_cast<uint64_t>(kk * 2), idesc, 1u);
+            // D += sum_k a_k * (-2^-6) over the same 32 k (A = the constant TMEM
+            // columns): after each pair D holds 2^-9 * sum a * q of the slices so
+            // far, so the offset cancels at the magnitude of a 32-element partial
+            // sum, not of the whole group
+            mma_f8_ts(dt, tmem + S::kTmemConst, bdesc + static_cast<uint64_t>(kk * 2), idesc, 1u);
           }
         }
         if constexpr (S::kUnified) {
@@ -465,6 +458,16 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     const int m = quad * 32 + lane;                 // weight row of the tile = TMEM lane
     const uint32_t swz = (m >> 1) & 3;              // 64-byte swizzle of the TMA box
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    if (S::kOffsetInMma && set == 0) {
+      // the constant A operand of the offset MMAs; the MMA warps first read it
+      // after this set's first afull arrival, which follows these stores
+      uint32_t c[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) c[i] = 0x88888888u;  // E4M3 0x88 = -2^-6
+      tmem_st_32x32b_x32(tmem + lane_base + S::kTmemConst, c);
+      tmem_wait_st();
+      tc_fence_before();
+    }
     for (int it = set; it < n_groups; it += S::kConvSets) {
       const int s = it % kWStages;
       const uint32_t ph = (it / kWStages) & 1;

@@ -154,17 +154,6 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// D (TMEM) (+)= A (SMEM descriptor) x B (SMEM descriptor), kind::f8f6f4.
-__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Instruction descriptor: kind::f8f6f4, A = B = E4M3, D = F32, both K-major,
 // M = 128, N = n (multiple of 16, 16..256).
 __host__ __device__ __forceinline__ uint32_t idesc_e4m3_f32_m128(uint32_t n) {
