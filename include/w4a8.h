@@ -105,6 +105,27 @@ W4A8_API w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, in
                            int32_t* packed, void* scales_bf16, void* stream);
 
 /*
+ * w4a8_pack_int4_mse_clip - as w4a8_pack_int4 (same uint4b8 words, same bf16
+ * scale layout, read the same way by w4a8_prepare_experts_b200 and
+ * w4a8_moe_forward), but each group's scale is chosen by the per-group MSE
+ * clip search of the GLM-5.3-W4A8 model card ("quantisation method": 11 shrink
+ * ratios from 1.00 to 0.70, the MSE-optimal scale kept).
+ *
+ * For r_i = float32((100 - 3 i) / 100), i = 0..10:
+ *   s_i = bf16(float32(float32(absmax * r_i) / 7));
+ *   q_i = clamp(rint(float32(w / s_i)), -8, 7) (0 when s_i == 0);
+ *   e_i = sum over the group of (w - q_i * s_i)^2 in float64, summed in this
+ *         order: runs of 4 consecutive elements in sequence, then five
+ *         pairwise combinations of the 32 partial sums (element index xor 16,
+ *         8, 4, 2, 1 runs);
+ * and the smallest i with the least e_i is kept (i = 0 is w4a8_pack_int4).
+ * With r < 1 the code -8 occurs.  Arguments and errors as w4a8_pack_int4.
+ */
+W4A8_API w4a8_status w4a8_pack_int4_mse_clip(const void* w_bf16, int64_t R, int64_t K,
+                                             int32_t group, int32_t* packed, void* scales_bf16,
+                                             void* stream);
+
+/*
  * w4a8_prepare_experts_b200 - lay out one projection's quantised experts the
  * way w4a8_moe_forward reads them.  The codes and scale values are those of
  * w4a8_pack_int4 (the pages fix the uint4b8 codes and the group-128 bf16

@@ -81,21 +81,23 @@ class ExpertStore:
     """The oracle's own quantised experts, built lazily from bf16 weights.
 
     ``get_weights(e)`` returns float64 arrays ``(w13 [2I, H], w2 [H, I])``
-    holding bf16 values.  Indexing returns
+    holding bf16 values; ``quantize`` is ``rtn_quantize_int4`` (default) or
+    ``mse_clip_quantize_int4``.  Indexing returns
     ``(w13_packed int32 [2I, H/8], s13 [2I, H/128], w2_packed int32 [H, I/8],
     s2 [H, I/128])``.
     """
 
-    def __init__(self, E: int, get_weights: Callable[[int], tuple]):
+    def __init__(self, E: int, get_weights: Callable[[int], tuple], quantize=None):
         self.E = E
         self._get = get_weights
+        self._quantize = quantize or rtn_quantize_int4
         self._cache: Dict[int, tuple] = {}
 
     def __getitem__(self, e: int):
         if e not in self._cache:
             w13, w2 = self._get(e)
-            q13, s13 = rtn_quantize_int4(w13)
-            q2, s2 = rtn_quantize_int4(w2)
+            q13, s13 = self._quantize(w13)
+            q2, s2 = self._quantize(w2)
             self._cache[e] = (pack_uint4b8(q13), s13, pack_uint4b8(q2), s2)
         return self._cache[e]
 

@@ -8,8 +8,10 @@ per group of 128 consecutive weights along K, stored in compressed-tensors
 unsigned nibble q + 8 ("uint4b8"), 8 nibbles per int32 word ("8 four-bit
 weights per int32 slot", the note on the ~370B parameter display).  The pages
 describe round-to-nearest with a per-group MSE search over 11 shrink ratios of
-the scale; this oracle implements the plain round-to-nearest (RTN) step with
-scale = absmax / 7, the ratio-1.00 member of that search.
+the scale (model card, "quantisation method": ratios 1.00 down to 0.70, the
+MSE-optimal scale kept).  ``rtn_quantize_int4`` is the plain round-to-nearest
+step with scale = absmax / 7 (the ratio-1.00 member of that search);
+``mse_clip_quantize_int4`` is the search.
 
 Readings taken where the pages are silent:
 * scale: s = bf16(absmax / 7), rounded to bf16 (the stored scale dtype) before
@@ -55,6 +57,65 @@ def rtn_quantize_int4(w, group: int = GROUP):
     q = np.clip(np.rint(ratio), -8, 7)
     q = np.where(s[..., None] == 0.0, 0.0, q)
     return q.astype(np.int8).reshape(R, K), s
+
+
+# The 11 shrink ratios 1.00, 0.97, ..., 0.70 (evenly spaced; the plainest reading
+# of "11 ratios from 1.00 to 0.70"), as float32 values (100 - 3 i) / 100.
+CLIP_RATIOS = np.array([np.float32((100.0 - 3.0 * i) / 100.0) for i in range(11)],
+                       dtype=np.float32)
+
+
+def _squared_error_fixed_order(d):
+    """Sum of d**2 over the last axis (128 = 32 x 4) in float64, in one fixed
+    order: each run of 4 consecutive values summed in sequence, then the 32
+    partial sums combined by five pairwise (xor 16, 8, 4, 2, 1) exchanges.
+    The pages do not say how the MSE is accumulated; fixing the order makes the
+    arg-min below a deterministic function of the inputs, which the kernel
+    reproduces operation for operation."""
+    sq = d * d
+    p = sq[..., 0::4] + sq[..., 1::4]
+    p = p + sq[..., 2::4]
+    p = p + sq[..., 3::4]
+    lanes = np.arange(32)
+    for off in (16, 8, 4, 2, 1):
+        p = p + p[..., lanes ^ off]
+    return p[..., 0]
+
+
+def mse_clip_quantize_int4(w, group: int = GROUP):
+    """Symmetric INT4 with the per-group MSE clip search (model card,
+    "quantisation method": for each group of 128, 11 shrink ratios of the
+    scale from 1.00 to 0.70 are tried and the MSE-optimal scale is kept).
+
+    For each ratio r (float32 ``CLIP_RATIOS``, tried from 1.00 down):
+      s_r = bf16(float32(float32(absmax * r) / 7));
+      q_r = clamp(round_half_even(float32(w / s_r)), -8, 7), 0 where s_r = 0;
+      e_r = sum over the group of (w - q_r * s_r)**2 in float64 (fixed order,
+            ``_squared_error_fixed_order``).
+    The first ratio with the smallest e_r is kept (ties keep the larger
+    scale).  r = 1.00 is exactly ``rtn_quantize_int4``.  With r < 1 the code
+    -8 becomes reachable.  Returns ``(q, s)`` as ``rtn_quantize_int4`` does.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    R, K = w.shape
+    if K % group or group != 128:
+        raise ValueError("group must be 128 and divide K")
+    wg = w.reshape(R, K // group, group)
+    amax = np.abs(wg).max(axis=2)
+    best_e = np.full(amax.shape, np.inf)
+    best_q = np.zeros(wg.shape)
+    best_s = np.zeros(amax.shape)
+    for r in CLIP_RATIOS:
+        s = bf16_round(f32_round(f32_round(amax * np.float64(r)) / 7.0))
+        with np.errstate(divide="ignore", invalid="ignore"):
+            q = np.clip(np.rint(f32_round(wg / s[..., None])), -8, 7)
+        q = np.where(s[..., None] == 0.0, 0.0, q)
+        e = _squared_error_fixed_order(wg - q * s[..., None])
+        take = e < best_e
+        best_e = np.where(take, e, best_e)
+        best_s = np.where(take, s, best_s)
+        best_q = np.where(take[..., None], q, best_q)
+    return best_q.astype(np.int8).reshape(R, K), best_s
 
 
 def pack_uint4b8(q):

@@ -24,18 +24,19 @@ MID_TOL = 1e-4          # h and Y rows (float32 GEMMs vs float64)
 CODE_MATCH = 0.999      # fraction of intermediate E4M3 codes equal to the oracle's
 
 
-def _store(w13, w2):
-    return oracle.ExpertStore(w13.shape[0], lambda e: (f64(w13[e]), f64(w2[e])))
+def _store(w13, w2, mse_clip=False):
+    return oracle.ExpertStore(w13.shape[0], lambda e: (f64(w13[e]), f64(w2[e])),
+                              quantize=oracle.mse_clip_quantize_int4 if mse_clip else None)
 
 
-def run_and_compare(cfg, hidden, logits, w13, w2, check_rows=None):
+def run_and_compare(cfg, hidden, logits, w13, w2, check_rows=None, mse_clip=False):
     E, k = cfg.E, cfg.k
     T, H, I = hidden.shape[0], cfg.H, cfg.I
-    layer = w4.W4A8MoELayer.from_bf16(w13.cuda(), w2.cuda(), k)
+    layer = w4.W4A8MoELayer.from_bf16(w13.cuda(), w2.cuda(), k, mse_clip=mse_clip)
     aux = aux_buffers(T, H, I, E, k)
     out = layer(hidden.cuda(), logits.cuda(), aux=aux)
     w4.w4a8_check_device_error()
-    store = _store(w13, w2)
+    store = _store(w13, w2, mse_clip)
     res = oracle.moe_forward(f64(hidden), logits.numpy(), store, k)
 
     # packed weights (bit-exact)
@@ -99,6 +100,16 @@ def test_forward_tiny_workload():
 ], ids=lambda c: c.name)
 def test_forward_edge_cases(cfg):
     run_and_compare(cfg, *small_case(cfg))
+
+
+@pytest.mark.parametrize("cfg", [
+    workloads.CONFIGS[0],
+    workloads.MoEConfig("ragged_clip", T=37, H=384, I=256, E=6, k=3, seed=13),
+    workloads.MoEConfig("multi_block_clip", T=300, H=256, I=128, E=2, k=2, seed=14),
+], ids=lambda c: c.name)
+def test_forward_with_mse_clip_weights(cfg):
+    # experts quantised by the clip search (codes -8 occur) on both sides
+    run_and_compare(cfg, *small_case(cfg), mse_clip=True)
 
 
 def test_forward_zero_token_row_and_no_aux_path():

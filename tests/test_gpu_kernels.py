@@ -38,6 +38,15 @@ def test_pack_int4_bit_exact(R, K):
     assert np.array_equal(bf16_bits(scales), oracle.f64_to_bf16_bits(s))
 
 
+@pytest.mark.parametrize("R,K", [(1, 128), (7, 256), (64, 6144), (300, 2048)])
+def test_pack_int4_mse_clip_bit_exact(R, K):
+    wb = _weights(R, K, R * 977 + K)
+    packed, scales = w4.w4a8_pack_int4(wb.cuda(), mse_clip=True)
+    q, s = oracle.mse_clip_quantize_int4(f64(wb))
+    assert np.array_equal(packed.cpu().numpy(), oracle.pack_uint4b8(q))
+    assert np.array_equal(bf16_bits(scales), oracle.f64_to_bf16_bits(s))
+
+
 def test_pack_int4_3d_and_empty():
     wb = _weights(2 * 64, 256, 5).reshape(2, 64, 256)
     packed, scales = w4.w4a8_pack_int4(wb.cuda())

@@ -54,6 +54,7 @@ def _declare(L):
         "w4a8_check_device_error": (i32, [vp]),
         "w4a8_selftest_wait_timeout": (i32, [ctypes.c_uint64, vp]),
         "w4a8_pack_int4": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+        "w4a8_pack_int4_mse_clip": (i32, [vp, i64, i64, i32, vp, vp, vp]),
         "w4a8_prepare_experts_b200": (i32, [vp, vp, i64, i64, i64, vp, vp, vp]),
         "w4a8_quant_act_fp8_per_token": (i32, [vp, i64, i64, vp, vp, vp]),
         "w4a8_moe_route_workspace_size": (sz, [i64, i32]),
@@ -138,10 +139,13 @@ def w4a8_selftest_wait_timeout(timeout_s: float = 0.05, device=None):
 
 
 def w4a8_pack_int4(w: torch.Tensor, group: int = 128, packed: Optional[torch.Tensor] = None,
-                   scales: Optional[torch.Tensor] = None):
-    """INT4 RTN group-128 quantisation + uint4b8 packing of bf16 ``w`` [..., K].
+                   scales: Optional[torch.Tensor] = None, mse_clip: bool = False):
+    """INT4 group-128 quantisation + uint4b8 packing of bf16 ``w`` [..., K].
 
-    Returns ``(packed int32 [..., K/8], scales bf16 [..., K/128])``.
+    ``mse_clip=False``: round-to-nearest with scale absmax / 7
+    (``w4a8_pack_int4``); ``True``: the per-group MSE clip search over 11
+    shrink ratios (``w4a8_pack_int4_mse_clip``).  Returns
+    ``(packed int32 [..., K/8], scales bf16 [..., K/128])``.
     """
     if w.dim() < 2:
         raise ValueError("w must have at least 2 dims")
@@ -153,8 +157,9 @@ def w4a8_pack_int4(w: torch.Tensor, group: int = 128, packed: Optional[torch.Ten
         packed = torch.empty(*lead, K // 8, dtype=torch.int32, device=w.device)
     if scales is None:
         scales = torch.empty(*lead, max(K // group, 0), dtype=torch.bfloat16, device=w.device)
-    _check("w4a8_pack_int4", lib().w4a8_pack_int4(_p(w2), R, K, group, _p(packed), _p(scales),
-                                                  _stream(w.device)))
+    name = "w4a8_pack_int4_mse_clip" if mse_clip else "w4a8_pack_int4"
+    _check(name, getattr(lib(), name)(_p(w2), R, K, group, _p(packed), _p(scales),
+                                      _stream(w.device)))
     return packed, scales
 
 
@@ -336,9 +341,10 @@ class W4A8MoELayer:
         self._ws = None
 
     @classmethod
-    def from_bf16(cls, w13: torch.Tensor, w2: torch.Tensor, k: int) -> "W4A8MoELayer":
-        p13, s13 = w4a8_pack_int4(w13)
-        p2, s2 = w4a8_pack_int4(w2)
+    def from_bf16(cls, w13: torch.Tensor, w2: torch.Tensor, k: int,
+                  mse_clip: bool = False) -> "W4A8MoELayer":
+        p13, s13 = w4a8_pack_int4(w13, mse_clip=mse_clip)
+        p2, s2 = w4a8_pack_int4(w2, mse_clip=mse_clip)
         p13, s13 = w4a8_prepare_experts_b200(p13, s13, packed_out=p13)
         p2, s2 = w4a8_prepare_experts_b200(p2, s2, packed_out=p2)
         return cls(p13, s13, p2, s2, k)

@@ -229,6 +229,27 @@ const char* set_last_error(const char* msg) {
 }
 }  // namespace w4a8
 
+namespace {
+w4a8_status pack_int4_common(const char* name, const void* w_bf16, int64_t R, int64_t K,
+                             int32_t group, int32_t* packed, void* scales_bf16, bool clip,
+                             void* stream) {
+  if (group != kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "group = %d; only 128", group);
+  if (R < 0 || K <= 0) return fail(W4A8_ERR_INVALID_ARG, "R = %lld, K = %lld",
+                                   static_cast<long long>(R), static_cast<long long>(K));
+  if (K % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "K = %lld is not a multiple of 128",
+                              static_cast<long long>(K));
+  if (R == 0) return W4A8_OK;
+  if (!w_bf16 || !packed || !scales_bf16) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(w_bf16) || !aligned16(packed) || !aligned16(scales_bf16))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_pack_int4(w_bf16, R, K, packed, scales_bf16, clip, di.sms,
+                                     static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, name);
+}
+}  // namespace
+
 extern "C" {
 
 int32_t w4a8_abi_version(void) { return 1; }
@@ -271,20 +292,14 @@ w4a8_status w4a8_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
 
 w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, int32_t group,
                            int32_t* packed, void* scales_bf16, void* stream) {
-  if (group != kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "group = %d; only 128", group);
-  if (R < 0 || K <= 0) return fail(W4A8_ERR_INVALID_ARG, "R = %lld, K = %lld",
-                                   static_cast<long long>(R), static_cast<long long>(K));
-  if (K % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "K = %lld is not a multiple of 128",
-                              static_cast<long long>(K));
-  if (R == 0) return W4A8_OK;
-  if (!w_bf16 || !packed || !scales_bf16) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
-  if (!aligned16(w_bf16) || !aligned16(packed) || !aligned16(scales_bf16))
-    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  DeviceInfo di;
-  if (w4a8_status st = device_info(&di)) return st;
-  cudaError_t err = launch_pack_int4(w_bf16, R, K, packed, scales_bf16, di.sms,
-                                     static_cast<cudaStream_t>(stream));
-  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "pack_int4 launch");
+  return pack_int4_common("pack_int4 launch", w_bf16, R, K, group, packed, scales_bf16, false,
+                          stream);
+}
+
+w4a8_status w4a8_pack_int4_mse_clip(const void* w_bf16, int64_t R, int64_t K, int32_t group,
+                                    int32_t* packed, void* scales_bf16, void* stream) {
+  return pack_int4_common("pack_int4_mse_clip launch", w_bf16, R, K, group, packed, scales_bf16,
+                          true, stream);
 }
 
 w4a8_status w4a8_quant_act_fp8_per_token(const void* x_bf16, int64_t T, int64_t H,

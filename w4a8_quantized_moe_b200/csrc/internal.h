@@ -25,8 +25,9 @@ inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok;
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
                              float* gsum, const int32_t* row_of, int k, uint8_t* perm,
                              int num_sms, cudaStream_t s);
+// clip_search: the per-group MSE search over 11 shrink ratios instead of absmax / 7.
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
-                             int num_sms, cudaStream_t s);
+                             bool clip_search, int num_sms, cudaStream_t s);
 // routing: top-k + per-block expert histogram; scan; stable scatter.
 // tile_prefix[e] = sum over experts e' < e of ceil(count[e'] / tile_n).
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,

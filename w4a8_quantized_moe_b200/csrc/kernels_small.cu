@@ -162,8 +162,18 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
 
 // ---------------------------------------------------------------- INT4 pack
 // One warp per group of 128 weights (grid-stride).  Lane l holds elements
-// 4l..4l+3; the group scale is bf16(absmax / 7); q = clamp(rint(w / s), -8, 7);
-// lanes 2i and 2i+1 form word i (nibbles little-endian along K).
+// 4l..4l+3; q = clamp(rint(w / s), -8, 7); lanes 2i and 2i+1 form word i
+// (nibbles little-endian along K).
+//   kClip = false: s = bf16(absmax / 7) (round-to-nearest);
+//   kClip = true:  the per-group MSE clip search over the 11 shrink ratios
+//     r = 1.00, 0.97, ..., 0.70 (GLM-5.3-W4A8 model card, "quantisation
+//     method"): candidate s_r = bf16(float32(absmax * r) / 7); the squared
+//     error of each candidate is summed in float64 in a fixed order (each lane
+//     sums its 4 values in sequence, then five xor-pairwise exchanges), with
+//     explicitly rounded double operations, so the arg-min is a deterministic
+//     function of the weights; the first (largest) ratio with the least error
+//     is kept.
+template <bool kClip>
 __global__ void __launch_bounds__(256) pack_int4_kernel(const __nv_bfloat16* __restrict__ w,
                                                         int64_t R, int64_t K,
                                                         int32_t* __restrict__ packed,
@@ -180,15 +190,43 @@ __global__ void __launch_bounds__(256) pack_int4_kernel(const __nv_bfloat16* __r
     float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
     float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
     amax = warp_max(amax);
-    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
-    const float s = __bfloat162float(sb);
+    auto codes = [&](float s, int (&q)[4]) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        q[i] = s != 0.0f ? static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -8.0f), 7.0f))
+                         : 0;
+    };
+    __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
+    int q[4];
+    codes(__bfloat162float(sb), q);
+    if constexpr (kClip) {
+      double best = 0.0;
+      for (int ri = 0; ri < 11; ++ri) {
+        const float r = static_cast<float>((100.0 - 3.0 * ri) / 100.0);
+        const __nv_bfloat16 cb = __float2bfloat16_rn(__fdiv_rn(__fmul_rn(amax, r), 7.0f));
+        const float c = __bfloat162float(cb);
+        int qc[4];
+        codes(c, qc);
+        double e = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const double d = __dsub_rn(static_cast<double>(v[i]),
+                                     __dmul_rn(static_cast<double>(qc[i]), static_cast<double>(c)));
+          e = i == 0 ? __dmul_rn(d, d) : __dadd_rn(e, __dmul_rn(d, d));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) e = __dadd_rn(e, __shfl_xor_sync(kFull, e, off));
+        if (ri == 0 || e < best) {  // every lane holds the same e: the choice is warp-uniform
+          best = e;
+          sb = cb;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) q[i] = qc[i];
+        }
+      }
+    }
     uint32_t nib = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int q = 0;
-      if (s != 0.0f) q = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v[i], s)), -8.0f), 7.0f));
-      nib |= static_cast<uint32_t>(q + 8) << (4 * i);
-    }
+    for (int i = 0; i < 4; ++i) nib |= static_cast<uint32_t>(q[i] + 8) << (4 * i);
     const uint32_t hi = __shfl_down_sync(kFull, nib, 1);
     if ((lane & 1) == 0)
       packed[r * (K / 8) + gi * (kGroup / 8) + (lane >> 1)] = static_cast<int32_t>(nib | (hi << 16));
@@ -491,12 +529,16 @@ cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes
 }
 
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
-                             int num_sms, cudaStream_t s) {
+                             bool clip_search, int num_sms, cudaStream_t s) {
   if (R == 0) return cudaSuccess;
   const int64_t ngroups = R * (K / kGroup);
   const int grid = grid_for(ngroups * 32, 256, num_sms, 16);
-  pack_int4_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), R, K, packed,
-                                        static_cast<__nv_bfloat16*>(scales));
+  if (clip_search)
+    pack_int4_kernel<true><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), R, K,
+                                                packed, static_cast<__nv_bfloat16*>(scales));
+  else
+    pack_int4_kernel<false><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), R, K,
+                                                 packed, static_cast<__nv_bfloat16*>(scales));
   return cudaGetLastError();
 }
 
