@@ -21,7 +21,9 @@ Sources.  The method is described by five web pages about 4-bit-weight /
   activations; dequantisation audit (section "Verification").
 * "GLM-5.3 EVAL_DETAILS" (zh), section 1: expert-weight reconstruction error
   (naive RTN 0.124, RTN with the per-group MSE clip search 0.103).
-* "GLM-5.3-Channel-INT4-w4a8" (hygon): per-channel variant (not built here).
+* "GLM-5.3-Channel-INT4-w4a8" (hygon): the per-channel INT4 weight /
+  per-token INT8 activation variant (quantisation table: RTN, static,
+  per-channel INT4 experts; dynamic per-token INT8 activations).
 * "From 755GB to 395GB" (Bitdeer AI blog): 256 routed experts per MoE layer,
   3 projections per expert.
 
@@ -40,12 +42,13 @@ have no pin beyond those of their parts.
 from .numerics import (bf16_bits_to_f64, f64_to_bf16_bits, bf16_round, f32_round,
                        e4m3_decode, e4m3_encode, E4M3_MAX)
 from .quant import (rtn_quantize_int4, mse_clip_quantize_int4, CLIP_RATIOS, pack_uint4b8,
-                    unpack_uint4b8, dequantize_int4, quant_act_fp8_per_token)
+                    unpack_uint4b8, dequantize_int4, quant_act_fp8_per_token,
+                    quant_act_int8_per_token, rtn_quantize_int4_channel)
 from .moe import route_topk, permute_by_expert, moe_forward, ExpertStore
 
 __all__ = ["bf16_bits_to_f64", "f64_to_bf16_bits", "bf16_round", "f32_round",
            "e4m3_decode", "e4m3_encode", "E4M3_MAX", "rtn_quantize_int4",
            "mse_clip_quantize_int4", "CLIP_RATIOS",
            "pack_uint4b8", "unpack_uint4b8", "dequantize_int4",
-           "quant_act_fp8_per_token", "route_topk", "permute_by_expert",
-           "moe_forward", "ExpertStore"]
+           "quant_act_fp8_per_token", "quant_act_int8_per_token", "route_topk", "permute_by_expert",
+           "moe_forward", "ExpertStore", "rtn_quantize_int4_channel"]

@@ -36,7 +36,7 @@ import numpy as np
 
 from .numerics import bf16_round, e4m3_decode, f32_round
 from .quant import (dequantize_int4, pack_uint4b8, quant_act_fp8_per_token,
-                    rtn_quantize_int4)
+                    quant_act_int8_per_token, rtn_quantize_int4)
 
 
 def route_topk(logits, k: int):
@@ -110,7 +110,8 @@ def _silu(x):
 
 
 def moe_forward(hidden, logits, experts: Sequence, k: int,
-                tokens: Optional[np.ndarray] = None, hidden_of_tokens=None):
+                tokens: Optional[np.ndarray] = None, hidden_of_tokens=None,
+                act_format: str = "fp8"):
     """The whole layer for all tokens, or for the token subset ``tokens``.
 
     ``hidden``: float64 [T, H] (bf16 values); ``logits``: float32 [T, E];
@@ -119,6 +120,10 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
     and the combine run only for the assignments of ``tokens`` (all tokens by
     default).  ``hidden`` may be None when ``hidden_of_tokens`` (float64
     [len(tokens), H], the rows of ``tokens``) is given instead.
+
+    ``act_format``: "fp8" (E4M3 per-token activations, the W4A8 layer) or
+    "int8" (symmetric INT8 per-token activations, the per-channel variant; the
+    experts' scales then have one column per row).
 
     Returns a dict with ``topk_ids``, ``topk_w``, ``expert_offsets``,
     ``sorted_token_ids``, ``row_of``, ``act_codes`` / ``act_scales`` (rows of
@@ -138,8 +143,14 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
                                                                          dtype=np.float64)
     H = x_rows.shape[1]
 
-    codes, a_scale = quant_act_fp8_per_token(x_rows)
-    x_deq = a_scale[:, None] * e4m3_decode(codes)          # exact: 24-bit x 4-bit significands
+    if act_format == "fp8":
+        quant, decode = quant_act_fp8_per_token, e4m3_decode
+    elif act_format == "int8":
+        quant, decode = quant_act_int8_per_token, lambda c: np.asarray(c, dtype=np.float64)
+    else:
+        raise ValueError(f"unknown act_format {act_format!r}")
+    codes, a_scale = quant(x_rows)
+    x_deq = a_scale[:, None] * decode(codes)               # exact: 24-bit x <= 8-bit significands
 
     need_rows = np.sort(row_of[tokens].reshape(-1))
     Y: Dict[int, np.ndarray] = {}
@@ -154,11 +165,12 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
         w13p, s13, w2p, s2 = experts[e]
         I = w13p.shape[0] // 2
         X = x_deq[[pos[int(sorted_tok[r])] for r in rows]]  # [n, H]
-        G = X @ dequantize_int4(w13p, s13).T                 # [n, 2I]
+        H_ = w13p.shape[1] * 8
+        G = X @ dequantize_int4(w13p, s13, group=H_ // s13.shape[1]).T   # [n, 2I]
         h = _silu(G[:, :I]) * G[:, I:]
-        hc, hs = quant_act_fp8_per_token(h)
-        hd = hs[:, None] * e4m3_decode(hc)
-        Ye = hd @ dequantize_int4(w2p, s2).T                 # [n, H]
+        hc, hs = quant(h)
+        hd = hs[:, None] * decode(hc)
+        Ye = hd @ dequantize_int4(w2p, s2, group=I // s2.shape[1]).T     # [n, H]
         for i, r in enumerate(rows):
             Y[int(r)] = Ye[i]
             inter_h[int(r)] = h[i]

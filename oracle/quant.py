@@ -118,6 +118,15 @@ def mse_clip_quantize_int4(w, group: int = GROUP):
     return best_q.astype(np.int8).reshape(R, K), best_s
 
 
+def rtn_quantize_int4_channel(w):
+    """Per-channel symmetric INT4 RTN ("GLM-5.3-Channel-INT4-w4a8" model card,
+    quantisation table: RTN, static, per-channel INT4 routed experts): one bf16
+    scale per output row, i.e. the group rule with the group spanning all of
+    K.  Returns ``(q int8 [R, K], s float64 [R, 1])``."""
+    w = np.asarray(w, dtype=np.float64)
+    return rtn_quantize_int4(w, group=w.shape[1])
+
+
 def pack_uint4b8(q):
     """Pack int [R, K] values in [-8, 7] into int32 [R, K // 8] uint4b8 words."""
     q = np.asarray(q).astype(np.int64)
@@ -149,6 +158,24 @@ def dequantize_int4(packed, scales, group: int = GROUP):
     R, K = q.shape
     s = np.asarray(scales, dtype=np.float64)
     return (q.reshape(R, K // group, group) * s[..., None]).reshape(R, K)
+
+
+def quant_act_int8_per_token(x):
+    """Per-row dynamic symmetric INT8 quantisation ("GLM-5.3-Channel-INT4-w4a8"
+    model card, quantisation table: activations dynamic, per-token INT8).
+
+    ``x``: float64 [T, H].  scale = float32(absmax / 127);
+    code = clamp(round_half_even(float32(x / scale)), -127, 127); a row whose
+    absmax is 0 gets scale 0 and codes 0.  Returns ``(codes int8 [T, H],
+    scale float64 [T] holding float32 values)``.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    amax = np.abs(x).max(axis=1) if x.shape[1] else np.zeros(x.shape[0])
+    scale = f32_round(amax / 127.0)
+    safe = np.where(scale > 0, scale, 1.0)
+    codes = np.clip(np.rint(f32_round(x / safe[:, None])), -127, 127)
+    codes[scale == 0] = 0
+    return codes.astype(np.int8), scale
 
 
 def quant_act_fp8_per_token(x):
