@@ -109,9 +109,22 @@ class ClockSampler:
         return out
 
 
-def build_layer(cfg, device, w4):
+def build_layer(cfg, device, w4, variant: str = "w4a8"):
     """Pack every expert's seeded bf16 weights on the device and lay them out for the GEMMs (not timed)."""
     E, H, I = cfg.E, cfg.H, cfg.I
+    if variant == "channel-int8":
+        p13 = torch.empty(E, 2 * I, H // 8, dtype=torch.int32, device=device)
+        s13 = torch.empty(E, 2 * I, dtype=torch.bfloat16, device=device)
+        p2 = torch.empty(E, H, I // 8, dtype=torch.int32, device=device)
+        s2 = torch.empty(E, H, dtype=torch.bfloat16, device=device)
+        for e in range(E):
+            w13, w2 = workloads.gen_expert_weights(cfg, e, device=device)
+            w4.w4a8_pack_int4_channel(w13, packed=p13[e], scales=s13[e])
+            w4.w4a8_pack_int4_channel(w2, packed=p2[e], scales=s2[e])
+        p13, n13 = w4.w4a8_prepare_experts_channel_b200(p13, packed_out=p13)
+        p2, n2 = w4.w4a8_prepare_experts_channel_b200(p2, packed_out=p2)
+        torch.cuda.synchronize(device)
+        return w4.W4A8ChannelInt8Layer(p13, s13, n13, p2, s2, n2, cfg.k)
     p13 = torch.empty(E, 2 * I, H // 8, dtype=torch.int32, device=device)
     s13 = torch.empty(E, 2 * I, H // 128, dtype=torch.bfloat16, device=device)
     p2 = torch.empty(E, H, I // 8, dtype=torch.int32, device=device)
@@ -162,13 +175,17 @@ def recorded_traffic(workload: str, kernel: str):
     return None
 
 
-def algorithmic_work(cfg, counts):
+def algorithmic_work(cfg, counts, variant: str = "w4a8"):
     """Algorithmic bytes and FLOPs of each grouped GEMM for the given expert counts."""
     T, H, I, k = cfg.T, cfg.H, cfg.I, cfg.k
     A = T * k
     active = int(np.count_nonzero(counts))
-    w13_bytes = 2 * I * H // 2 + 2 * I * (H // 128) * 2
-    w2_bytes = H * I // 2 + H * (I // 128) * 2
+    if variant == "channel-int8":   # one bf16 scale and one int32 nibble sum per row
+        w13_bytes = 2 * I * H // 2 + 2 * I * (2 + 4)
+        w2_bytes = H * I // 2 + H * (2 + 4)
+    else:                           # one bf16 scale per 128-wide group
+        w13_bytes = 2 * I * H // 2 + 2 * I * (H // 128) * 2
+        w2_bytes = H * I // 2 + H * (I // 128) * 2
     g1 = dict(bytes=active * w13_bytes + T * H + T * 4 + A * I * 4 + A * 4 + A * 8,
               flops=2 * A * 2 * I * H)
     g2 = dict(bytes=active * w2_bytes + A * I + A * 4 + A * H * 4, flops=2 * A * H * I)
@@ -178,9 +195,10 @@ def algorithmic_work(cfg, counts):
 class OracleSample:
     """The CPU oracle on a seeded sample of tokens, experts quantised up front."""
 
-    def __init__(self, cfg, n_tokens: int, seed_tokens: int = 7):
+    def __init__(self, cfg, n_tokens: int, seed_tokens: int = 7, variant: str = "w4a8"):
         import oracle
         self.oracle, self.cfg = oracle, cfg
+        self.act_format = "int8" if variant == "channel-int8" else "fp8"
         try:
             from threadpoolctl import threadpool_info
             self.cores = max((p.get("num_threads", 1) for p in threadpool_info()), default=None)
@@ -199,14 +217,16 @@ class OracleSample:
             a, b = workloads.gen_expert_weights(cfg, e)
             return f(a), f(b)
 
-        self.store = oracle.ExpertStore(cfg.E, weights)
+        self.store = oracle.ExpertStore(
+            cfg.E, weights,
+            quantize=oracle.rtn_quantize_int4_channel if self.act_format == "int8" else None)
         for e in sorted(set(ids[self.tokens].reshape(-1).tolist())):
             self.store[e]                          # quantise outside the timed region
 
     def run(self) -> float:
         t0 = time.perf_counter()
         self.oracle.moe_forward(self.hidden, self.logits, self.store, self.cfg.k,
-                                tokens=self.tokens)
+                                tokens=self.tokens, act_format=self.act_format)
         return time.perf_counter() - t0
 
     def describe(self, dt: float) -> str:
@@ -215,8 +235,8 @@ class OracleSample:
                 f"numpy, {dt:.2f} s per step")
 
 
-def cpu_baseline(cfg, n_tokens: int):
-    s = OracleSample(cfg, n_tokens)
+def cpu_baseline(cfg, n_tokens: int, variant: str = "w4a8"):
+    s = OracleSample(cfg, n_tokens, variant=variant)
     dt = s.run()
     return dict(value=len(s.tokens) / dt, unit="tokens/s", cores=s.cores, kind="oracle",
                 sample=s.describe(dt))
@@ -225,7 +245,7 @@ def cpu_baseline(cfg, n_tokens: int):
 def bench_reference(args, cfg, rank):
     if rank != 0:
         return 0
-    s = OracleSample(cfg, max(1, args.ref_tokens))
+    s = OracleSample(cfg, max(1, args.ref_tokens), variant=args.variant)
     for _ in range(args.warmup):
         s.run()
     times = [s.run() for _ in range(args.steps)]
@@ -260,6 +280,9 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="run the workload with this many experts instead (a smaller case for "
                          "profiler captures; recorded in config)")
+    ap.add_argument("--variant", default="w4a8", choices=["w4a8", "channel-int8"],
+                    help="w4a8: group-128 INT4 experts x FP8 E4M3 activations (default); "
+                         "channel-int8: per-channel INT4 experts x per-token INT8 activations")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload with this many tokens instead (a smaller case for "
                          "profiler captures; recorded in config)")
@@ -290,7 +313,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
 
-    layer = build_layer(cfg, device, w4)
+    layer = build_layer(cfg, device, w4, args.variant)
     rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)      # each rank its own batch
     hidden = workloads.gen_hidden(rank_cfg, device=device)
     logits = workloads.gen_logits(rank_cfg, device=device)
@@ -365,7 +388,7 @@ def main():
     e2e_value = whole_job_throughput(cfg.T, world, args.steps, e2e_ms)
 
     pk = peaks()
-    g1, g2, active = algorithmic_work(cfg, counts)
+    g1, g2, active = algorithmic_work(cfg, counts, args.variant)
     prefill = cfg.T >= 4096
     gi = 2 if stage_ms[2] >= stage_ms[4] else 4          # dominant kernel: the slower GEMM
     work = g1 if gi == 2 else g2
@@ -386,9 +409,12 @@ def main():
     line = dict(
         metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=ms / args.steps, higher_is_better=True, scaling="weak",
-        vs_baseline=None, dtype="e4m3xint4-f32acc", data="synthetic",
+        vs_baseline=None,
+        dtype="s8xint4-s32acc" if args.variant == "channel-int8" else "e4m3xint4-f32acc",
+        data="synthetic",
         config=dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
-                    active_experts=active, parallelism=f"dp{world}" if world > 1 else "single",
+                    variant=args.variant, active_experts=active,
+                    parallelism=f"dp{world}" if world > 1 else "single",
                     l2=("inputs larger than L2: %.2f GB of packed experts streamed per step"
                         % ((g1["bytes"] + g2["bytes"]) / 1e9))),
         stage_ms={n: round(x, 5) for n, x in zip(w4.STAGE_NAMES, stage_ms)},
@@ -400,7 +426,7 @@ def main():
         clocks=clk.summary(),
     )
     if rank == 0 and world == 1 and args.cpu_tokens > 0:
-        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens)
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, args.variant)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

@@ -309,6 +309,60 @@ W4A8_API w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logi
                              void* out_bf16, void* workspace, size_t workspace_bytes,
                              const w4a8_moe_aux* aux, void* stream);
 
+/*
+ * The per-channel INT4 weight / per-token INT8 activation variant
+ * ("GLM-5.3-Channel-INT4-w4a8" model card, quantisation table: RTN, static,
+ * per-channel INT4 routed experts; dynamic per-token INT8 activations).
+ *
+ * w4a8_pack_int4_channel - per output row: s = bf16(float32(absmax / 7)) over
+ * the whole row, q = clamp(rint(float32(w / s)), -8, 7) (0 when s == 0),
+ * packed as w4a8_pack_int4 packs (uint4b8, 8 per int32, little-endian).
+ *   w_bf16       [R, K] bf16; K > 0, K % 128 == 0
+ *   packed       [R, K / 8] int32, written
+ *   scales_bf16  [R] bf16, written
+ */
+W4A8_API w4a8_status w4a8_pack_int4_channel(const void* w_bf16, int64_t R, int64_t K,
+                                            int32_t* packed, void* scales_bf16, void* stream);
+
+/*
+ * w4a8_prepare_experts_channel_b200 - the words of w4a8_prepare_experts_b200
+ * (same nibble interleave) plus, per row, the sum over K of the stored
+ * nibbles u = q + 8 (the INT8 GEMM multiplies unsigned bytes and removes the
+ * offsets with these sums).  Scales are used as packed ([E, rows] bf16).
+ *   packed       [E, rows, K / 8] int32 from w4a8_pack_int4_channel
+ *   packed_out   [E, rows, K / 8] int32, written; may be `packed` (in place)
+ *   nibble_sums  [E, rows] int32, written
+ */
+W4A8_API w4a8_status w4a8_prepare_experts_channel_b200(const int32_t* packed, int64_t E,
+                                                       int64_t rows, int64_t K,
+                                                       int32_t* packed_out, int32_t* nibble_sums,
+                                                       void* stream);
+
+/*
+ * w4a8_moe_forward_channel_int8 - the layer of w4a8_moe_forward with
+ * per-channel INT4 experts and per-token INT8 activations:
+ *   a[t] = clamp(rint(float32(x[t] / sa[t])), -127, 127), sa[t] = float32(absmax / 127);
+ *   G[r, n] = sa[t] * s13[e, n] * sum_k a[t, k] * q13[e, n, k]   (exact int32 sums);
+ *   h = silu(G[:, :I]) * G[:, I:]; h requantised per segment row to INT8 by the
+ *   same rule; Y[r, n] = sh[r] * s2[e, n] * sum_k c[r, k] * q2[e, n, k];
+ *   combine as w4a8_moe_forward.
+ * The grouped GEMMs run tcgen05 kind::i8 MMAs on unsigned bytes (stored nibble
+ * u = q + 8, activation code + 128) with one int32 accumulator per tile and
+ * remove both offsets exactly with the per-row nibble sums and per-token code
+ * sums.  Routing, permutation, workspace (w4a8_moe_workspace_size) and aux as
+ * w4a8_moe_forward, except that aux->act_codes and aux->inter_codes receive
+ * the INT8 codes stored offset-binary (code + 128).
+ *   w13_packed / w2_packed  from w4a8_prepare_experts_channel_b200
+ *   w13_scales [E, 2I] bf16, w2_scales [E, H] bf16 (from w4a8_pack_int4_channel)
+ *   w13_nibble_sums [E, 2I], w2_nibble_sums [E, H] int32
+ */
+W4A8_API w4a8_status w4a8_moe_forward_channel_int8(
+    const void* hidden_bf16, const float* logits, const int32_t* w13_packed,
+    const void* w13_scales, const int32_t* w13_nibble_sums, const int32_t* w2_packed,
+    const void* w2_scales, const int32_t* w2_nibble_sums, int64_t T, int64_t H, int64_t I,
+    int32_t E, int32_t k, void* out_bf16, void* workspace, size_t workspace_bytes,
+    const w4a8_moe_aux* aux, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -63,6 +63,10 @@ def _declare(L):
         "w4a8_moe_workspace_size": (sz, [i64, i64, i64, i32, i32]),
         "w4a8_moe_forward": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, sz,
                                    vp, vp]),
+        "w4a8_pack_int4_channel": (i32, [vp, i64, i64, vp, vp, vp]),
+        "w4a8_prepare_experts_channel_b200": (i32, [vp, i64, i64, i64, vp, vp, vp]),
+        "w4a8_moe_forward_channel_int8": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                                i32, i32, vp, vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -266,6 +270,27 @@ _AUX_FIELDS = ["topk_ids", "topk_w", "expert_offsets", "sorted_token_ids", "row_
                "act_scales", "inter_h", "inter_codes", "inter_scales", "y_rows"]
 
 
+def _aux_struct(aux, stage_events):
+    """The w4a8_moe_aux of a dict of caller buffers and optional stage events
+    (None when neither is given), plus the objects that must outlive the call."""
+    if not aux and not stage_events:
+        return None, []
+    st, keep = MoEAux(), []
+    for name, t in (aux or {}).items():
+        if name not in _AUX_FIELDS:
+            raise KeyError(f"unknown aux buffer {name!r}")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"aux[{name!r}] must be a contiguous CUDA tensor")
+        setattr(st, name, t.data_ptr())
+    if stage_events:
+        if len(stage_events) != 2 * NUM_STAGES:
+            raise ValueError(f"need {2 * NUM_STAGES} events")
+        arr = (ctypes.c_void_p * (2 * NUM_STAGES))(*[e.cuda_event for e in stage_events])
+        keep.append(arr)
+        st.stage_events = ctypes.cast(arr, ctypes.c_void_p)
+    return st, keep
+
+
 def w4a8_moe_forward(hidden: torch.Tensor, logits: torch.Tensor, w13_packed: torch.Tensor,
                      w13_scales: torch.Tensor, w2_packed: torch.Tensor, w2_scales: torch.Tensor,
                      k: int, out: Optional[torch.Tensor] = None,
@@ -298,22 +323,7 @@ def w4a8_moe_forward(hidden: torch.Tensor, logits: torch.Tensor, w13_packed: tor
     need = w4a8_moe_workspace_size(T, H, I, E, k)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-    aux_struct = None
-    keep = []
-    if aux or stage_events:
-        aux_struct = MoEAux()
-        for name, t in (aux or {}).items():
-            if name not in _AUX_FIELDS:
-                raise KeyError(f"unknown aux buffer {name!r}")
-            if not t.is_cuda or not t.is_contiguous():
-                raise ValueError(f"aux[{name!r}] must be a contiguous CUDA tensor")
-            setattr(aux_struct, name, t.data_ptr())
-        if stage_events:
-            if len(stage_events) != 2 * NUM_STAGES:
-                raise ValueError(f"need {2 * NUM_STAGES} events")
-            arr = (ctypes.c_void_p * (2 * NUM_STAGES))(*[e.cuda_event for e in stage_events])
-            keep.append(arr)
-            aux_struct.stage_events = ctypes.cast(arr, ctypes.c_void_p)
+    aux_struct, keep = _aux_struct(aux, stage_events)
     _check("w4a8_moe_forward",
            lib().w4a8_moe_forward(_p(hidden), _p(logits), _p(w13_packed), _p(w13_scales),
                                   _p(w2_packed), _p(w2_scales), T, H, I, E, k, _p(out),
@@ -360,3 +370,105 @@ class W4A8MoELayer:
         return w4a8_moe_forward(hidden, logits, self.w13_packed, self.w13_scales, self.w2_packed,
                                 self.w2_scales, self.k, out=out,
                                 workspace=self.workspace(hidden.shape[0]), **kw)
+
+
+# ---------------------------------------------------------------- per-channel INT4 x INT8
+
+def w4a8_pack_int4_channel(w: torch.Tensor, packed: Optional[torch.Tensor] = None,
+                           scales: Optional[torch.Tensor] = None):
+    """Per-channel INT4 RTN of bf16 ``w`` [..., K] -> (packed int32 [..., K/8], scales bf16 [...])."""
+    if w.dim() < 2:
+        raise ValueError("w must have at least 2 dims")
+    lead, K = tuple(w.shape[:-1]), w.shape[-1]
+    w2 = w.reshape(-1, K)
+    _need(w2, "w", torch.bfloat16, 2)
+    if packed is None:
+        packed = torch.empty(*lead, K // 8, dtype=torch.int32, device=w.device)
+    if scales is None:
+        scales = torch.empty(*lead, dtype=torch.bfloat16, device=w.device)
+    _check("w4a8_pack_int4_channel",
+           lib().w4a8_pack_int4_channel(_p(w2), w2.shape[0], K, _p(packed), _p(scales),
+                                        _stream(w.device)))
+    return packed, scales
+
+
+def w4a8_prepare_experts_channel_b200(packed: torch.Tensor, packed_out: Optional[torch.Tensor] = None):
+    """``packed`` int32 [E, rows, K/8] -> (packed_out in the GEMM's word layout,
+    nibble_sums int32 [E, rows]).  ``packed_out`` may be ``packed`` (in place)."""
+    _need(packed, "packed", torch.int32, 3)
+    E, rows, k8 = packed.shape
+    if packed_out is None:
+        packed_out = torch.empty_like(packed)
+    sums = torch.empty(E, rows, dtype=torch.int32, device=packed.device)
+    _check("w4a8_prepare_experts_channel_b200",
+           lib().w4a8_prepare_experts_channel_b200(_p(packed), E, rows, k8 * 8, _p(packed_out),
+                                                   _p(sums), _stream(packed.device)))
+    return packed_out, sums
+
+
+def w4a8_moe_forward_channel_int8(hidden, logits, w13_packed, w13_scales, w13_sums, w2_packed,
+                                  w2_scales, w2_sums, k: int, out=None, workspace=None,
+                                  aux: Optional[Dict[str, torch.Tensor]] = None,
+                                  stage_events: Optional[Sequence[torch.cuda.Event]] = None
+                                  ) -> torch.Tensor:
+    """The per-channel INT4 x per-token INT8 layer; bf16 [T, H].  aux codes are offset-binary."""
+    _need(hidden, "hidden", torch.bfloat16, 2)
+    _need(logits, "logits", torch.float32, 2)
+    _need(w13_packed, "w13_packed", torch.int32, 3)
+    _need(w2_packed, "w2_packed", torch.int32, 3)
+    _need(w13_scales, "w13_scales", torch.bfloat16, 2)
+    _need(w2_scales, "w2_scales", torch.bfloat16, 2)
+    _need(w13_sums, "w13_sums", torch.int32, 2)
+    _need(w2_sums, "w2_sums", torch.int32, 2)
+    T, H = hidden.shape
+    E = logits.shape[1]
+    I = w2_packed.shape[2] * 8
+    if logits.shape[0] != T or w13_packed.shape != (E, 2 * I, H // 8) or \
+            w2_packed.shape != (E, H, I // 8) or w13_scales.shape != (E, 2 * I) or \
+            w2_scales.shape != (E, H) or w13_sums.shape != (E, 2 * I) or w2_sums.shape != (E, H):
+        raise ValueError("inconsistent shapes")
+    dev = hidden.device
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    need = w4a8_moe_workspace_size(T, H, I, E, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    aux_struct, keep = _aux_struct(aux, stage_events)
+    _check("w4a8_moe_forward_channel_int8",
+           lib().w4a8_moe_forward_channel_int8(
+               _p(hidden), _p(logits), _p(w13_packed), _p(w13_scales), _p(w13_sums),
+               _p(w2_packed), _p(w2_scales), _p(w2_sums), T, H, I, E, k, _p(out), _p(workspace),
+               workspace.numel(), None if aux_struct is None else ctypes.byref(aux_struct),
+               _stream(dev)))
+    return out
+
+
+class W4A8ChannelInt8Layer:
+    """Per-channel INT4 experts with per-token INT8 activations (resident, prepared)."""
+
+    def __init__(self, w13_packed, w13_scales, w13_sums, w2_packed, w2_scales, w2_sums, k: int):
+        self.w13 = (w13_packed, w13_scales, w13_sums)
+        self.w2 = (w2_packed, w2_scales, w2_sums)
+        self.k = k
+        self.E, twoI, h8 = w13_packed.shape
+        self.H, self.I = h8 * 8, twoI // 2
+        self._ws = None
+
+    @classmethod
+    def from_bf16(cls, w13: torch.Tensor, w2: torch.Tensor, k: int) -> "W4A8ChannelInt8Layer":
+        p13, s13 = w4a8_pack_int4_channel(w13)
+        p2, s2 = w4a8_pack_int4_channel(w2)
+        p13, n13 = w4a8_prepare_experts_channel_b200(p13, packed_out=p13)
+        p2, n2 = w4a8_prepare_experts_channel_b200(p2, packed_out=p2)
+        return cls(p13, s13, n13, p2, s2, n2, k)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = max(w4a8_moe_workspace_size(T, self.H, self.I, self.E, self.k), 1)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.w13[0].device)
+        return self._ws
+
+    def __call__(self, hidden, logits, out=None, aux=None, stage_events=None) -> torch.Tensor:
+        return w4a8_moe_forward_channel_int8(hidden, logits, *self.w13, *self.w2, self.k, out=out,
+                                             workspace=self.workspace(hidden.shape[0]), aux=aux,
+                                             stage_events=stage_events)

@@ -124,6 +124,8 @@ struct ForwardBufs {
   uint8_t* inter_codes;
   float* inter_scales;
   float* inter_gsum;
+  int32_t* act_rowsum;    // INT8 variant: per token, sum of code + 128
+  int32_t* inter_rowsum;  // INT8 variant: per segment row
   float* y;
 };
 
@@ -145,6 +147,8 @@ ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int
   b.inter_codes = c.take<uint8_t>(A * static_cast<size_t>(I));
   b.inter_scales = c.take<float>(A);
   b.inter_gsum = c.take<float>(A * static_cast<size_t>(I / kGroup));
+  b.act_rowsum = c.take<int32_t>(static_cast<size_t>(T));
+  b.inter_rowsum = c.take<int32_t>(A);
   b.y = c.take<float>(A * static_cast<size_t>(H));
   return b;
 }
@@ -392,12 +396,23 @@ size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32
   return c.off + 256;
 }
 
-w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
+}  // extern "C"
+
+namespace {
+// The layer, for both variants: i8 == nullptr runs the W4A8 (FP8 E4M3
+// activations, group-128 scales) path; otherwise the per-channel INT4 x
+// per-token INT8 path with i8 = {w13 nibble row sums, w2 nibble row sums}.
+struct Int8Weights {
+  const int32_t* w13_nsum;
+  const int32_t* w2_nsum;
+};
+
+w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
                              const int32_t* w13_packed, const void* w13_scales,
                              const int32_t* w2_packed, const void* w2_scales, int64_t T,
                              int64_t H, int64_t I, int32_t E, int32_t k, void* out_bf16,
                              void* workspace, size_t workspace_bytes, const w4a8_moe_aux* aux,
-                             void* stream) {
+                             void* stream, const Int8Weights* i8) {
   if (w4a8_status st = check_route_args(logits, T, E, k)) return st;
   if (H <= 0 || I <= 0 || H % kGroup || I % kGroup)
     return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld and I = %lld must be positive multiples of 128",
@@ -409,7 +424,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
     return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "E * rows exceeds 2^31 - 1");
   if (T == 0) return W4A8_OK;
   const void* ptrs[] = {hidden_bf16, w13_packed, w13_scales, w2_packed, w2_scales, out_bf16,
-                        workspace};
+                        workspace, i8 ? i8->w13_nsum : workspace, i8 ? i8->w2_nsum : workspace};
   for (const void* p : ptrs) {
     if (!p) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
@@ -471,14 +486,19 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
                                     static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
   // group-major scales as bytes: [E * G, 2 * rows]; one box = one tile's scales
-  if (w4a8_status st = encode_u8_2d(&ts1, w13_scales, static_cast<uint64_t>(2 * I) * 2,
-                                    static_cast<uint64_t>(E) * (H / kGroup), 128,
-                                    static_cast<uint32_t>(H / kGroup), CU_TENSOR_MAP_SWIZZLE_NONE))
-    return st;
-  if (w4a8_status st = encode_u8_2d(&ts2, w2_scales, static_cast<uint64_t>(H) * 2,
-                                    static_cast<uint64_t>(E) * (I / kGroup), 256,
-                                    static_cast<uint32_t>(I / kGroup), CU_TENSOR_MAP_SWIZZLE_NONE))
-    return st;
+  // (W4A8 only; the INT8 variant reads its per-row scales in the epilogue)
+  if (!i8) {
+    if (w4a8_status st = encode_u8_2d(&ts1, w13_scales, static_cast<uint64_t>(2 * I) * 2,
+                                      static_cast<uint64_t>(E) * (H / kGroup), 128,
+                                      static_cast<uint32_t>(H / kGroup),
+                                      CU_TENSOR_MAP_SWIZZLE_NONE))
+      return st;
+    if (w4a8_status st = encode_u8_2d(&ts2, w2_scales, static_cast<uint64_t>(H) * 2,
+                                      static_cast<uint64_t>(E) * (I / kGroup), 256,
+                                      static_cast<uint32_t>(I / kGroup),
+                                      CU_TENSOR_MAP_SWIZZLE_NONE))
+      return st;
+  }
 
   auto record = [&](int i) -> cudaError_t {
     return ev && ev[i] ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
@@ -500,7 +520,7 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   W4A8_STEP(record(3), "cudaEventRecord");
   W4A8_STEP(record(0), "cudaEventRecord");
   W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, b.act_gsum, b.row_of, k,
-                             b.perm_codes, di.sms, s),
+                             b.perm_codes, di.sms, s, i8 ? b.act_rowsum : nullptr),
             "act_quant launch");
   W4A8_STEP(record(1), "cudaEventRecord");
 
@@ -521,13 +541,17 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
   g1.nb_fastest = tile_order_nb_fastest(decode);
+  g1.wsum = i8 ? i8->w13_nsum : nullptr;
+  g1.act_sum = b.act_rowsum;
   W4A8_STEP(record(4), "cudaEventRecord");
-  W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, g1, di.sms, s), "gate/up GEMM launch");
+  W4A8_STEP(i8 ? launch_grouped_gemm_i8(true, decode, tw1, ta1, g1, di.sms, s)
+               : launch_grouped_gemm(true, decode, tw1, ta1, ts1, g1, di.sms, s),
+            "gate/up GEMM launch");
   W4A8_STEP(record(5), "cudaEventRecord");
 
   W4A8_STEP(record(6), "cudaEventRecord");
   W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales, b.inter_gsum,
-                                di.sms, s),
+                                di.sms, s, i8 ? b.inter_rowsum : nullptr),
             "intermediate quant launch");
   W4A8_STEP(record(7), "cudaEventRecord");
 
@@ -548,8 +572,12 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   g2.act_rows = A;
   g2.timeout_ns = wait_timeout_ns();
   g2.nb_fastest = tile_order_nb_fastest(decode);
+  g2.wsum = i8 ? i8->w2_nsum : nullptr;
+  g2.act_sum = b.inter_rowsum;
   W4A8_STEP(record(8), "cudaEventRecord");
-  W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, ts2, g2, di.sms, s), "down GEMM launch");
+  W4A8_STEP(i8 ? launch_grouped_gemm_i8(false, decode, tw2, ta2, g2, di.sms, s)
+               : launch_grouped_gemm(false, decode, tw2, ta2, ts2, g2, di.sms, s),
+            "down GEMM launch");
   W4A8_STEP(record(9), "cudaEventRecord");
 
   W4A8_STEP(record(10), "cudaEventRecord");
@@ -558,6 +586,74 @@ w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
   W4A8_STEP(record(11), "cudaEventRecord");
 #undef W4A8_STEP
   return W4A8_OK;
+}
+}  // namespace
+
+extern "C" {
+
+w4a8_status w4a8_moe_forward(const void* hidden_bf16, const float* logits,
+                             const int32_t* w13_packed, const void* w13_scales,
+                             const int32_t* w2_packed, const void* w2_scales, int64_t T,
+                             int64_t H, int64_t I, int32_t E, int32_t k, void* out_bf16,
+                             void* workspace, size_t workspace_bytes, const w4a8_moe_aux* aux,
+                             void* stream) {
+  return moe_forward_impl(hidden_bf16, logits, w13_packed, w13_scales, w2_packed, w2_scales, T, H,
+                          I, E, k, out_bf16, workspace, workspace_bytes, aux, stream, nullptr);
+}
+
+w4a8_status w4a8_moe_forward_channel_int8(const void* hidden_bf16, const float* logits,
+                                          const int32_t* w13_packed, const void* w13_scales,
+                                          const int32_t* w13_nibble_sums,
+                                          const int32_t* w2_packed, const void* w2_scales,
+                                          const int32_t* w2_nibble_sums, int64_t T, int64_t H,
+                                          int64_t I, int32_t E, int32_t k, void* out_bf16,
+                                          void* workspace, size_t workspace_bytes,
+                                          const w4a8_moe_aux* aux, void* stream) {
+  const Int8Weights i8{w13_nibble_sums, w2_nibble_sums};
+  return moe_forward_impl(hidden_bf16, logits, w13_packed, w13_scales, w2_packed, w2_scales, T, H,
+                          I, E, k, out_bf16, workspace, workspace_bytes, aux, stream, &i8);
+}
+
+w4a8_status w4a8_pack_int4_channel(const void* w_bf16, int64_t R, int64_t K, int32_t* packed,
+                                   void* scales_bf16, void* stream) {
+  if (R < 0 || K <= 0) return fail(W4A8_ERR_INVALID_ARG, "R = %lld, K = %lld",
+                                   static_cast<long long>(R), static_cast<long long>(K));
+  if (K % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "K = %lld is not a multiple of 128",
+                              static_cast<long long>(K));
+  if (R == 0) return W4A8_OK;
+  if (!w_bf16 || !packed || !scales_bf16) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(w_bf16) || !aligned16(packed) || !aligned16(scales_bf16))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_pack_int4_channel(w_bf16, R, K, packed, scales_bf16, di.sms,
+                                             static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "pack_int4_channel launch");
+}
+
+w4a8_status w4a8_prepare_experts_channel_b200(const int32_t* packed, int64_t E, int64_t rows,
+                                              int64_t K, int32_t* packed_out,
+                                              int32_t* nibble_sums, void* stream) {
+  if (E < 0 || rows < 0 || K <= 0)
+    return fail(W4A8_ERR_INVALID_ARG, "E = %lld, rows = %lld, K = %lld", static_cast<long long>(E),
+                static_cast<long long>(rows), static_cast<long long>(K));
+  if (K % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "K = %lld is not a multiple of 128",
+                              static_cast<long long>(K));
+  const int64_t R = E * rows, nwords = R * (K / 8);
+  if (nwords == 0) return W4A8_OK;
+  if (!packed || !packed_out || !nibble_sums) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  for (const void* p : {static_cast<const void*>(packed), static_cast<const void*>(packed_out),
+                        static_cast<const void*>(nibble_sums)})
+    if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (packed != packed_out && packed < packed_out + nwords && packed_out < packed + nwords)
+    return fail(W4A8_ERR_INVALID_ARG, "packed and packed_out overlap without being the same buffer");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the sums do not depend on the nibble order: take them before an in-place repack
+  cudaError_t err = launch_nibble_row_sum(packed, R, K / 8, nibble_sums, di.sms, s);
+  if (err == cudaSuccess) err = launch_repack_int4_b200(packed, nwords, packed_out, di.sms, s);
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "prepare_experts_channel launch");
 }
 
 }  // extern "C"

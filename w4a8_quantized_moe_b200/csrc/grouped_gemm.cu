@@ -139,6 +139,10 @@ using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2, 0>;
 using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 3, 3, 1, 4, 16, 2, 1, 1>;
 using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 3, 2, 1, 2, 16, 2, 1, 1>;
 using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
+// INT8 per-channel shapes: one accumulator per tile, single MMA issuer
+using I8Decode  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 1, 1, 0>;
+using I8Decode2 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;  // 4 tiles x 2 chains
+using I8Prefill = Shape<kTileNPrefill, 4, 4, 4, 2, 1, 4, 16, 1, 1, 0>;
 
 struct Tile {
   int e, mb, n_valid, n_mma;
@@ -216,7 +220,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
   }
 }
 
-template <class S, bool kGateUp>
+template <class S, bool kGateUp, bool kI8>
 __global__ void __launch_bounds__(S::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         const __grid_constant__ CUtensorMap tmap_act,
@@ -253,10 +257,13 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   uint64_t* drain = upempty + S::kEpiSets;   // all MMAs of this CTA complete
   uint64_t* sfull = drain + 1;            // [kEpiSets][kEpiPerQuad] a slice's S_g staged
   uint64_t* sempty = sfull + S::kEpiSets * S::kEpiPerQuad;  // [..] the slice's warps are done
-  if constexpr (S::kUnified) {            // one "group's MMAs done" barrier per slot
-    bempty = aempty;
-    dfull = aempty;
-  }
+  // FP8: one commit per group releases the A slot, B stage and accumulator when
+  // the three rings have one size.  INT8: one accumulator per tile, so only
+  // the A and B rings can share a barrier.
+  constexpr bool kUniAll = S::kUnified && !kI8;
+  constexpr bool kUniAB = kI8 ? (kASlots == kBStages) : kUniAll;
+  if constexpr (kUniAB) bempty = aempty;
+  if constexpr (kUniAll) dfull = aempty;
   uint64_t* tfull = sempty + S::kEpiSets * S::kEpiPerQuad;  // [kTileScBufs] tile scales landed
   uint64_t* tempty = tfull + S::kTileScBufs;    // [kTileScBufs] epilogue warps are done
   // Group loops run in tile order, one set at a time (completion n = tile n's loop
@@ -276,14 +283,14 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&bfull[s], 1);
-      if (!S::kUnified) mbar_init(&bempty[s], 1);
+      if (!kUniAB) mbar_init(&bempty[s], 1);
     }
     for (int s = 0; s < kASlots; ++s) {
       mbar_init(&afull[s], 4);
       mbar_init(&aempty[s], 1);
     }
     for (int d = 0; d < kDBufs; ++d) {
-      if (!S::kUnified) mbar_init(&dfull[d], 1);
+      if (!kUniAll) mbar_init(&dfull[d], kI8 ? S::kMmaWarps : 1);
       mbar_init(&dempty[d], S::kEpiPerSet);   // each group is read by one set
     }
     for (int i = 0; i < S::kEpiSets; ++i) {
@@ -333,7 +340,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
         const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
         const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
-        {  // the tile's weight scales: box [G groups x 128 (or 2 x 64) rows] of bf16
+        if constexpr (!kI8) {  // the tile's weight scales: box [G groups x 128 (or 2 x 64) rows] of bf16
           const int tb = nt % S::kTileScBufs;
           const uint32_t tph = (nt / S::kTileScBufs) & 1;
           if (!mbar_wait(&tempty[tb], tph ^ 1, abort_flag, tmo)) break;
@@ -365,8 +372,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       // The latest fill of every stage must have landed before the CTA exits.
       for (int i = (it > kWStages ? it - kWStages : 0); i < it; ++i)
         mbar_wait_drain(&wfull[i % kWStages], (i / kWStages) & 1, tmo);
-      for (int i = (nt > S::kTileScBufs ? nt - S::kTileScBufs : 0); i < nt; ++i)
-        mbar_wait_drain(&tfull[i % S::kTileScBufs], (i / S::kTileScBufs) & 1, tmo);
+      if (!kI8)
+        for (int i = (nt > S::kTileScBufs ? nt - S::kTileScBufs : 0); i < nt; ++i)
+          mbar_wait_drain(&tfull[i % S::kTileScBufs], (i / S::kTileScBufs) & 1, tmo);
     }
     __syncwarp();
   } else if (warp == S::kWarpB) {
@@ -398,7 +406,56 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   } else if (warp >= S::kWarpMma && warp < S::kWarpB) {
     // ------------------------------------------------------------ MMA issuers
     const int mw = warp - S::kWarpMma;              // takes groups it % kMmaWarps == mw
-    if (lane == 0) {
+    if constexpr (kI8) {
+      // INT8, per-channel scales: a tile's groups accumulate into kMmaWarps
+      // int32 accumulators ("chains"); issuer mw takes the groups with global
+      // index it = mw (mod kMmaWarps), so each chain's first, non-accumulating
+      // MMA is issued ahead of the rest by the same thread, and every A slot /
+      // B stage keeps a single issuer.  A tile's accumulators are released once
+      // per tile (dfull counts one commit per chain).  Chains need G >= kMmaWarps.
+      constexpr int kChains = S::kMmaWarps;
+      constexpr int kTileSlots = kDBufs / kChains;
+      if (lane == 0) {
+        uint32_t idesc = 0, dt = 0;
+        int dcur = 0, cur_tile = -1;
+        bool first = true, ok = true;
+        for (int it = mw; ok && it < n_groups; it += kChains) {
+          const int tl = it / G, g = it - tl * G;
+          if (tl != cur_tile) {  // this chain's first group of the tile
+            cur_tile = tl;
+            first = true;
+            const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest,
+                                               blockIdx.x + tl * gridDim.x);
+            idesc = idesc_u8_s32_m128(static_cast<uint32_t>(t.n_mma));
+            dcur = tl % kTileSlots;
+            if (!mbar_wait(&dempty[dcur], ((tl / kTileSlots) & 1) ^ 1, abort_flag, tmo)) break;
+            dt = tmem + kTmemD + (dcur * kChains + mw) * kTileN;
+          }
+          const int sb = it % kBStages;
+          const uint32_t phb = (it / kBStages) & 1;
+          const int as = it % kASlots;
+          const uint32_t pha = (it / kASlots) & 1;
+          const bool rb = mbar_test_wait(&bfull[sb], phb);
+          const bool ra = mbar_test_wait(&afull[as], pha);
+          if (!(rb && ra) && (!mbar_wait(&bfull[sb], phb, abort_flag, tmo) ||
+                              !mbar_wait(&afull[as], pha, abort_flag, tmo)))
+            break;
+          tc_fence_after();
+          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + sb * kBStageBytes));
+          const uint32_t at = tmem + kTmemA + as * 32;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // K = 32 bytes per MMA
+            mma_i8_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                      (!first || kk > 0) ? 1u : 0u);
+          first = false;
+          tc_commit(&aempty[as]);
+          if constexpr (!kUniAB) tc_commit(&bempty[sb]);
+          if (g + kChains >= G) tc_commit(&dfull[dcur]);  // this chain's last group of the tile
+        }
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, tmo);
+      }
+    } else if (lane == 0) {
       int cur = -1;
       uint32_t idesc = 0;
       for (int it = mw; it < n_groups; it += S::kMmaWarps) {
@@ -439,7 +496,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
             mma_f8_ts(dt, tmem + S::kTmemConst, bdesc + static_cast<uint64_t>(kk * 2), idesc, 1u);
           }
         }
-        if constexpr (S::kUnified) {
+        if constexpr (kUniAll) {
           tc_commit(&aempty[as]);               // A slot, B stage and accumulator at once
         } else {
           tc_commit(&dfull[d]);
@@ -538,6 +595,61 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         }
         ts[i] = v;
       }
+      float acc[kEpiN];  // this warp's rows x columns of the tile, before the token scale
+      if constexpr (kI8) {
+        // per-channel INT8: D = sum_k u * a' with u = q + 8 and a' = code + 128
+        // (both stored unsigned); sum_k q * code = D - 128 U_m - 8 A'_t + 1024 K
+        // with U_m = sum_k u of weight row m and A'_t = sum_k a' of token t
+        const int wrow = kGateUp ? (m < 64 ? t.mb * 64 + m : a.half_rows + t.mb * 64 + (m - 64))
+                                 : t.mb * kBM + m;
+        const int64_t widx = static_cast<int64_t>(t.e) * a.n_rows + wrow;
+        const float wsm = __bfloat162float(static_cast<const __nv_bfloat16*>(a.wscale)[widx]);
+        const int base = 1024 * a.K - 128 * __ldg(a.wsum + widx);
+        int asum[kEpiN / 32];
+#pragma unroll
+        for (int i = 0; i < kEpiN / 32; ++i) {
+          const int j = j0 + lane + 32 * i;
+          int v = 0;
+          if (j < t.n_valid) {
+            const int64_t r = t.row0 + j;
+            v = kGateUp ? __ldg(a.act_sum + __ldg(a.row_tokens + r)) : __ldg(a.act_sum + r);
+          }
+          asum[i] = v;
+        }
+#pragma unroll
+        for (int j = 0; j < kEpiN; ++j) acc[j] = 0.0f;
+        constexpr int kChains = S::kMmaWarps;
+        const int d = ntile % (kDBufs / kChains);
+        if (!mbar_wait(&dfull[d], (ntile / (kDBufs / kChains)) & 1, abort_flag, tmo)) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem + lane_base + kTmemD + d * kChains * kTileN + j0;
+#pragma unroll
+        for (int c = 0; c < kEpiN / kLdCols; ++c) {
+          if (j0 + c * kLdCols < t.n_mma) {
+            int sum[kLdCols];
+#pragma unroll
+            for (int i = 0; i < kLdCols; ++i) sum[i] = 0;
+#pragma unroll
+            for (int ch = 0; ch < kChains; ++ch) {  // the tile's accumulation chains
+              uint32_t v[kLdCols];
+              if constexpr (kLdCols == 32) tmem_ld_32x32b_x32(taddr + ch * kTileN + c * 32, v);
+              else tmem_ld_32x32b_x16(taddr + ch * kTileN + c * 16, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < kLdCols; ++i) sum[i] += static_cast<int>(v[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < kLdCols; ++i) {
+              const int jj = c * kLdCols + i;
+              const int aj = __shfl_sync(kFull, asum[jj >> 5], jj & 31);
+              acc[jj] = wsm * static_cast<float>(sum[i] + base - 8 * aj);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dempty[d]);
+      } else {
       const uint32_t phs = lt & 1;
       if constexpr (!S::kOffsetInMma) {  // stage S_g of this warp's quarter of the slice's columns
         constexpr int kTok = kEpiN / 4;
@@ -624,7 +736,6 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         }
       }
       if (!ok) break;
-      float acc[kEpiN];
 #pragma unroll
       for (int j = 0; j < kEpiN / 2; ++j) {
         acc[2 * j] = acc2[j].x;
@@ -636,6 +747,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         mbar_arrive(&tempty[tb]);
         if (S::kEpiSets > 1) mbar_arrive(loopdone);
       }
+      }  // FP8
       if constexpr (kGateUp) {
         const uint32_t phu = lt & 1;
         if (q >= 2) {  // up rows: stage u = acc * token scale for the gate warps
@@ -713,7 +825,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in limit of sm_100
 
-template <class S, bool kGateUp>
+template <class S, bool kGateUp, bool kI8 = false>
 cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
                          const CUtensorMap& tmap_sc, const GemmArgs& a, int num_ctas,
                          cudaStream_t s) {
@@ -724,14 +836,15 @@ cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<S, kGateUp>,
+    err = cudaFuncSetAttribute(grouped_gemm_kernel<S, kGateUp, kI8>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                S::smem_bytes(kGateUp, kMaxGroups, kMaxExperts));
     if (err != cudaSuccess) return err;
     if (dev < 64) attr_set[dev] = true;
   }
   const int smem = S::smem_bytes(kGateUp, a.K / kGroup, a.E);
-  grouped_gemm_kernel<S, kGateUp><<<num_ctas, S::kThreads, smem, s>>>(tmap_w, tmap_act, tmap_sc, a);
+  grouped_gemm_kernel<S, kGateUp, kI8><<<num_ctas, S::kThreads, smem, s>>>(tmap_w, tmap_act,
+                                                                           tmap_sc, a);
   return cudaGetLastError();
 }
 
@@ -797,6 +910,21 @@ __global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, cudaStream_t s) {
   wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(timeout_ns);
   return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap& tmap_w,
+                                   const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
+                                   cudaStream_t s) {
+  if (a.K % kGroup || a.K / kGroup > kMaxGroups || a.K <= 0) return cudaErrorInvalidValue;
+  // the tile-scale map is unused in this mode; any valid map fills the slot
+  if (decode && a.K / kGroup >= 2)  // two accumulation chains need two groups per tile
+    return gate_up ? launch_shape<I8Decode2, true, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s)
+                   : launch_shape<I8Decode2, false, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s);
+  if (decode)
+    return gate_up ? launch_shape<I8Decode, true, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s)
+                   : launch_shape<I8Decode, false, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s);
+  return gate_up ? launch_shape<I8Prefill, true, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s)
+                 : launch_shape<I8Prefill, false, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s);
 }
 
 cudaError_t read_and_clear_device_error(int* value) {

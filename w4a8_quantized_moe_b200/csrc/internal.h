@@ -22,9 +22,11 @@ inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok;
 // gsum (nullable): [T, H / 128] sums of the E4M3 values of each 128-wide group.
 // perm (nullable): [T * k, H] codes in expert-segment order; row r = row_of[t, j]
 // receives token t's codes for every slot j.
+// int8_row_sum (non-null): INT8 mode instead of E4M3 -- codes are offset-binary
+// (code + 128) and the row sums of those bytes go to int8_row_sum [T].
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
                              float* gsum, const int32_t* row_of, int k, uint8_t* perm,
-                             int num_sms, cudaStream_t s);
+                             int num_sms, cudaStream_t s, int32_t* int8_row_sum = nullptr);
 // clip_search: the per-group MSE search over 11 shrink ratios instead of absmax / 7.
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
                              bool clip_search, int num_sms, cudaStream_t s);
@@ -37,13 +39,19 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          cudaStream_t s);
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, float* gsum, int num_sms,
-                               cudaStream_t s);
+                               cudaStream_t s, int32_t* int8_row_sum = nullptr);
 // packed uint4b8 words -> the word-local nibble interleave the grouped GEMM reads.
 cudaError_t launch_repack_int4_b200(const int32_t* in, int64_t nwords, int32_t* out, int num_sms,
                                     cudaStream_t s);
 // bf16 weight scales [E, rows, G] -> group-major [E, G, rows].
 cudaError_t launch_transpose_scales(const void* in, int64_t E, int64_t rows, int64_t G, void* out,
                                     int num_sms, cudaStream_t s);
+// per-channel INT4: scales bf16 [R] = bf16(row absmax / 7).
+cudaError_t launch_pack_int4_channel(const void* w, int64_t R, int64_t K, int32_t* packed,
+                                     void* scales, int num_sms, cudaStream_t s);
+// sums[r] = sum of the 2 * 4 * words_per_row stored nibbles of row r.
+cudaError_t launch_nibble_row_sum(const int32_t* packed, int64_t R, int64_t words_per_row,
+                                  int32_t* sums, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
                            int64_t H, int k, void* out, int num_sms, cudaStream_t s);
 
@@ -64,6 +72,9 @@ struct GemmArgs {
   uint32_t* row_amax;             // gate/up only: float bits of max |h| per segment row
   int64_t act_rows;               // rows of the activation tensor (T or A)
   int nb_fastest;                 // tile order within an expert (see grouped_gemm.cu)
+  // INT8 per-channel mode only: wscale is bf16 [E, n_rows] (one scale per row)
+  const int32_t* wsum;            // [E, n_rows] sum over K of the stored nibbles u = q + 8
+  const int32_t* act_sum;         // per token (gate/up) or row (down): sum of code + 128
   uint64_t timeout_ns;
 };
 // decode = the shape for few tokens per expert (see grouped_gemm.cu).
@@ -73,6 +84,11 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
                                 const CUtensorMap& tmap_act, const CUtensorMap& tmap_sc,
                                 const GemmArgs& a, int num_ctas, cudaStream_t s);
 int grouped_gemm_tile_n(bool decode);
+// The per-channel INT4 x per-token INT8 grouped GEMM (kind::i8, one int32
+// accumulator per tile); tmap_act holds offset-binary codes.
+cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap& tmap_w,
+                                   const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
+                                   cudaStream_t s);
 // One bounded wait on an mbarrier nothing arrives on (failure-detection self-test).
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
 

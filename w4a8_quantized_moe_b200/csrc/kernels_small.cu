@@ -45,6 +45,26 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float scale) {
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
+// 8 values -> 8 offset-binary INT8 codes (byte = code + 128), code =
+// clamp(rint(float32(v / scale)), -127, 127); scale 0 -> code 0.  The grouped
+// GEMM multiplies unsigned bytes, so the codes are stored offset by 128.
+__device__ __forceinline__ uint2 quant8_i8(const float (&v)[8], float scale) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int c = 0;
+    if (scale != 0.0f) c = static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v[i], scale)), -127.0f), 127.0f));
+    b[i] = static_cast<uint32_t>(c + 128);
+  }
+  return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                    b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+}
+
+// Sum of the 8 bytes of a uint2, as unsigned bytes (the unsigned dp4a).
+__device__ __forceinline__ int sum8_u8(uint2 q) {
+  return static_cast<int>(__dp4a(q.x, 0x01010101u, __dp4a(q.y, 0x01010101u, 0u)));
+}
+
 // Sum of the E4M3 values of the eight codes in c (low byte first).
 __device__ __forceinline__ float sum8_e4m3(uint2 c) {
   float s = 0.0f;
@@ -87,6 +107,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 constexpr int kAqThreads = 256;
 constexpr int kAqCache = 4;
 
+template <bool kInt8>
 __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat16* __restrict__ x,
                                                                int64_t T, int64_t H,
                                                                uint8_t* __restrict__ codes,
@@ -94,8 +115,10 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
                                                                float* __restrict__ gsum,
                                                                const int32_t* __restrict__ row_of,
                                                                int k,
-                                                               uint8_t* __restrict__ perm) {
+                                                               uint8_t* __restrict__ perm,
+                                                               int32_t* __restrict__ row_sum) {
   __shared__ float red[kAqThreads / 32];
+  __shared__ int ired[kAqThreads / 32];
   __shared__ int64_t dst_rows[kMaxTopK];
   const int64_t nchunk = H / 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,10 +144,11 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
     amax = red[0];
 #pragma unroll
     for (int w = 1; w < kAqThreads / 32; ++w) amax = fmaxf(amax, red[w]);
-    const float scale = __fdiv_rn(amax, 448.0f);
+    const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
     if (threadIdx.x == 0) scales[t] = scale;
     uint2* out = reinterpret_cast<uint2*>(codes + t * H);
-    float* gs = gsum ? gsum + t * (H / kGroup) : nullptr;
+    float* gs = !kInt8 && gsum ? gsum + t * (H / kGroup) : nullptr;
+    int isum = 0;  // INT8: this thread's share of the row's offset-binary code sum
     // Every thread runs every chunk slot (the slot bounds are uniform) so that
     // the 16-lane group reductions see full warps.
     auto emit = [&](int64_t c, const uint4& raw) {
@@ -132,10 +156,11 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
       if (c < nchunk) {
         float v[8];
         unpack8(raw, v);
-        const uint2 q = quant8(v, scale);
+        const uint2 q = kInt8 ? quant8_i8(v, scale) : quant8(v, scale);
         out[c] = q;
         if (perm)  // the token's codes again at each of its k segment rows
           for (int j = 0; j < k; ++j) reinterpret_cast<uint2*>(perm + dst_rows[j] * H)[c] = q;
+        if (kInt8) isum += sum8_u8(q);
         if (gs) part = sum8_e4m3(q);
       }
       if (gs) {
@@ -156,7 +181,18 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
       const int64_t c = base + threadIdx.x;
       emit(c, c < nchunk ? __ldg(row + c) : make_uint4(0u, 0u, 0u, 0u));
     }
-    __syncthreads();  // red[] is reused by the next row
+    if (kInt8) {  // exact integer row sum of the offset-binary codes
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(kFull, isum, o);
+      if (lane == 0) ired[warp] = isum;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int tot = 0;
+        for (int w = 0; w < kAqThreads / 32; ++w) tot += ired[w];
+        row_sum[t] = tot;
+      }
+    }
+    __syncthreads();  // red[] and ired[] are reused by the next row
   }
 }
 
@@ -231,6 +267,65 @@ __global__ void __launch_bounds__(256) pack_int4_kernel(const __nv_bfloat16* __r
     if ((lane & 1) == 0)
       packed[r * (K / 8) + gi * (kGroup / 8) + (lane >> 1)] = static_cast<int32_t>(nib | (hi << 16));
     if (lane == 0) scales[r * groups_per_row + gi] = sb;
+  }
+}
+
+// ---------------------------------------------------------------- per-channel INT4 pack
+// One CTA per row: s = bf16(absmax of the whole row / 7) (per-channel RTN),
+// q = clamp(rint(w / s), -8, 7), 8 nibbles per word little-endian along K.
+__global__ void __launch_bounds__(256) pack_int4_channel_kernel(const __nv_bfloat16* __restrict__ w,
+                                                                int64_t R, int64_t K,
+                                                                int32_t* __restrict__ packed,
+                                                                __nv_bfloat16* __restrict__ scales) {
+  __shared__ float red[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nchunk = K / 8;
+  for (int64_t r = blockIdx.x; r < R; r += gridDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(w + r * K);
+    float amax = 0.0f;
+    for (int64_t c = threadIdx.x; c < nchunk; c += blockDim.x) amax = fmaxf(amax, absmax8(__ldg(row + c)));
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
+    const float sc = __bfloat162float(sb);
+    if (threadIdx.x == 0) scales[r] = sb;
+    for (int64_t c = threadIdx.x; c < nchunk; c += blockDim.x) {
+      float v[8];
+      unpack8(__ldg(row + c), v);
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int q =
+            sc != 0.0f ? static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -8.0f), 7.0f)) : 0;
+        word |= static_cast<uint32_t>(q + 8) << (4 * i);
+      }
+      packed[r * nchunk + c] = static_cast<int32_t>(word);
+    }
+    __syncthreads();  // red[] is reused by the next row
+  }
+}
+
+// Warp per row: sum of all stored nibbles u = q + 8 of the row (any nibble order).
+__global__ void __launch_bounds__(256) nibble_row_sum_kernel(const uint32_t* __restrict__ packed,
+                                                             int64_t R, int64_t words_per_row,
+                                                             int32_t* __restrict__ sums) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wg = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = wg; r < R; r += nw) {
+    int acc = 0;
+    for (int64_t i = lane; i < words_per_row; i += 32) {
+      const uint32_t x = __ldg(packed + r * words_per_row + i);
+      acc = static_cast<int>(__dp4a(x & 0x0F0F0F0Fu, 0x01010101u, static_cast<unsigned>(acc)));
+      acc = static_cast<int>(__dp4a((x >> 4) & 0x0F0F0F0Fu, 0x01010101u, static_cast<unsigned>(acc)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (lane == 0) sums[r] = acc;
   }
 }
 
@@ -397,12 +492,14 @@ __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
 // codes = E4M3(h / scale), and the sum of the E4M3 values of each 128-wide
 // group (8 consecutive threads).  Whole warps run every iteration so that
 // the group reduction can use shuffles.
+template <bool kInt8>
 __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restrict__ h,
                                                           const uint32_t* __restrict__ row_amax,
                                                           int64_t A, int64_t I,
                                                           uint8_t* __restrict__ codes,
                                                           float* __restrict__ scales,
-                                                          float* __restrict__ gsum) {
+                                                          float* __restrict__ gsum,
+                                                          int32_t* __restrict__ row_sum) {
   const int64_t per_row = I / 16;
   const int64_t n = A * per_row;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -416,7 +513,7 @@ __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restric
       r = i / per_row;
       c = i - r * per_row;
       const float amax = __uint_as_float(__ldg(row_amax + r));
-      const float scale = __fdiv_rn(amax, 448.0f);
+      const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
       if (c == 0) scales[r] = scale;
       const float4* src = reinterpret_cast<const float4*>(h + r * I + c * 16);
       uint2 out[2];
@@ -424,13 +521,14 @@ __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restric
       for (int half = 0; half < 2; ++half) {
         const float4 a = __ldg(src + 2 * half), b = __ldg(src + 2 * half + 1);
         const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        out[half] = quant8(v, scale);
+        out[half] = kInt8 ? quant8_i8(v, scale) : quant8(v, scale);
       }
       *reinterpret_cast<uint4*>(codes + r * I + c * 16) =
           make_uint4(out[0].x, out[0].y, out[1].x, out[1].y);
-      if (gsum) part = sum8_e4m3(out[0]) + sum8_e4m3(out[1]);
+      if (kInt8) atomicAdd(row_sum + r, sum8_u8(out[0]) + sum8_u8(out[1]));  // exact, any order
+      else if (gsum) part = sum8_e4m3(out[0]) + sum8_e4m3(out[1]);
     }
-    if (gsum) {
+    if (!kInt8 && gsum) {
       part += __shfl_xor_sync(kFull, part, 4);
       part += __shfl_xor_sync(kFull, part, 2);
       part += __shfl_xor_sync(kFull, part, 1);
@@ -518,13 +616,19 @@ inline int grid_for(int64_t work_items, int threads, int num_sms, int per_sm = 8
 
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
                              float* gsum, const int32_t* row_of, int k, uint8_t* perm, int num_sms,
-                             cudaStream_t s) {
+                             cudaStream_t s, int32_t* int8_row_sum) {
   if (T == 0) return cudaSuccess;
   if (perm && (!row_of || k < 1 || k > kMaxTopK)) return cudaErrorInvalidValue;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(T < cap ? T : cap);
-  act_quant_kernel<<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H, codes,
-                                               scales, gsum, row_of, k, perm);
+  if (int8_row_sum)
+    act_quant_kernel<true><<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H,
+                                                       codes, scales, nullptr, row_of, k, perm,
+                                                       int8_row_sum);
+  else
+    act_quant_kernel<false><<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H,
+                                                        codes, scales, gsum, row_of, k, perm,
+                                                        nullptr);
   return cudaGetLastError();
 }
 
@@ -581,10 +685,18 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
 
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, float* gsum, int num_sms,
-                               cudaStream_t s) {
+                               cudaStream_t s, int32_t* int8_row_sum) {
   if (A == 0) return cudaSuccess;
   const int grid = grid_for(A * (I / 16), 256, num_sms);
-  inter_quant_kernel<<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, gsum);
+  if (int8_row_sum) {
+    cudaError_t err = cudaMemsetAsync(int8_row_sum, 0, static_cast<size_t>(A) * sizeof(int32_t), s);
+    if (err != cudaSuccess) return err;
+    inter_quant_kernel<true><<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, nullptr,
+                                                  int8_row_sum);
+  } else {
+    inter_quant_kernel<false><<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, gsum,
+                                                   nullptr);
+  }
   return cudaGetLastError();
 }
 
@@ -604,6 +716,25 @@ cudaError_t launch_transpose_scales(const void* in, int64_t E, int64_t rows, int
   const int grid = grid_for(n, 256, num_sms, 16);
   transpose_scales_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(in), E, rows, G,
                                                static_cast<uint16_t*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int4_channel(const void* w, int64_t R, int64_t K, int32_t* packed,
+                                     void* scales, int num_sms, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  const int grid = static_cast<int>(R < cap ? R : cap);
+  pack_int4_channel_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), R, K, packed,
+                                                static_cast<__nv_bfloat16*>(scales));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nibble_row_sum(const int32_t* packed, int64_t R, int64_t words_per_row,
+                                  int32_t* sums, int num_sms, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  const int grid = grid_for(R * 32, 256, num_sms, 16);
+  nibble_row_sum_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(packed), R,
+                                             words_per_row, sums);
   return cudaGetLastError();
 }
 

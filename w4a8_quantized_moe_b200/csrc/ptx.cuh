@@ -163,6 +163,26 @@ __host__ __device__ __forceinline__ uint32_t idesc_e4m3_f32_m128(uint32_t n) {
          | ((128u >> 4) << 24);    // M >> 4
 }
 
+// Instruction descriptor: kind::i8, A = B = unsigned 8-bit, D = S32, both
+// K-major, M = 128, N = n (multiple of 16, 16..256).  Same-signedness operands.
+__host__ __device__ __forceinline__ uint32_t idesc_u8_s32_m128(uint32_t n) {
+  return (2u << 4)                 // D format: S32
+         | (0u << 7) | (0u << 10)  // A, B format: unsigned 8-bit
+         | ((n >> 3) << 17)        // N >> 3
+         | ((128u >> 4) << 24);    // M >> 4
+}
+
+// D (TMEM, S32) (+)= A (TMEM, u8) x B (SMEM descriptor, u8), kind::i8, K = 32.
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle, rows of 128 B,
 // 8-row atoms 1024 B apart.  `saddr` must be 1024-byte aligned (base offset 0);
 // advancing K inside the 128-byte row adds the byte offset >> 4 to the start.
