@@ -163,7 +163,8 @@ def kernel_source_id() -> str:
 def recorded_traffic(workload: str, kernel: str):
     """dram__bytes_read.sum + dram__bytes_write.sum per launch from the ncu record in
     profiles/dram_traffic.txt, or None when there is none for this workload and
-    kernel or the kernel source has changed since it was taken."""
+    kernel or the kernel source has changed since it was taken.  The workload is
+    the config name, with ":<variant>" appended for variants other than w4a8."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -393,17 +394,18 @@ def main():
     gi = 2 if stage_ms[2] >= stage_ms[4] else 4          # dominant kernel: the slower GEMM
     work = g1 if gi == 2 else g2
     kname = "grouped_gemm_gate_up" if gi == 2 else "grouped_gemm_down"
+    traffic_key = cfg.name if args.variant == "w4a8" else f"{cfg.name}:{args.variant}"
     if prefill:
         achieved = work["flops"] / (stage_ms[gi] / 1e3) / 1e12
         peak = 2.0 * pk["bf16_sus"]                     # FP8 = 2 x bf16 (nominal ratio)
         roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
-                    frac=achieved / peak, traffic=recorded_traffic(cfg.name, kname), kernel=kname,
+                    frac=achieved / peak, traffic=recorded_traffic(traffic_key, kname), kernel=kname,
                     peak_source=f"{pk['src']} sustained bf16 x 2")
     else:
         achieved = work["bytes"] / (stage_ms[gi] / 1e3) / 1e9
         peak = pk["hbm"]
         roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
-                    traffic=recorded_traffic(cfg.name, kname), kernel=kname,
+                    traffic=recorded_traffic(traffic_key, kname), kernel=kname,
                     peak_source=f"{pk['src']} HBM copy")
 
     line = dict(
