@@ -124,6 +124,8 @@ struct ForwardBufs {
   uint8_t* inter_codes;
   float* inter_scales;
   float* inter_gsum;
+  uint16_t* act_parts;    // [A, sum_parts_ld(H)] three-part bf16 group sums
+  uint16_t* inter_parts;  // [A, sum_parts_ld(I)] the same for the intermediate codes
   int32_t* act_rowsum;    // INT8 variant: per token, sum of code + 128
   int32_t* inter_rowsum;  // INT8 variant: per segment row
   float* y;
@@ -147,6 +149,8 @@ ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int
   b.inter_codes = c.take<uint8_t>(A * static_cast<size_t>(I));
   b.inter_scales = c.take<float>(A);
   b.inter_gsum = c.take<float>(A * static_cast<size_t>(I / kGroup));
+  b.act_parts = c.take<uint16_t>(A * static_cast<size_t>(sum_parts_ld(H)));
+  b.inter_parts = c.take<uint16_t>(A * static_cast<size_t>(sum_parts_ld(I)));
   b.act_rowsum = c.take<int32_t>(static_cast<size_t>(T));
   b.inter_rowsum = c.take<int32_t>(A);
   b.y = c.take<float>(A * static_cast<size_t>(H));
@@ -470,7 +474,7 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
 
   // TMA descriptors: packed weights [E * rows, K / 2] bytes, 64-byte swizzle;
   // activation codes in segment order [A, K] bytes, 128-byte swizzle, 16-row boxes.
-  CUtensorMap tw1, ta1, tw2, ta2, ts1, ts2;
+  CUtensorMap tw1, ta1, tw2, ta2, ts1, ts2, tg1, tg2;
   if (w4a8_status st = encode_u8_2d(&tw1, w13_packed, static_cast<uint64_t>(H / 2),
                                     static_cast<uint64_t>(E) * 2 * I, 64, 64,
                                     CU_TENSOR_MAP_SWIZZLE_64B))
@@ -483,6 +487,15 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
                                     CU_TENSOR_MAP_SWIZZLE_64B))
     return st;
   if (w4a8_status st = encode_u8_2d(&ta2, b.inter_codes, static_cast<uint64_t>(I),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  // three-part group sums as bytes [A, 2 ld], 16 rows x 128 bytes per box
+  const bool parts = !i8 && grouped_gemm_uses_sum_parts(decode);
+  if (w4a8_status st = encode_u8_2d(&tg1, b.act_parts, static_cast<uint64_t>(2 * sum_parts_ld(H)),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&tg2, b.inter_parts,
+                                    static_cast<uint64_t>(2 * sum_parts_ld(I)),
                                     static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
   // group-major scales as bytes: [E * G, 2 * rows]; one box = one tile's scales
@@ -519,8 +532,9 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
             "route launch");
   W4A8_STEP(record(3), "cudaEventRecord");
   W4A8_STEP(record(0), "cudaEventRecord");
-  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales, b.act_gsum, b.row_of, k,
-                             b.perm_codes, di.sms, s, i8 ? b.act_rowsum : nullptr),
+  W4A8_STEP(launch_act_quant(hidden_bf16, T, H, b.act_codes, b.act_scales,
+                             parts ? nullptr : b.act_gsum, b.row_of, k, b.perm_codes, di.sms, s,
+                             i8 ? b.act_rowsum : nullptr, parts ? b.act_parts : nullptr),
             "act_quant launch");
   W4A8_STEP(record(1), "cudaEventRecord");
 
@@ -545,13 +559,14 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   g1.act_sum = b.act_rowsum;
   W4A8_STEP(record(4), "cudaEventRecord");
   W4A8_STEP(i8 ? launch_grouped_gemm_i8(true, decode, tw1, ta1, g1, di.sms, s)
-               : launch_grouped_gemm(true, decode, tw1, ta1, ts1, g1, di.sms, s),
+               : launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
             "gate/up GEMM launch");
   W4A8_STEP(record(5), "cudaEventRecord");
 
   W4A8_STEP(record(6), "cudaEventRecord");
-  W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales, b.inter_gsum,
-                                di.sms, s, i8 ? b.inter_rowsum : nullptr),
+  W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales,
+                               parts ? nullptr : b.inter_gsum, di.sms, s,
+                               i8 ? b.inter_rowsum : nullptr, parts ? b.inter_parts : nullptr),
             "intermediate quant launch");
   W4A8_STEP(record(7), "cudaEventRecord");
 
@@ -576,7 +591,7 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   g2.act_sum = b.inter_rowsum;
   W4A8_STEP(record(8), "cudaEventRecord");
   W4A8_STEP(i8 ? launch_grouped_gemm_i8(false, decode, tw2, ta2, g2, di.sms, s)
-               : launch_grouped_gemm(false, decode, tw2, ta2, ts2, g2, di.sms, s),
+               : launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),
             "down GEMM launch");
   W4A8_STEP(record(9), "cudaEventRecord");
 

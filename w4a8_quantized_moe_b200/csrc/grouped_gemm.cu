@@ -47,6 +47,12 @@
 // After the last group the epilogue applies the token (or row) scale and
 // writes h (plus the SwiGLU and absmax) or Y.
 //
+// The -8 S_g term can also be left to the tensor core (the shape's OffsetMode):
+// four more MMAs per group against a constant -2^-6 A operand, or once per
+// tile as sum_g s_g S_g, a K = G bf16 product of the tile's scales (written to
+// TMEM by the converter warps) with the rows' group sums (three bf16 parts
+// each, written by the activation quantisers), accumulated like one more group.
+//
 // Two shapes of the same kernel: a decode shape (32-token tiles, 8 A slots,
 // 8 accumulators, 3 converter sets, 16 weight stages) for batches with few
 // tokens per expert, where pipeline depth hides the MMA and TMEM latencies,
@@ -75,7 +81,7 @@ constexpr int kWStageBytes = kBM * kGroup / 2;      // 8 KB of packed INT4
 constexpr uint32_t kTmemCols = 512;
 
 template <int TileN, int WStages, int BStages, int ASlots, int DBufs, int ConvSets,
-          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetInMma>
+          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetMode>
 struct Shape {
   static constexpr int kTileN = TileN;
   static constexpr int kWStages = WStages;
@@ -88,9 +94,16 @@ struct Shape {
   static constexpr int kMmaWarps = MmaWarps;
   static constexpr int kConvWarps = 4 * ConvSets;
   static constexpr int kEpiSets = EpiSets;                // epilogue sets taking turns by tile
-  // The +8 offset of the stored nibbles is removed by the tensor core (four more
-  // MMAs per group against a constant -2^-6 operand) instead of by the epilogue.
-  static constexpr bool kOffsetInMma = OffsetInMma != 0;
+  // Where the +8 offset of the stored nibbles is removed (OffsetMode):
+  //   0  the epilogue, per group: acc += s_g * (512 D_g - 8 S_g);
+  //   1  the tensor core, per group: four more MMAs against a constant -2^-6
+  //      A operand, so that D_g holds 2^-9 sum a q;
+  //   2  the tensor core, once per tile: sum_g s_g S_g is a K = G product of the
+  //      tile's weight scales with the rows' group sums, one bf16 MMA chain
+  //      (the sums split in three bf16 parts) into one more accumulator.
+  static constexpr bool kOffsetInMma = OffsetMode == 1;
+  static constexpr bool kOffsetTile = OffsetMode == 2;
+  static constexpr bool kEpiOffset = OffsetMode == 0;
   static constexpr int kEpiPerSet = 4 * EpiPerQuad;
   static constexpr int kEpiWarps = kEpiPerSet * EpiSets;
   static constexpr int kWarpW = kConvWarps + kEpiWarps;   // TMA: packed weights
@@ -106,7 +119,7 @@ struct Shape {
   static constexpr int kTileScBufs = 2;                   // tile weight-scale buffers
   static constexpr uint32_t kTmemA = 0;                   // A slots: 32 columns each
   static constexpr uint32_t kTmemConst = ASlots * 32;     // E4M3 -2^-6 in every byte (offset MMAs)
-  static constexpr uint32_t kTmemD = kTmemConst + (OffsetInMma ? 32 : 0);  // TileN columns each
+  static constexpr uint32_t kTmemD = kTmemConst + (kOffsetInMma ? 32 : 0);  // TileN columns each
   static constexpr int kNumBars = 2 * WStages + 2 * BStages + 2 * ASlots + 2 * DBufs + 3 +
                                   2 * EpiSets * (1 + EpiPerQuad) + 2 * kTileScBufs + 1;
   static_assert(kTmemD + DBufs * TileN <= kTmemCols, "TMEM budget exceeded");
@@ -115,10 +128,13 @@ struct Shape {
   static_assert(TileN % 16 == 0 && TileN <= 256, "MMA N");
   static_assert(MmaWarps == 1 || MmaWarps == 2, "MMA issuers");
   static_assert(EpiSets == 1 || EpiSets == kTileScBufs, "one tile-scale buffer per epilogue set");
+  // the correction takes more A/B steps than accumulators per tile, and one
+  // converter set walks the tile's groups and correction chunks in order
+  static_assert(!kOffsetTile || (!kUnified && ConvSets == 1), "per-tile correction rings");
   // Runtime-sized regions (G = K / 128 groups): staged S_g, per set
   // [kEpiPerQuad][G][kSumLd] floats, and the tile scales, [kTileScBufs][G][128] bf16.
   static constexpr __host__ __device__ int sum_bytes(int G) {
-    return kOffsetInMma ? 0 : (EpiPerQuad * G * kSumLd * 4 + 127) & ~127;
+    return kEpiOffset ? (EpiPerQuad * G * kSumLd * 4 + 127) & ~127 : 0;
   }
   static constexpr __host__ __device__ int tile_sc_bytes(int G) { return 256 * G; }
   // tile_prefix and expert_offsets, [E + 1] int32 each
@@ -131,14 +147,16 @@ struct Shape {
 };
 
 // Shapes.  By default each projection takes the shape measured fastest for it;
-// W4A8_GEMM_DECODE_SHAPE / W4A8_GEMM_PREFILL_SHAPE = 1, 2, 3 force one for both.
-//                            TileN        W   B  A  D cvt epi/q ld mma sets offset-in-MMA
+// W4A8_GEMM_DECODE_SHAPE = 1..3 / W4A8_GEMM_PREFILL_SHAPE = 1..4 force one for both.
+//                            TileN        W   B  A  D cvt epi/q ld mma sets offset mode
 using DecodeOneSet  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;
 using DecodeTwoSets = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2, 0>;
 using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2, 0>;
+using DecodeTileCorr = Shape<kTileNDecode, 16, 8, 8, 7, 1, 1, 32, 2, 1, 2>;
 using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 3, 3, 1, 4, 16, 2, 1, 1>;
 using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 3, 2, 1, 2, 16, 2, 1, 1>;
 using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
+using PrefillTileCorr = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 2>;
 // INT8 per-channel shapes: one accumulator per tile, single MMA issuer
 using I8Decode  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 1, 1, 0>;
 using I8Decode2 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;  // 4 tiles x 2 chains
@@ -224,7 +242,8 @@ template <class S, bool kGateUp, bool kI8>
 __global__ void __launch_bounds__(S::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         const __grid_constant__ CUtensorMap tmap_act,
-                        const __grid_constant__ CUtensorMap tmap_sc, const GemmArgs a) {
+                        const __grid_constant__ CUtensorMap tmap_sc,
+                        const __grid_constant__ CUtensorMap tmap_gs, const GemmArgs a) {
   constexpr int kTileN = S::kTileN, kWStages = S::kWStages, kBStages = S::kBStages;
   constexpr int kASlots = S::kASlots, kDBufs = S::kDBufs, kEpiN = S::kEpiN;
   constexpr int kBStageBytes = S::kBStageBytes, kUpBytes = S::kUpBytes;
@@ -304,7 +323,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     }
     for (int i = 0; i < S::kTileScBufs; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], S::kEpiPerSet);  // a tile's scales are read by one set
+      // a tile's scales are read by one epilogue set (and, for the per-tile
+      // correction, by the 4 converter warps)
+      mbar_init(&tempty[i], S::kEpiPerSet + (S::kOffsetTile ? 4 : 0));
     }
     mbar_init(loopdone, S::kEpiPerSet);
     *abort_flag = 0;
@@ -314,7 +335,10 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_sc);
   }
-  if (warp == S::kWarpB && lane == 0) prefetch_tmap(&tmap_act);
+  if (warp == S::kWarpB && lane == 0) {
+    prefetch_tmap(&tmap_act);
+    if (S::kOffsetTile) prefetch_tmap(&tmap_gs);
+  }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -330,6 +354,16 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   const int total = sTP[a.E] * mb_count;
   const int my_tiles = blockIdx.x < total ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   const int n_groups = my_tiles * G;  // every tile has G groups
+  // Per-tile correction (offset mode 2): the rows' group sums S_g come as three
+  // bf16 parts, [rows][3 * Gp] with Gp = G rounded up to 16 (padding zero);
+  // the product with the tile's scales takes kNC more A/B ring steps of K = 64
+  // and one more accumulator per tile.
+  const int Gp = (G + 15) & ~15;
+  const int KC = 3 * Gp;
+  const int kNC = S::kOffsetTile ? (KC + 63) / 64 : 0;
+  const int ab_per_tile = G + kNC;                       // A slot / B stage steps
+  const int units_per_tile = G + (S::kOffsetTile ? 1 : 0);  // accumulators
+  const int n_units = my_tiles * units_per_tile;
 
   if (warp == S::kWarpW) {
     // ------------------------------------------------------------ TMA: packed weights
@@ -388,14 +422,19 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       const int n_ops = t.n_mma >> 4;
       const uint32_t tx = t.n_mma * kGroup;
       const int32_t y0 = static_cast<int32_t>(t.row0) + 16 * lane;
-      for (int g = 0; g < G; ++g) {
+      // G stages of codes, then (per-tile correction) kNC stages of the bf16
+      // group-sum parts, 128 bytes of each row per stage
+      for (int g = 0; g < ab_per_tile; ++g) {
         const int s = it % kBStages;
         const uint32_t ph = (it / kBStages) & 1;
         if (!mbar_wait(&bempty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
         const uint32_t dB = smem_u32(sB + s * kBStageBytes);
         if (lane == 0) mbar_arrive_expect_tx(&bfull[s], tx);
         __syncwarp();
-        if (lane < n_ops) tma_load_2d(dB + lane * 16 * kGroup, &tmap_act, &bfull[s], g * kGroup, y0);
+        if (lane < n_ops) {
+          if (g < G) tma_load_2d(dB + lane * 16 * kGroup, &tmap_act, &bfull[s], g * kGroup, y0);
+          else tma_load_2d(dB + lane * 16 * kGroup, &tmap_gs, &bfull[s], (g - G) * 128, y0);
+        }
         ++it;
       }
     }
@@ -457,20 +496,54 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       }
     } else if (lane == 0) {
       int cur = -1;
-      uint32_t idesc = 0;
-      for (int it = mw; it < n_groups; it += S::kMmaWarps) {
-        const int tl = it / G;
+      uint32_t idesc = 0, idesc_c = 0;
+      // unit = one accumulator: the tile's G groups, then (offset mode 2) the
+      // correction, whose kNC chunks one issuer runs back to back
+      for (int it = mw; it < n_units; it += S::kMmaWarps) {
+        const int tl = it / units_per_tile;
+        const int u = it - tl * units_per_tile;
         if (tl != cur) {
           cur = tl;
           const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, blockIdx.x + tl * gridDim.x);
           idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
+          idesc_c = idesc_bf16_f32_m128(static_cast<uint32_t>(t.n_mma));
         }
-        const int sb = it % kBStages;
-        const uint32_t phb = (it / kBStages) & 1;
-        const int as = it % kASlots;
-        const uint32_t pha = (it / kASlots) & 1;
         const int d = it % kDBufs;
         const uint32_t phd = (it / kDBufs) & 1;
+        if (S::kOffsetTile && u == G) {
+          if (!mbar_wait(&dempty[d], phd ^ 1, abort_flag, tmo)) break;
+          const uint32_t dt = tmem + kTmemD + d * kTileN;
+          bool okc = true;
+          for (int c = 0; c < kNC; ++c) {
+            const int ab = tl * ab_per_tile + G + c;
+            const int sb = ab % kBStages;
+            const uint32_t phb = (ab / kBStages) & 1;
+            const int as = ab % kASlots;
+            const uint32_t pha = (ab / kASlots) & 1;
+            if (!mbar_wait(&bfull[sb], phb, abort_flag, tmo) ||
+                !mbar_wait(&afull[as], pha, abort_flag, tmo)) {
+              okc = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + sb * kBStageBytes));
+            const uint32_t at = tmem + kTmemA + as * 32;
+            const int nk = min(4, (KC - 64 * c) >> 4);   // K = 16 bf16 per MMA
+            for (int kk = 0; kk < nk; ++kk)
+              mma_bf16_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc_c,
+                          (c > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&aempty[as]);
+            tc_commit(&bempty[sb]);
+          }
+          if (!okc) break;
+          tc_commit(&dfull[d]);
+          continue;
+        }
+        const int ab = S::kOffsetTile ? tl * ab_per_tile + u : it;
+        const int sb = ab % kBStages;
+        const uint32_t phb = (ab / kBStages) & 1;
+        const int as = ab % kASlots;
+        const uint32_t pha = (ab / kASlots) & 1;
         // poll all three at once (each poll is a ~100-cycle round trip)
         const bool rd = mbar_test_wait(&dempty[d], phd ^ 1);
         const bool rb = mbar_test_wait(&bfull[sb], phb);
@@ -525,16 +598,17 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
     }
-    for (int it = set; it < n_groups; it += S::kConvSets) {
-      const int s = it % kWStages;
-      const uint32_t ph = (it / kWStages) & 1;
-      const int as = it % kASlots;
-      const uint32_t pha = (it / kASlots) & 1;
+    // one weight group: W stage wit -> A slot ait
+    auto convert = [&](int wit, int ait) -> bool {
+      const int s = wit % kWStages;
+      const uint32_t ph = (wit / kWStages) & 1;
+      const int as = ait % kASlots;
+      const uint32_t pha = (ait / kASlots) & 1;
       const bool rw = mbar_test_wait(&wfull[s], ph);   // both polls in flight at once
       const bool ra = mbar_test_wait(&aempty[as], pha ^ 1);
       if (!(rw && ra) && (!mbar_wait(&wfull[s], ph, abort_flag, tmo) ||
                           !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo)))
-        break;
+        return false;
       tc_fence_after();
       const uint32_t row = smem_u32(sW + s * kWStageBytes) + m * 64;
       uint32_t r[32];
@@ -555,6 +629,53 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&afull[as]);
+      return true;
+    };
+    if constexpr (S::kOffsetTile) {
+      // per tile: the G weight groups, then the correction's A operand, kNC
+      // slots of bf16 pairs: column k of the correction is the row's scale of
+      // group k mod Gp (zero past G), repeated for the three parts of S_g
+      const int sc_off = kGateUp ? (m < 64 ? m : 64 * G + (m - 64)) : m;
+      constexpr int kScStride = kGateUp ? 64 : 128;
+      int ait = 0;
+      bool ok = true;
+      for (int nt = 0; ok && nt < my_tiles; ++nt) {
+        for (int g = 0; g < G; ++g)
+          if (!convert(nt * G + g, ait++)) { ok = false; break; }
+        if (!ok) break;
+        const int tb = nt % S::kTileScBufs;
+        if (!mbar_wait(&tfull[tb], (nt / S::kTileScBufs) & 1, abort_flag, tmo)) break;
+        const uint16_t* sTs = reinterpret_cast<const uint16_t*>(sT + tb * S::tile_sc_bytes(G)) + sc_off;
+        for (int c = 0; c < kNC; ++c, ++ait) {
+          const int as = ait % kASlots;
+          if (!mbar_wait(&aempty[as], ((ait / kASlots) & 1) ^ 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {   // 16 columns of K (8 TMEM columns) per part run
+            const int kb = 64 * c + 16 * j;
+            const int part = kb < KC ? kb / Gp : 3;
+            const int gb = kb - part * Gp;
+#pragma unroll
+            for (int t2 = 0; t2 < 8; ++t2) {
+              const int g0 = gb + 2 * t2;
+              const uint32_t lo = part < 3 && g0 < G ? sTs[g0 * kScStride] : 0u;
+              const uint32_t hi = part < 3 && g0 + 1 < G ? sTs[(g0 + 1) * kScStride] : 0u;
+              r[8 * j + t2] = lo | (hi << 16);
+            }
+          }
+          tmem_st_32x32b_x32(tmem + lane_base + kTmemA + as * 32, r);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[as]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+      }
+    } else {
+      for (int it = set; it < n_groups; it += S::kConvSets)
+        if (!convert(it, it)) break;
     }
   } else if (warp < S::kWarpW) {
     // ------------------------------------------------------------ epilogue
@@ -580,7 +701,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     for (int tile = blockIdx.x + set * gridDim.x, ntile = set; ok && tile < total;
          tile += S::kEpiSets * gridDim.x, ntile += S::kEpiSets) {
       const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
-      int it = ntile * G;                           // CTA-wide index of the tile's first group
+      int it = ntile * units_per_tile;              // CTA-wide index of the tile's first unit
       const uint32_t lt = ntile / S::kEpiSets;      // this set's tile count: barrier phases
       // token (gate/up) or row (down) scales of this warp's columns, lane-strided;
       // loaded now so their latency hides behind the group loop
@@ -651,7 +772,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         if (lane == 0) mbar_arrive(&dempty[d]);
       } else {
       const uint32_t phs = lt & 1;
-      if constexpr (!S::kOffsetInMma) {  // stage S_g of this warp's quarter of the slice's columns
+      if constexpr (S::kEpiOffset) {  // stage S_g of this warp's quarter of the slice's columns
         constexpr int kTok = kEpiN / 4;
         if (!mbar_wait(my_sempty, phs ^ 1, abort_flag, tmo)) break;
         constexpr int kBatch = kTok < 8 ? kTok : 8;   // loads in flight per lane
@@ -682,7 +803,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(my_sfull);
       }
-      if (!S::kOffsetInMma && !mbar_wait(my_sfull, phs, abort_flag, tmo)) break;
+      if (S::kEpiOffset && !mbar_wait(my_sfull, phs, abort_flag, tmo)) break;
       const int tb = ntile % S::kTileScBufs;
       if (!mbar_wait(&tfull[tb], (ntile / S::kTileScBufs) & 1, abort_flag, tmo)) break;
       const __nv_bfloat16* sTm =
@@ -695,9 +816,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       for (int j = 0; j < kEpiN / 2; ++j) acc2[j] = make_float2(0.0f, 0.0f);
       int d = it % kDBufs;
       uint32_t phd = (it / kDBufs) & 1;
-      for (int g = 0; g < G; ++g) {
-        const float sg = __bfloat162float(sTm[g * kScStride]);
-        const float2 s512x2 = make_float2(sg * 512.0f, sg * 512.0f);
+      // units: the G groups, then (offset mode 2) the correction sum_g s_g S_g,
+      // which enters with the factor -8
+      for (int g = 0; g < units_per_tile; ++g) {
+        const float sg = g < G ? __bfloat162float(sTm[g * kScStride]) : 0.0f;
+        const float f = g < G ? sg * 512.0f : -8.0f;
+        const float2 s512x2 = make_float2(f, f);
         const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
         const float* sg_row = sSl + g * kSumLd;
         if (!mbar_wait(&dfull[d], phd, abort_flag, tmo)) { ok = false; break; }
@@ -718,7 +842,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
               acc2[o + 1] = __ffma2_rn(
                   s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
                   acc2[o + 1]);
-              if constexpr (!S::kOffsetInMma) {  // remove the +8 offset: - 8 s_g S_g
+              if constexpr (S::kEpiOffset) {  // remove the +8 offset: - 8 s_g S_g
                 const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
                 acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
                 acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
@@ -743,7 +867,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        if (!S::kOffsetInMma) mbar_arrive(my_sempty);
+        if (S::kEpiOffset) mbar_arrive(my_sempty);
         mbar_arrive(&tempty[tb]);
         if (S::kEpiSets > 1) mbar_arrive(loopdone);
       }
@@ -827,8 +951,8 @@ constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in limit of sm_100
 
 template <class S, bool kGateUp, bool kI8 = false>
 cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
-                         const CUtensorMap& tmap_sc, const GemmArgs& a, int num_ctas,
-                         cudaStream_t s) {
+                         const CUtensorMap& tmap_sc, const CUtensorMap& tmap_gs,
+                         const GemmArgs& a, int num_ctas, cudaStream_t s) {
   static_assert(S::smem_bytes(kGateUp, kMaxGroups, kMaxExperts) <= kMaxSmemPerBlock,
                 "shared memory");
   static bool attr_set[64] = {};
@@ -844,16 +968,16 @@ cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
   }
   const int smem = S::smem_bytes(kGateUp, a.K / kGroup, a.E);
   grouped_gemm_kernel<S, kGateUp, kI8><<<num_ctas, S::kThreads, smem, s>>>(tmap_w, tmap_act,
-                                                                           tmap_sc, a);
+                                                                           tmap_sc, tmap_gs, a);
   return cudaGetLastError();
 }
 
 template <class S>
 cudaError_t launch_either(bool gate_up, const CUtensorMap& tw, const CUtensorMap& ta,
-                          const CUtensorMap& tsc, const GemmArgs& a, int num_ctas,
-                          cudaStream_t s) {
-  return gate_up ? launch_shape<S, true>(tw, ta, tsc, a, num_ctas, s)
-                 : launch_shape<S, false>(tw, ta, tsc, a, num_ctas, s);
+                          const CUtensorMap& tsc, const CUtensorMap& tgs, const GemmArgs& a,
+                          int num_ctas, cudaStream_t s) {
+  return gate_up ? launch_shape<S, true>(tw, ta, tsc, tgs, a, num_ctas, s)
+                 : launch_shape<S, false>(tw, ta, tsc, tgs, a, num_ctas, s);
 }
 
 int shape_choice(const char* env) {
@@ -861,31 +985,47 @@ int shape_choice(const char* env) {
   return v ? std::atoi(v) : 0;
 }
 
+int prefill_shape() {
+  static const int pshape = shape_choice("W4A8_GEMM_PREFILL_SHAPE");
+  return pshape != 0 ? pshape : 1;
+}
+
+int decode_shape_forced() {
+  static const int dshape = shape_choice("W4A8_GEMM_DECODE_SHAPE");
+  return dshape;
+}
+
 }  // namespace
 
 int grouped_gemm_tile_n(bool decode) { return decode ? kTileNDecode : kTileNPrefill; }
 
+bool grouped_gemm_uses_sum_parts(bool decode) {
+  return decode ? decode_shape_forced() == 4 : prefill_shape() == 4;
+}
+
 cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_act, const CUtensorMap& tmap_sc,
-                                const GemmArgs& a, int num_ctas, cudaStream_t s) {
-  static const int dshape = shape_choice("W4A8_GEMM_DECODE_SHAPE");
-  static const int pshape = shape_choice("W4A8_GEMM_PREFILL_SHAPE");
+                                const CUtensorMap& tmap_gs, const GemmArgs& a, int num_ctas,
+                                cudaStream_t s) {
+  const int dshape = decode_shape_forced();
   if (a.K % kGroup || a.K / kGroup > kMaxGroups || a.K <= 0) return cudaErrorInvalidValue;
+  const CUtensorMap &tw = tmap_w, &ta = tmap_act, &tsc = tmap_sc, &tgs = tmap_gs;
   if (decode) {
     // gate/up (48 groups per tile at H = 6144) runs best with one epilogue set
     // and a deep weight ring; down (16 groups per tile) with two epilogue sets,
     // whose tile finalize then overlaps the other set's groups
     const int d = dshape != 0 ? dshape : (gate_up ? 1 : 2);
-    if (d == 1) return launch_either<DecodeOneSet>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
-    if (d == 3) return launch_either<DecodeTwoCvt>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
-    return launch_either<DecodeTwoSets>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    if (d == 1) return launch_either<DecodeOneSet>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
+    if (d == 3) return launch_either<DecodeTwoCvt>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
+    if (d == 4) return launch_either<DecodeTileCorr>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
+    return launch_either<DecodeTwoSets>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
   }
-  const int p = pshape != 0 ? pshape : 1;
-  if (p == 2) return launch_either<Prefill8Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+  const int p = prefill_shape();
+  if (p == 2) return launch_either<Prefill8Epi>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
   if (p == 3)
-    return launch_either<Prefill16EpiEpilogueOffset>(gate_up, tmap_w, tmap_act, tmap_sc, a,
-                                                     num_ctas, s);
-  return launch_either<Prefill16Epi>(gate_up, tmap_w, tmap_act, tmap_sc, a, num_ctas, s);
+    return launch_either<Prefill16EpiEpilogueOffset>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
+  if (p == 4) return launch_either<PrefillTileCorr>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
+  return launch_either<Prefill16Epi>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
 }
 
 namespace {
@@ -918,13 +1058,13 @@ cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap&
   if (a.K % kGroup || a.K / kGroup > kMaxGroups || a.K <= 0) return cudaErrorInvalidValue;
   // the tile-scale map is unused in this mode; any valid map fills the slot
   if (decode && a.K / kGroup >= 2)  // two accumulation chains need two groups per tile
-    return gate_up ? launch_shape<I8Decode2, true, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s)
-                   : launch_shape<I8Decode2, false, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s);
+    return gate_up ? launch_shape<I8Decode2, true, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s)
+                   : launch_shape<I8Decode2, false, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s);
   if (decode)
-    return gate_up ? launch_shape<I8Decode, true, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s)
-                   : launch_shape<I8Decode, false, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s);
-  return gate_up ? launch_shape<I8Prefill, true, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s)
-                 : launch_shape<I8Prefill, false, true>(tmap_w, tmap_act, tmap_w, a, num_ctas, s);
+    return gate_up ? launch_shape<I8Decode, true, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s)
+                   : launch_shape<I8Decode, false, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s);
+  return gate_up ? launch_shape<I8Prefill, true, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s)
+                 : launch_shape<I8Prefill, false, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s);
 }
 
 cudaError_t read_and_clear_device_error(int* value) {

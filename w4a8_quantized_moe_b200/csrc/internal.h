@@ -17,6 +17,13 @@ constexpr int kMaxTopK = 32;
 constexpr int kMaxGroups = 64;     // K / 128 per GEMM (K <= 8192)
 
 inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok; }
+// Three-part group sums (per-tile offset correction): one part spans Gp =
+// K / 128 groups rounded up to 16 columns; a row holds the three parts and is
+// at least 64 columns (one 128-byte TMA box) long.
+__host__ __device__ inline int64_t sum_part_cols(int64_t K) { return ((K / kGroup) + 15) / 16 * 16; }
+__host__ __device__ inline int64_t sum_parts_ld(int64_t K) {
+  return 3 * sum_part_cols(K) < 64 ? 64 : 3 * sum_part_cols(K);
+}
 
 // ---- kernels_small.cu
 // gsum (nullable): [T, H / 128] sums of the E4M3 values of each 128-wide group.
@@ -24,9 +31,13 @@ inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok;
 // receives token t's codes for every slot j.
 // int8_row_sum (non-null): INT8 mode instead of E4M3 -- codes are offset-binary
 // (code + 128) and the row sums of those bytes go to int8_row_sum [T].
+// sum_parts (nullable, needs perm): [T * k, sum_parts_ld(H)] bf16; segment row r gets each group sum S as three bf16 parts p0 =
+// bf16(S), p1 = bf16(S - p0), p2 = bf16(S - p0 - p1) at columns g, Gp + g,
+// 2 Gp + g, and zeros at the padding columns.
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
                              float* gsum, const int32_t* row_of, int k, uint8_t* perm,
-                             int num_sms, cudaStream_t s, int32_t* int8_row_sum = nullptr);
+                             int num_sms, cudaStream_t s, int32_t* int8_row_sum = nullptr,
+                             uint16_t* sum_parts = nullptr);
 // clip_search: the per-group MSE search over 11 shrink ratios instead of absmax / 7.
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
                              bool clip_search, int num_sms, cudaStream_t s);
@@ -37,9 +48,11 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                          int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
                          cudaStream_t s);
+// sum_parts (nullable): [A, sum_parts_ld(I)] bf16 as for launch_act_quant.
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, float* gsum, int num_sms,
-                               cudaStream_t s, int32_t* int8_row_sum = nullptr);
+                               cudaStream_t s, int32_t* int8_row_sum = nullptr,
+                               uint16_t* sum_parts = nullptr);
 // packed uint4b8 words -> the word-local nibble interleave the grouped GEMM reads.
 cudaError_t launch_repack_int4_b200(const int32_t* in, int64_t nwords, int32_t* out, int num_sms,
                                     cudaStream_t s);
@@ -80,10 +93,18 @@ struct GemmArgs {
 // decode = the shape for few tokens per expert (see grouped_gemm.cu).
 // tmap_sc: the group-major weight scales as bytes [E * K / 128, 2 * n_rows],
 // box [K / 128 rows, 128 bytes (gate/up) or 256 bytes (down)].
+// tmap_gs (read only when grouped_gemm_uses_sum_parts(decode)): the rows' E4M3
+// group sums as three bf16 parts, bytes [act rows, 2 * sum_parts_ld(K)], part p
+// of group g at column p * Gp + g (Gp = sum_part_cols(K)), zero up to 3 * Gp;
+// box [16 rows x 128 bytes], 128-byte swizzle.
 cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tmap_w,
                                 const CUtensorMap& tmap_act, const CUtensorMap& tmap_sc,
-                                const GemmArgs& a, int num_ctas, cudaStream_t s);
+                                const CUtensorMap& tmap_gs, const GemmArgs& a, int num_ctas,
+                                cudaStream_t s);
 int grouped_gemm_tile_n(bool decode);
+// Whether the shape for this regime removes the +8 nibble offset once per
+// tile (and so reads the three-part group sums instead of act_gsum).
+bool grouped_gemm_uses_sum_parts(bool decode);
 // The per-channel INT4 x per-token INT8 grouped GEMM (kind::i8, one int32
 // accumulator per tile); tmap_act holds offset-binary codes.
 cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap& tmap_w,

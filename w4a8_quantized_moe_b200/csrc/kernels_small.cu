@@ -79,6 +79,22 @@ __device__ __forceinline__ float sum8_e4m3(uint2 c) {
   return s;
 }
 
+// A group sum as three bf16 parts, p0 + p1 + p2 = S to ~2^-27 |S| (each
+// remainder is exact in FP32), at columns g, gp + g, 2 gp + g of `row`; the
+// writer of the last group also zeroes the padding columns G .. gp - 1.
+__device__ __forceinline__ void store_sum_parts(uint16_t* row, float S, int g, int G, int gp) {
+  const __nv_bfloat16 p0 = __float2bfloat16_rn(S);
+  const float r1 = S - __bfloat162float(p0);
+  const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(p1);
+  const __nv_bfloat16 p2 = __float2bfloat16_rn(r2);
+  row[g] = __bfloat16_as_ushort(p0);
+  row[gp + g] = __bfloat16_as_ushort(p1);
+  row[2 * gp + g] = __bfloat16_as_ushort(p2);
+  if (g == G - 1)
+    for (int z = G; z < gp; ++z) row[z] = row[gp + z] = row[2 * gp + z] = 0;
+}
+
 __device__ __forceinline__ void unpack8(uint4 c, float (&v)[8]) {
   v[0] = bf16_lo(c.x); v[1] = bf16_hi(c.x); v[2] = bf16_lo(c.y); v[3] = bf16_hi(c.y);
   v[4] = bf16_lo(c.z); v[5] = bf16_hi(c.z); v[6] = bf16_lo(c.w); v[7] = bf16_hi(c.w);
@@ -116,7 +132,8 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
                                                                const int32_t* __restrict__ row_of,
                                                                int k,
                                                                uint8_t* __restrict__ perm,
-                                                               int32_t* __restrict__ row_sum) {
+                                                               int32_t* __restrict__ row_sum,
+                                                               uint16_t* __restrict__ parts) {
   __shared__ float red[kAqThreads / 32];
   __shared__ int ired[kAqThreads / 32];
   __shared__ int64_t dst_rows[kMaxTopK];
@@ -148,6 +165,9 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
     if (threadIdx.x == 0) scales[t] = scale;
     uint2* out = reinterpret_cast<uint2*>(codes + t * H);
     float* gs = !kInt8 && gsum ? gsum + t * (H / kGroup) : nullptr;
+    const bool want_sums = !kInt8 && (gsum || parts);
+    const int G = static_cast<int>(H / kGroup);
+    const int gp = (G + 15) / 16 * 16;
     int isum = 0;  // INT8: this thread's share of the row's offset-binary code sum
     // Every thread runs every chunk slot (the slot bounds are uniform) so that
     // the 16-lane group reductions see full warps.
@@ -161,14 +181,19 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
         if (perm)  // the token's codes again at each of its k segment rows
           for (int j = 0; j < k; ++j) reinterpret_cast<uint2*>(perm + dst_rows[j] * H)[c] = q;
         if (kInt8) isum += sum8_u8(q);
-        if (gs) part = sum8_e4m3(q);
+        if (want_sums) part = sum8_e4m3(q);
       }
-      if (gs) {
+      if (want_sums) {
         part += __shfl_xor_sync(kFull, part, 8);
         part += __shfl_xor_sync(kFull, part, 4);
         part += __shfl_xor_sync(kFull, part, 2);
         part += __shfl_xor_sync(kFull, part, 1);
-        if (c < nchunk && (c & 15) == 0) gs[c >> 4] = part;
+        if (c < nchunk && (c & 15) == 0) {
+          if (gs) gs[c >> 4] = part;
+          if (parts)
+            for (int j = 0; j < k; ++j)
+              store_sum_parts(parts + dst_rows[j] * sum_parts_ld(H), part, static_cast<int>(c >> 4), G, gp);
+        }
       }
     };
 #pragma unroll
@@ -499,8 +524,12 @@ __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restric
                                                           uint8_t* __restrict__ codes,
                                                           float* __restrict__ scales,
                                                           float* __restrict__ gsum,
-                                                          int32_t* __restrict__ row_sum) {
+                                                          int32_t* __restrict__ row_sum,
+                                                          uint16_t* __restrict__ parts) {
   const int64_t per_row = I / 16;
+  const bool want_sums = !kInt8 && (gsum || parts);
+  const int G = static_cast<int>(I / kGroup);
+  const int gp = (G + 15) / 16 * 16;
   const int64_t n = A * per_row;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t n_iter = (n + stride - 1) / stride;
@@ -526,13 +555,16 @@ __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restric
       *reinterpret_cast<uint4*>(codes + r * I + c * 16) =
           make_uint4(out[0].x, out[0].y, out[1].x, out[1].y);
       if (kInt8) atomicAdd(row_sum + r, sum8_u8(out[0]) + sum8_u8(out[1]));  // exact, any order
-      else if (gsum) part = sum8_e4m3(out[0]) + sum8_e4m3(out[1]);
+      else if (want_sums) part = sum8_e4m3(out[0]) + sum8_e4m3(out[1]);
     }
-    if (!kInt8 && gsum) {
+    if (want_sums) {
       part += __shfl_xor_sync(kFull, part, 4);
       part += __shfl_xor_sync(kFull, part, 2);
       part += __shfl_xor_sync(kFull, part, 1);
-      if (active && (c & 7) == 0) gsum[r * (I / kGroup) + (c >> 3)] = part;
+      if (active && (c & 7) == 0) {
+        if (gsum) gsum[r * (I / kGroup) + (c >> 3)] = part;
+        if (parts) store_sum_parts(parts + r * sum_parts_ld(I), part, static_cast<int>(c >> 3), G, gp);
+      }
     }
   }
 }
@@ -616,19 +648,20 @@ inline int grid_for(int64_t work_items, int threads, int num_sms, int per_sm = 8
 
 cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes, float* scales,
                              float* gsum, const int32_t* row_of, int k, uint8_t* perm, int num_sms,
-                             cudaStream_t s, int32_t* int8_row_sum) {
+                             cudaStream_t s, int32_t* int8_row_sum, uint16_t* sum_parts) {
   if (T == 0) return cudaSuccess;
   if (perm && (!row_of || k < 1 || k > kMaxTopK)) return cudaErrorInvalidValue;
+  if (sum_parts && (!perm || int8_row_sum)) return cudaErrorInvalidValue;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(T < cap ? T : cap);
   if (int8_row_sum)
     act_quant_kernel<true><<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H,
                                                        codes, scales, nullptr, row_of, k, perm,
-                                                       int8_row_sum);
+                                                       int8_row_sum, nullptr);
   else
     act_quant_kernel<false><<<grid, kAqThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, H,
                                                         codes, scales, gsum, row_of, k, perm,
-                                                        nullptr);
+                                                        nullptr, sum_parts);
   return cudaGetLastError();
 }
 
@@ -685,17 +718,18 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
 
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, float* gsum, int num_sms,
-                               cudaStream_t s, int32_t* int8_row_sum) {
+                               cudaStream_t s, int32_t* int8_row_sum, uint16_t* sum_parts) {
   if (A == 0) return cudaSuccess;
   const int grid = grid_for(A * (I / 16), 256, num_sms);
   if (int8_row_sum) {
     cudaError_t err = cudaMemsetAsync(int8_row_sum, 0, static_cast<size_t>(A) * sizeof(int32_t), s);
     if (err != cudaSuccess) return err;
+    if (sum_parts) return cudaErrorInvalidValue;
     inter_quant_kernel<true><<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, nullptr,
-                                                  int8_row_sum);
+                                                  int8_row_sum, nullptr);
   } else {
     inter_quant_kernel<false><<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, gsum,
-                                                   nullptr);
+                                                   nullptr, sum_parts);
   }
   return cudaGetLastError();
 }

@@ -183,6 +183,27 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// Instruction descriptor: kind::f16, A = B = BF16, D = F32, both K-major,
+// M = 128, N = n (multiple of 16, 16..256).
+__host__ __device__ __forceinline__ uint32_t idesc_bf16_f32_m128(uint32_t n) {
+  return (1u << 4)                 // D format: F32
+         | (1u << 7) | (1u << 10)  // A, B format: BF16
+         | ((n >> 3) << 17)        // N >> 3
+         | ((128u >> 4) << 24);    // M >> 4
+}
+
+// D (TMEM, F32) (+)= A (TMEM, bf16) x B (SMEM descriptor, bf16), kind::f16,
+// K = 16 (32 bytes of each operand row, 8 TMEM columns of A).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle, rows of 128 B,
 // 8-row atoms 1024 B apart.  `saddr` must be 1024-byte aligned (base offset 0);
 // advancing K inside the 128-byte row adds the byte offset >> 4 to the start.
