@@ -26,6 +26,9 @@ Sources.  The method is described by five web pages about 4-bit-weight /
   per-channel INT4 experts; dynamic per-token INT8 activations).
 * "From 755GB to 395GB" (Bitdeer AI blog): 256 routed experts per MoE layer,
   3 projections per expert.
+* The non-expert layers, the shared expert among them, keep FP8 E4M3 weights
+  with 128 x 128 block scales (GLM-5.3-W4A8 model card, intro and
+  "quantisation method"); ``shared.py`` is that expert.
 
 Steps the pages leave open are fixed by the plainest reading; each function's
 docstring states the reading it takes.  Where a float decides an integer (an
@@ -45,10 +48,14 @@ from .quant import (rtn_quantize_int4, mse_clip_quantize_int4, CLIP_RATIOS, pack
                     unpack_uint4b8, dequantize_int4, quant_act_fp8_per_token,
                     quant_act_int8_per_token, rtn_quantize_int4_channel)
 from .moe import route_topk, permute_by_expert, moe_forward, ExpertStore
+from .shared import (quant_fp8_block, dequant_fp8_block, quant_act_fp8_group,
+                     dequant_act_fp8_group, shared_expert_forward)
 
 __all__ = ["bf16_bits_to_f64", "f64_to_bf16_bits", "bf16_round", "f32_round",
            "e4m3_decode", "e4m3_encode", "E4M3_MAX", "rtn_quantize_int4",
            "mse_clip_quantize_int4", "CLIP_RATIOS",
            "pack_uint4b8", "unpack_uint4b8", "dequantize_int4",
            "quant_act_fp8_per_token", "quant_act_int8_per_token", "route_topk", "permute_by_expert",
-           "moe_forward", "ExpertStore", "rtn_quantize_int4_channel"]
+           "moe_forward", "ExpertStore", "rtn_quantize_int4_channel", "quant_fp8_block",
+           "dequant_fp8_block", "quant_act_fp8_group", "dequant_act_fp8_group",
+           "shared_expert_forward"]

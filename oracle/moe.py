@@ -22,7 +22,9 @@ the combine.  Readings taken here:
   as the input activations (scale = float32(absmax / 448));
 * down: Y = (h-scale * h-codes) @ (q2 * s2)^T;
 * combine: out[t] = bf16(sum_j w[t, j] * Y[row_of[t, j]]), summed in slot
-  order; no extra routed scaling factor, no shared expert.
+  order; no extra routed scaling factor.  With a shared expert (the FP8-block
+  expert of ``shared.py``), its output is added to that sum before the bf16
+  rounding.
 
 All products and sums are float64; the only roundings are the quantisation
 points of the method (bf16 scales, INT4 values, FP8 codes, float32 scales and
@@ -37,6 +39,7 @@ import numpy as np
 from .numerics import bf16_round, e4m3_decode, f32_round
 from .quant import (dequantize_int4, pack_uint4b8, quant_act_fp8_per_token,
                     quant_act_int8_per_token, rtn_quantize_int4)
+from .shared import shared_expert_forward
 
 
 def route_topk(logits, k: int):
@@ -111,7 +114,7 @@ def _silu(x):
 
 def moe_forward(hidden, logits, experts: Sequence, k: int,
                 tokens: Optional[np.ndarray] = None, hidden_of_tokens=None,
-                act_format: str = "fp8"):
+                act_format: str = "fp8", shared=None):
     """The whole layer for all tokens, or for the token subset ``tokens``.
 
     ``hidden``: float64 [T, H] (bf16 values); ``logits``: float32 [T, E];
@@ -124,6 +127,11 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
     ``act_format``: "fp8" (E4M3 per-token activations, the W4A8 layer) or
     "int8" (symmetric INT8 per-token activations, the per-channel variant; the
     experts' scales then have one column per row).
+
+    ``shared``: optional FP8-block shared expert ``(w13_codes, w13_scales,
+    w2_codes, w2_scales)``; its ``shared_expert_forward`` result for the rows
+    of ``tokens`` is returned under ``shared`` and its ``y`` is added to the
+    routed sum before the bf16 rounding.
 
     Returns a dict with ``topk_ids``, ``topk_w``, ``expert_offsets``,
     ``sorted_token_ids``, ``row_of``, ``act_codes`` / ``act_scales`` (rows of
@@ -177,14 +185,17 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
             inter_codes[int(r)] = hc[i]
             inter_scales[int(r)] = float(hs[i])
 
+    sh = shared_expert_forward(x_rows, *shared) if shared is not None else None
     out = np.zeros((len(tokens), H), dtype=np.float64)
     for i, t in enumerate(tokens):
         acc = np.zeros(H, dtype=np.float64)
         for j in range(k):
             acc = acc + float(w[t, j]) * Y[int(row_of[t, j])]
+        if sh is not None:
+            acc = acc + sh["y"][i]
         out[i] = bf16_round(acc)
 
     return dict(topk_ids=ids, topk_w=w, expert_offsets=offsets, sorted_token_ids=sorted_tok,
                 row_of=row_of, act_codes=codes, act_scales=a_scale, inter_h=inter_h,
                 inter_codes=inter_codes, inter_scales=inter_scales, y_rows=Y, out=out,
-                tokens=tokens)
+                tokens=tokens, shared=sh)

@@ -150,3 +150,14 @@ def gen_expert_weights(cfg: MoEConfig, e: int, device="cpu"):
     w2 = (torch.randn(cfg.H, cfg.I, generator=g, device=device, dtype=torch.float32)
           * cfg.weight_std).to(torch.bfloat16)
     return w13, w2
+
+
+def gen_shared_weights(cfg: MoEConfig, device="cpu"):
+    """(w13 bf16 [2I, H], w2 bf16 [H, I]) of the shared expert, which has the
+    routed experts' shape (its own seed stream)."""
+    g = _gen(cfg.seed * 1000003 + 7, device)
+    w13 = (torch.randn(2 * cfg.I, cfg.H, generator=g, device=device, dtype=torch.float32)
+           * cfg.weight_std).to(torch.bfloat16)
+    w2 = (torch.randn(cfg.H, cfg.I, generator=g, device=device, dtype=torch.float32)
+          * cfg.weight_std).to(torch.bfloat16)
+    return w13, w2
