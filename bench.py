@@ -32,6 +32,7 @@ import workloads  # noqa: E402
 METRIC = "MoE-layer tokens/s on 1 B200 + % of HBM (decode) / FP8-peak (prefill) roofline"
 DEFAULT_CONFIG = workloads.CONFIGS[1].name
 KERNELS_PER_STEP = 8   # act_quant, route topk/scan/scatter, gemm1, inter_quant, gemm2, combine
+SHARED_KERNELS_PER_STEP = 5   # tables, input group quant, gate/up GEMM, h group quant, down GEMM
 
 
 def peaks():
@@ -137,6 +138,11 @@ def build_layer(cfg, device, w4, variant: str = "w4a8"):
     p2, s2g = w4.w4a8_prepare_experts_b200(p2, s2, packed_out=p2)
     torch.cuda.synchronize(device)
     del s13, s2
+    if variant == "w4a8+shared":   # plus the FP8 128x128-block shared expert
+        ws13, ws2 = workloads.gen_shared_weights(cfg, device=device)
+        shared = w4.SharedExpertFP8.from_bf16(ws13, ws2)
+        torch.cuda.synchronize(device)
+        return w4.W4A8MoELayerShared(p13, s13g, p2, s2g, cfg.k, shared)
     return w4.W4A8MoELayer(p13, s13g, p2, s2g, cfg.k)
 
 
@@ -193,6 +199,17 @@ def algorithmic_work(cfg, counts, variant: str = "w4a8"):
     return g1, g2, active
 
 
+def shared_work(cfg):
+    """Algorithmic bytes and FLOPs of the shared expert's two GEMMs (E4M3 weights,
+    one float32 scale per 128 x 128 block, per-token-group activation scales)."""
+    T, H, I = cfg.T, cfg.H, cfg.I
+    s1 = dict(bytes=2 * I * H + (2 * I // 128) * (H // 128) * 4 + T * H + T * (H // 128) * 4
+              + T * I * 4, flops=2 * T * 2 * I * H)
+    s2 = dict(bytes=H * I + (H // 128) * (I // 128) * 4 + T * I + T * (I // 128) * 4 + T * H * 4,
+              flops=2 * T * H * I)
+    return s1, s2
+
+
 class OracleSample:
     """The CPU oracle on a seeded sample of tokens, experts quantised up front."""
 
@@ -200,6 +217,7 @@ class OracleSample:
         import oracle
         self.oracle, self.cfg = oracle, cfg
         self.act_format = "int8" if variant == "channel-int8" else "fp8"
+        self.shared = None
         try:
             from threadpoolctl import threadpool_info
             self.cores = max((p.get("num_threads", 1) for p in threadpool_info()), default=None)
@@ -223,11 +241,15 @@ class OracleSample:
             quantize=oracle.rtn_quantize_int4_channel if self.act_format == "int8" else None)
         for e in sorted(set(ids[self.tokens].reshape(-1).tolist())):
             self.store[e]                          # quantise outside the timed region
+        if variant == "w4a8+shared":
+            a, b = workloads.gen_shared_weights(cfg)
+            self.shared = (*oracle.quant_fp8_block(f(a)), *oracle.quant_fp8_block(f(b)))
 
     def run(self) -> float:
         t0 = time.perf_counter()
         self.oracle.moe_forward(self.hidden, self.logits, self.store, self.cfg.k,
-                                tokens=self.tokens, act_format=self.act_format)
+                                tokens=self.tokens, act_format=self.act_format,
+                                shared=self.shared)
         return time.perf_counter() - t0
 
     def describe(self, dt: float) -> str:
@@ -281,9 +303,10 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="run the workload with this many experts instead (a smaller case for "
                          "profiler captures; recorded in config)")
-    ap.add_argument("--variant", default="w4a8", choices=["w4a8", "channel-int8"],
+    ap.add_argument("--variant", default="w4a8", choices=["w4a8", "channel-int8", "w4a8+shared"],
                     help="w4a8: group-128 INT4 experts x FP8 E4M3 activations (default); "
-                         "channel-int8: per-channel INT4 experts x per-token INT8 activations")
+                         "channel-int8: per-channel INT4 experts x per-token INT8 activations; "
+                         "w4a8+shared: w4a8 plus the FP8 128x128-block shared expert")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload with this many tokens instead (a smaller case for "
                          "profiler captures; recorded in config)")
@@ -323,13 +346,20 @@ def main():
     offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
 
+    shared = args.variant == "w4a8+shared"
+    n_ev = 2 * w4.NUM_STAGES + (8 if shared else 0)
+
     def step(events=None):
         if events:
             # torch only reports elapsed time for events it recorded itself; the
             # library re-records each one at its stage boundary later in the stream
             for e in events:
                 e.record(stream)
-        layer(hidden, logits, out=out, aux={"expert_offsets": offsets}, stage_events=events)
+        kw = {}
+        if shared:
+            kw["shared_stage_events"] = events[2 * w4.NUM_STAGES:] if events else None
+            events = events[:2 * w4.NUM_STAGES] if events else None
+        layer(hidden, logits, out=out, aux={"expert_offsets": offsets}, stage_events=events, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -337,7 +367,7 @@ def main():
     counts = np.diff(offsets.cpu().numpy().astype(np.int64))
 
     # ---------------- device-resident timing (kernel path)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * w4.NUM_STAGES)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
@@ -354,7 +384,7 @@ def main():
     w4.w4a8_check_device_error(device)
     ms = t_start.elapsed_time(t_end)
     stage_ms = [statistics.mean(ev[i][2 * s].elapsed_time(ev[i][2 * s + 1])
-                                for i in range(args.steps)) for s in range(w4.NUM_STAGES)]
+                                for i in range(args.steps)) for s in range(n_ev // 2)]
 
     # ---------------- end to end through the public API, host buffers
     h_host = hidden.cpu().pin_memory()
@@ -419,14 +449,29 @@ def main():
                     parallelism=f"dp{world}" if world > 1 else "single",
                     l2=("inputs larger than L2: %.2f GB of packed experts streamed per step"
                         % ((g1["bytes"] + g2["bytes"]) / 1e9))),
-        stage_ms={n: round(x, 5) for n, x in zip(w4.STAGE_NAMES, stage_ms)},
+        stage_ms={n: round(x, 5) for n, x in
+                  zip(w4.STAGE_NAMES + (w4.SHARED_STAGE_NAMES if shared else []), stage_ms)},
         roofline=roof,
         e2e=dict(value=e2e_value, unit="tokens/s",
                  h2d_bytes_per_step=cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
                  d2h_bytes_per_step=cfg.T * cfg.H * 2),
-        gpu_launches=KERNELS_PER_STEP * args.steps,
+        gpu_launches=(KERNELS_PER_STEP + (SHARED_KERNELS_PER_STEP if shared else 0)) * args.steps,
         clocks=clk.summary(),
     )
+    if shared:   # the shared expert's slower GEMM against the same peak
+        s1, s2 = shared_work(cfg)
+        # stages 6..9: shared input quantisation, gate/up GEMM, requantisation, down GEMM
+        si = 1 if stage_ms[7] >= stage_ms[9] else 3
+        sw_, st_ = (s1, stage_ms[7]) if si == 1 else (s2, stage_ms[9])
+        sname = "shared_gemm_gate_up" if si == 1 else "shared_gemm_down"
+        if prefill:
+            a_ = sw_["flops"] / (st_ / 1e3) / 1e12
+            line["shared_roofline"] = dict(bound="tensor", achieved=a_, peak=roof["peak"],
+                                           unit="TFLOP/s", frac=a_ / roof["peak"], kernel=sname)
+        else:
+            a_ = sw_["bytes"] / (st_ / 1e3) / 1e9
+            line["shared_roofline"] = dict(bound="hbm", achieved=a_, peak=roof["peak"],
+                                           unit="GB/s", frac=a_ / roof["peak"], kernel=sname)
     if rank == 0 and world == 1 and args.cpu_tokens > 0:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, args.variant)
     if dist:

@@ -363,6 +363,92 @@ W4A8_API w4a8_status w4a8_moe_forward_channel_int8(
     int32_t E, int32_t k, void* out_bf16, void* workspace, size_t workspace_bytes,
     const w4a8_moe_aux* aux, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * The FP8-block shared expert.
+ *
+ * GLM-5.3-W4A8 model card, intro and "quantisation method" (item on the
+ * non-expert layers): only the routed experts are INT4; the shared expert
+ * keeps the official FP8 format, E4M3 weights with one float32 scale per
+ * 128 x 128 block.  Readings where the pages are silent: the block scale is
+ * absmax / 448 (float32 division) for weights quantised here; the expert's
+ * activations are quantised at run time per token and 128-wide channel group
+ * (scale = absmax / 448); the intermediate h is requantised the same way;
+ * the layer adds the shared expert's output to the routed sum before the
+ * bf16 rounding of the combine.
+ * ------------------------------------------------------------------------- */
+
+/*
+ * w4a8_quant_fp8_block - bf16 w [R, K] -> E4M3 codes [R, K] (uint8) and
+ * float32 scales [R / 128, K / 128]: per 128 x 128 block, scale =
+ * float32(absmax / 448), code = E4M3 round-to-nearest-even, saturating, of
+ * float32(w / scale); an all-zero block gets scale 0 and codes 0.
+ * R and K multiples of 128 (else W4A8_ERR_UNSUPPORTED_SHAPE), R / 128 <= 65535.
+ */
+W4A8_API w4a8_status w4a8_quant_fp8_block(const void* w_bf16, int64_t R, int64_t K,
+                                          uint8_t* codes, float* scales, void* stream);
+
+/*
+ * w4a8_quant_act_fp8_group - bf16 x [T, H] -> E4M3 codes [T, H] and float32
+ * scales [T, H / 128]: per token and 128-wide group, scale =
+ * float32(absmax / 448), code = E4M3(float32(x / scale)); scale 0 -> codes 0.
+ * H a multiple of 128.
+ */
+W4A8_API w4a8_status w4a8_quant_act_fp8_group(const void* x_bf16, int64_t T, int64_t H,
+                                              uint8_t* codes, float* scales, void* stream);
+
+/* Optional outputs of the shared expert (each NULL = not wanted). */
+typedef struct w4a8_shared_aux {
+    uint8_t* act_codes;   /* [T, H] E4M3 codes of the input */
+    float* act_scales;    /* [T, H / 128] */
+    float* h;             /* [T, I] float32 SwiGLU output before requantisation */
+    uint8_t* h_codes;     /* [T, I] */
+    float* h_scales;      /* [T, I / 128] */
+    /* If non-NULL: 8 cudaEvent_t handles (host memory array), recorded on
+     * `stream` before / after: input quantisation (0/1), gate/up GEMM (2/3),
+     * requantisation of h (4/5), down GEMM (6/7). */
+    void* const* stage_events;
+} w4a8_shared_aux;
+
+W4A8_API size_t w4a8_shared_expert_workspace_size(int64_t T, int64_t H, int64_t I);
+
+/*
+ * w4a8_shared_expert_forward - the FP8-block SwiGLU expert on T tokens:
+ *   a = w4a8_quant_act_fp8_group(hidden);
+ *   G[t, n] = sum_g a_s[t, g] * s13[n / 128, g] * sum_{kappa in g} a[t, kappa] * w13[n, kappa]
+ *             for n < 2I (tensor cores: E4M3 x E4M3 products exact, float32
+ *             accumulation, one float32 promotion per 128-wide group);
+ *   h = silu(G[:, :I]) * G[:, I:];  h requantised per token and 128-group;
+ *   y[t, n] = sum_g h_s[t, g] * s2[n / 128, g] * sum h[t, kappa] * w2[n, kappa].
+ * hidden bf16 [T, H]; w13_codes [2I, H] and w2_codes [H, I] E4M3 with
+ * float32 block scales [2I / 128, H / 128] and [H / 128, I / 128] (as
+ * w4a8_quant_fp8_block writes them); y float32 [T, H].  H and I multiples of
+ * 128, at most 64 groups each.
+ */
+W4A8_API w4a8_status w4a8_shared_expert_forward(
+    const void* hidden_bf16, const uint8_t* w13_codes, const float* w13_scales,
+    const uint8_t* w2_codes, const float* w2_scales, int64_t T, int64_t H, int64_t I,
+    float* y, void* workspace, size_t workspace_bytes, const w4a8_shared_aux* aux, void* stream);
+
+W4A8_API size_t w4a8_moe_shared_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E,
+                                               int32_t k, int64_t I_shared);
+
+/*
+ * w4a8_moe_forward_shared - w4a8_moe_forward plus the FP8-block shared
+ * expert (ws13 [2 I_shared, H], ws2 [H, I_shared], as for
+ * w4a8_shared_expert_forward), in the same call:
+ *   out[t] = bf16_rn(sum_j topk_w[t, j] * Y[row_of[t, j]] + y_shared[t]).
+ * The routed arguments, aux and errors are those of w4a8_moe_forward;
+ * shared_aux those of w4a8_shared_expert_forward.  The workspace size is
+ * w4a8_moe_shared_workspace_size.
+ */
+W4A8_API w4a8_status w4a8_moe_forward_shared(
+    const void* hidden_bf16, const float* logits, const int32_t* w13_packed,
+    const void* w13_scales, const int32_t* w2_packed, const void* w2_scales,
+    const uint8_t* ws13_codes, const float* ws13_scales, const uint8_t* ws2_codes,
+    const float* ws2_scales, int64_t T, int64_t H, int64_t I, int64_t I_shared, int32_t E,
+    int32_t k, void* out_bf16, void* workspace, size_t workspace_bytes, const w4a8_moe_aux* aux,
+    const w4a8_shared_aux* shared_aux, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -18,12 +18,16 @@ __all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_ab
            "w4a8_status_string", "w4a8_pack_int4", "w4a8_quant_act_fp8_per_token",
            "w4a8_moe_route_workspace_size", "w4a8_moe_route_permute",
            "w4a8_moe_route_permute_noalloc", "w4a8_moe_workspace_size",
-           "w4a8_moe_forward", "w4a8_check_device_error", "W4A8MoELayer"]
+           "w4a8_moe_forward", "w4a8_check_device_error", "W4A8MoELayer",
+           "w4a8_quant_fp8_block", "w4a8_quant_act_fp8_group", "w4a8_shared_expert_forward",
+           "w4a8_moe_forward_shared", "SharedExpertFP8", "SHARED_STAGE_NAMES"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a8.so")
 NUM_STAGES = 6
 STAGE_NAMES = ["act_quant", "route_permute", "gemm_gate_up", "inter_quant", "gemm_down",
                "combine"]
+SHARED_STAGE_NAMES = ["shared_act_quant", "shared_gemm_gate_up", "shared_inter_quant",
+                      "shared_gemm_down"]
 
 _lib = None
 
@@ -43,6 +47,12 @@ class MoEAux(ctypes.Structure):
                 ("act_scales", ctypes.c_void_p), ("inter_h", ctypes.c_void_p),
                 ("inter_codes", ctypes.c_void_p), ("inter_scales", ctypes.c_void_p),
                 ("y_rows", ctypes.c_void_p), ("stage_events", ctypes.c_void_p)]
+
+
+class SharedAux(ctypes.Structure):
+    _fields_ = [("act_codes", ctypes.c_void_p), ("act_scales", ctypes.c_void_p),
+                ("h", ctypes.c_void_p), ("h_codes", ctypes.c_void_p),
+                ("h_scales", ctypes.c_void_p), ("stage_events", ctypes.c_void_p)]
 
 
 def _declare(L):
@@ -67,6 +77,14 @@ def _declare(L):
         "w4a8_prepare_experts_channel_b200": (i32, [vp, i64, i64, i64, vp, vp, vp]),
         "w4a8_moe_forward_channel_int8": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
                                                 i32, i32, vp, vp, sz, vp, vp]),
+        "w4a8_quant_fp8_block": (i32, [vp, i64, i64, vp, vp, vp]),
+        "w4a8_quant_act_fp8_group": (i32, [vp, i64, i64, vp, vp, vp]),
+        "w4a8_shared_expert_workspace_size": (sz, [i64, i64, i64]),
+        "w4a8_shared_expert_forward": (i32, [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp,
+                                             vp]),
+        "w4a8_moe_shared_workspace_size": (sz, [i64, i64, i64, i32, i32, i64]),
+        "w4a8_moe_forward_shared": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                          i64, i32, i32, vp, vp, sz, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -472,3 +490,159 @@ class W4A8ChannelInt8Layer:
         return w4a8_moe_forward_channel_int8(hidden, logits, *self.w13, *self.w2, self.k, out=out,
                                              workspace=self.workspace(hidden.shape[0]), aux=aux,
                                              stage_events=stage_events)
+
+
+# ---------------------------------------------------------------- FP8-block shared expert
+
+def w4a8_quant_fp8_block(w: torch.Tensor):
+    """bf16 ``w`` [R, K] -> (E4M3 codes uint8 [R, K], float32 scales [R/128, K/128])."""
+    _need(w, "w", torch.bfloat16, 2)
+    R, K = w.shape
+    codes = torch.empty(R, K, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(R // 128, K // 128, dtype=torch.float32, device=w.device)
+    _check("w4a8_quant_fp8_block",
+           lib().w4a8_quant_fp8_block(_p(w), R, K, _p(codes), _p(scales), _stream(w.device)))
+    return codes, scales
+
+
+def w4a8_quant_act_fp8_group(x: torch.Tensor):
+    """bf16 ``x`` [T, H] -> (E4M3 codes uint8 [T, H], float32 scales [T, H/128])."""
+    _need(x, "x", torch.bfloat16, 2)
+    T, H = x.shape
+    codes = torch.empty(T, H, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(T, H // 128, dtype=torch.float32, device=x.device)
+    _check("w4a8_quant_act_fp8_group",
+           lib().w4a8_quant_act_fp8_group(_p(x), T, H, _p(codes), _p(scales), _stream(x.device)))
+    return codes, scales
+
+
+_SHARED_AUX_FIELDS = ["act_codes", "act_scales", "h", "h_codes", "h_scales"]
+
+
+def _shared_aux_struct(aux, stage_events):
+    if not aux and not stage_events:
+        return None, []
+    st, keep = SharedAux(), []
+    for name, t in (aux or {}).items():
+        if name not in _SHARED_AUX_FIELDS:
+            raise KeyError(f"unknown shared aux buffer {name!r}")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"shared aux[{name!r}] must be a contiguous CUDA tensor")
+        setattr(st, name, t.data_ptr())
+    if stage_events:
+        if len(stage_events) != 8:
+            raise ValueError("need 8 events")
+        arr = (ctypes.c_void_p * 8)(*[e.cuda_event for e in stage_events])
+        keep.append(arr)
+        st.stage_events = ctypes.cast(arr, ctypes.c_void_p)
+    return st, keep
+
+
+def _check_shared_weights(w13_codes, w13_scales, w2_codes, w2_scales, H):
+    _need(w13_codes, "w13_codes", torch.uint8, 2)
+    _need(w13_scales, "w13_scales", torch.float32, 2)
+    _need(w2_codes, "w2_codes", torch.uint8, 2)
+    _need(w2_scales, "w2_scales", torch.float32, 2)
+    I = w2_codes.shape[1]
+    if w13_codes.shape != (2 * I, H) or w2_codes.shape != (H, I) or \
+            w13_scales.shape != (2 * I // 128, H // 128) or w2_scales.shape != (H // 128, I // 128):
+        raise ValueError("shared expert: w13 [2I, H], w2 [H, I], scales [2I/128, H/128] and "
+                         "[H/128, I/128]")
+    return I
+
+
+def w4a8_shared_expert_forward(hidden, w13_codes, w13_scales, w2_codes, w2_scales, y=None,
+                               workspace=None, aux=None, stage_events=None) -> torch.Tensor:
+    """The FP8-block shared expert alone: float32 [T, H] (see include/w4a8.h)."""
+    _need(hidden, "hidden", torch.bfloat16, 2)
+    T, H = hidden.shape
+    I = _check_shared_weights(w13_codes, w13_scales, w2_codes, w2_scales, H)
+    dev = hidden.device
+    if y is None:
+        y = torch.empty(T, H, dtype=torch.float32, device=dev)
+    need = int(lib().w4a8_shared_expert_workspace_size(T, H, I))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st, keep = _shared_aux_struct(aux, stage_events)
+    _check("w4a8_shared_expert_forward",
+           lib().w4a8_shared_expert_forward(
+               _p(hidden), _p(w13_codes), _p(w13_scales), _p(w2_codes), _p(w2_scales), T, H, I,
+               _p(y), _p(workspace), workspace.numel(), None if st is None else ctypes.byref(st),
+               _stream(dev)))
+    return y
+
+
+def w4a8_moe_forward_shared(hidden, logits, w13_packed, w13_scales, w2_packed, w2_scales,
+                            shared, k: int, out=None, workspace=None, aux=None, stage_events=None,
+                            shared_aux=None, shared_stage_events=None) -> torch.Tensor:
+    """The W4A8 layer plus the FP8-block shared expert ``shared`` = (w13_codes,
+    w13_scales, w2_codes, w2_scales): bf16 [T, H]."""
+    _need(hidden, "hidden", torch.bfloat16, 2)
+    _need(logits, "logits", torch.float32, 2)
+    T, H = hidden.shape
+    E = logits.shape[1]
+    I = w2_packed.shape[2] * 8
+    Is = _check_shared_weights(*shared, H)
+    if logits.shape[0] != T or w13_packed.shape != (E, 2 * I, H // 8) or \
+            w2_packed.shape != (E, H, I // 8) or w13_scales.shape != (E, H // 128, 2 * I) or \
+            w2_scales.shape != (E, I // 128, H):
+        raise ValueError("inconsistent routed-expert shapes")
+    dev = hidden.device
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    need = int(lib().w4a8_moe_shared_workspace_size(T, H, I, E, k, Is))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    ast, keep = _aux_struct(aux, stage_events)
+    sst, keep2 = _shared_aux_struct(shared_aux, shared_stage_events)
+    _check("w4a8_moe_forward_shared",
+           lib().w4a8_moe_forward_shared(
+               _p(hidden), _p(logits), _p(w13_packed), _p(w13_scales), _p(w2_packed),
+               _p(w2_scales), *[_p(t) for t in shared], T, H, I, Is, E, k, _p(out),
+               _p(workspace), workspace.numel(), None if ast is None else ctypes.byref(ast),
+               None if sst is None else ctypes.byref(sst), _stream(dev)))
+    return out
+
+
+class SharedExpertFP8:
+    """The shared expert's E4M3 weights and 128 x 128 block scales, resident."""
+
+    def __init__(self, w13_codes, w13_scales, w2_codes, w2_scales):
+        self.weights = (w13_codes, w13_scales, w2_codes, w2_scales)
+        self.H, self.I = w2_codes.shape
+
+    @classmethod
+    def from_bf16(cls, w13: torch.Tensor, w2: torch.Tensor) -> "SharedExpertFP8":
+        return cls(*w4a8_quant_fp8_block(w13), *w4a8_quant_fp8_block(w2))
+
+    def __call__(self, hidden, **kw) -> torch.Tensor:
+        return w4a8_shared_expert_forward(hidden, *self.weights, **kw)
+
+
+class W4A8MoELayerShared(W4A8MoELayer):
+    """``W4A8MoELayer`` plus an FP8-block shared expert, in one forward call."""
+
+    def __init__(self, w13_packed, w13_scales, w2_packed, w2_scales, k: int,
+                 shared: SharedExpertFP8):
+        super().__init__(w13_packed, w13_scales, w2_packed, w2_scales, k)
+        self.shared = shared
+
+    @classmethod
+    def from_bf16_with_shared(cls, w13, w2, k: int, ws13, ws2,
+                              mse_clip: bool = False) -> "W4A8MoELayerShared":
+        base = W4A8MoELayer.from_bf16(w13, w2, k, mse_clip=mse_clip)
+        return cls(base.w13_packed, base.w13_scales, base.w2_packed, base.w2_scales, k,
+                   SharedExpertFP8.from_bf16(ws13, ws2))
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = max(int(lib().w4a8_moe_shared_workspace_size(T, self.H, self.I, self.E, self.k,
+                                                             self.shared.I)), 1)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.w13_packed.device)
+        return self._ws
+
+    def __call__(self, hidden, logits, out=None, **kw) -> torch.Tensor:
+        return w4a8_moe_forward_shared(hidden, logits, self.w13_packed, self.w13_scales,
+                                       self.w2_packed, self.w2_scales, self.shared.weights,
+                                       self.k, out=out, workspace=self.workspace(hidden.shape[0]),
+                                       **kw)

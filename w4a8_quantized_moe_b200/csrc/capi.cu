@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -154,6 +155,30 @@ ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int
   b.act_rowsum = c.take<int32_t>(static_cast<size_t>(T));
   b.inter_rowsum = c.take<int32_t>(A);
   b.y = c.take<float>(A * static_cast<size_t>(H));
+  return b;
+}
+
+// The FP8-block shared expert's scratch.
+struct SharedBufs {
+  uint8_t* act_codes;   // [T, H] E4M3 codes, per-token-group scaled
+  float* act_scales;    // [T, H / 128]
+  float* h;             // [T, I] float32 SwiGLU output
+  uint8_t* h_codes;     // [T, I]
+  float* h_scales;      // [T, I / 128]
+  int32_t* tables;      // [4]: expert offsets {0, T}, tile prefix {0, tiles}
+  float* y;             // [T, H] float32 output (the combined layer only)
+};
+
+SharedBufs carve_shared(Carver& c, int64_t T, int64_t H, int64_t I, bool with_y) {
+  SharedBufs b;
+  const size_t t = static_cast<size_t>(T);
+  b.act_codes = c.take<uint8_t>(t * static_cast<size_t>(H));
+  b.act_scales = c.take<float>(t * static_cast<size_t>(H / kGroup));
+  b.h = c.take<float>(t * static_cast<size_t>(I));
+  b.h_codes = c.take<uint8_t>(t * static_cast<size_t>(I));
+  b.h_scales = c.take<float>(t * static_cast<size_t>(I / kGroup));
+  b.tables = c.take<int32_t>(4);
+  b.y = with_y ? c.take<float>(t * static_cast<size_t>(H)) : nullptr;
   return b;
 }
 
@@ -403,6 +428,124 @@ size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32
 }  // extern "C"
 
 namespace {
+w4a8_status check_shared_shape(int64_t T, int64_t H, int64_t I) {
+  if (T < 0) return fail(W4A8_ERR_INVALID_ARG, "T = %lld < 0", static_cast<long long>(T));
+  if (H <= 0 || I <= 0 || H % kGroup || I % kGroup)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE,
+                "shared expert: H = %lld and I = %lld must be positive multiples of 128",
+                static_cast<long long>(H), static_cast<long long>(I));
+  if (H / kGroup > kMaxGroups || I / kGroup > kMaxGroups)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "shared expert: at most %d groups of 128 per row",
+                kMaxGroups);
+  if (T > INT32_MAX) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "T exceeds 2^31 - 1");
+  return W4A8_OK;
+}
+
+// The FP8-block shared expert for T rows of hidden: group-quantise x, gate/up
+// GEMM + SwiGLU, group-requantise h, down GEMM into y [T, H] float32.
+// Stage events (aux->stage_events, 8 handles): 0/1 input quantisation, 2/3
+// gate/up GEMM, 4/5 requantisation of h, 6/7 down GEMM.
+w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_codes,
+                                const float* w13_scales, const uint8_t* w2_codes,
+                                const float* w2_scales, int64_t T, int64_t H, int64_t I,
+                                float* y, SharedBufs b, const w4a8_shared_aux* aux,
+                                const DeviceInfo& di, cudaStream_t s) {
+  void* const* ev = nullptr;
+  if (aux) {
+    auto pick = [](auto* user, auto* ws) { return user ? user : ws; };
+    b.act_codes = pick(aux->act_codes, b.act_codes);
+    b.act_scales = pick(aux->act_scales, b.act_scales);
+    b.h = pick(aux->h, b.h);
+    b.h_codes = pick(aux->h_codes, b.h_codes);
+    b.h_scales = pick(aux->h_scales, b.h_scales);
+    for (const void* p : {static_cast<const void*>(b.act_codes), static_cast<const void*>(b.act_scales),
+                          static_cast<const void*>(b.h), static_cast<const void*>(b.h_codes),
+                          static_cast<const void*>(b.h_scales)})
+      if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "aux buffers must be 16-byte aligned");
+    ev = aux->stage_events;
+  }
+  // E4M3 weights [rows, K] bytes, 128-byte swizzle: boxes of 64 rows (the
+  // gate and up halves of a gate/up tile) or 128 rows (down); activation codes
+  // [T, K] in 16-row boxes, as for the routed experts.
+  CUtensorMap tw1, ta1, tw2, ta2;
+  if (w4a8_status st = encode_u8_2d(&tw1, w13_codes, static_cast<uint64_t>(H),
+                                    static_cast<uint64_t>(2 * I), 128, 64,
+                                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ta1, b.act_codes, static_cast<uint64_t>(H),
+                                    static_cast<uint64_t>(T), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&tw2, w2_codes, static_cast<uint64_t>(I),
+                                    static_cast<uint64_t>(H), 128, 128,
+                                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ta2, b.h_codes, static_cast<uint64_t>(I),
+                                    static_cast<uint64_t>(T), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  auto record = [&](int i) -> cudaError_t {
+    return ev && ev[i] ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+  cudaError_t err = cudaSuccess;
+#define W4A8_STEP(call, what)                              \
+  do {                                                     \
+    err = (call);                                          \
+    if (err != cudaSuccess) return cuda_fail(err, what);   \
+  } while (0)
+  const int tile_n = grouped_gemm_tile_n(false);
+  W4A8_STEP(launch_dense_tables(b.tables, b.tables + 2, T, tile_n, s), "dense tables launch");
+  W4A8_STEP(record(0), "cudaEventRecord");
+  W4A8_STEP(launch_act_quant_group(hidden_bf16, nullptr, T, H, b.act_codes, b.act_scales, di.sms, s),
+            "shared input quantisation launch");
+  W4A8_STEP(record(1), "cudaEventRecord");
+  const int64_t tiles_n = (T + tile_n - 1) / tile_n;
+  GemmArgs g1{};
+  g1.K = static_cast<int>(H);
+  g1.n_rows = static_cast<int>(2 * I);
+  g1.half_rows = static_cast<int>(I);
+  g1.E = 1;
+  g1.expert_offsets = b.tables;
+  g1.tile_prefix = b.tables + 2;
+  g1.act_gsum = b.act_scales;
+  g1.wscale = w13_scales;
+  g1.out = b.h;
+  g1.out_ld = I;
+  g1.act_rows = T;
+  g1.timeout_ns = wait_timeout_ns();
+  g1.nb_fastest = 1;
+  const int ctas1 = static_cast<int>(std::min<int64_t>(tiles_n * (I / 64), di.sms));
+  W4A8_STEP(record(2), "cudaEventRecord");
+  W4A8_STEP(launch_fp8_block_gemm(true, tw1, ta1, g1, ctas1, s), "shared gate/up GEMM launch");
+  W4A8_STEP(record(3), "cudaEventRecord");
+  W4A8_STEP(record(4), "cudaEventRecord");
+  W4A8_STEP(launch_act_quant_group(nullptr, b.h, T, I, b.h_codes, b.h_scales, di.sms, s),
+            "shared intermediate quantisation launch");
+  W4A8_STEP(record(5), "cudaEventRecord");
+  GemmArgs g2 = g1;
+  g2.K = static_cast<int>(I);
+  g2.n_rows = static_cast<int>(H);
+  g2.half_rows = 0;
+  g2.act_gsum = b.h_scales;
+  g2.wscale = w2_scales;
+  g2.out = y;
+  g2.out_ld = H;
+  const int ctas2 = static_cast<int>(std::min<int64_t>(tiles_n * (H / kGroup), di.sms));
+  W4A8_STEP(record(6), "cudaEventRecord");
+  W4A8_STEP(launch_fp8_block_gemm(false, tw2, ta2, g2, ctas2, s), "shared down GEMM launch");
+  W4A8_STEP(record(7), "cudaEventRecord");
+#undef W4A8_STEP
+  return W4A8_OK;
+}
+
+// The layer's optional FP8-block shared expert.
+struct SharedExpert {
+  const uint8_t* w13_codes;
+  const float* w13_scales;
+  const uint8_t* w2_codes;
+  const float* w2_scales;
+  int64_t I;
+  const w4a8_shared_aux* aux;
+};
+
 // The layer, for both variants: i8 == nullptr runs the W4A8 (FP8 E4M3
 // activations, group-128 scales) path; otherwise the per-channel INT4 x
 // per-token INT8 path with i8 = {w13 nibble row sums, w2 nibble row sums}.
@@ -416,8 +559,16 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
                              const int32_t* w2_packed, const void* w2_scales, int64_t T,
                              int64_t H, int64_t I, int32_t E, int32_t k, void* out_bf16,
                              void* workspace, size_t workspace_bytes, const w4a8_moe_aux* aux,
-                             void* stream, const Int8Weights* i8) {
+                             void* stream, const Int8Weights* i8,
+                             const SharedExpert* sh = nullptr) {
   if (w4a8_status st = check_route_args(logits, T, E, k)) return st;
+  if (sh) {
+    if (w4a8_status st = check_shared_shape(T, H, sh->I)) return st;
+    const void* sp[] = {sh->w13_codes, sh->w13_scales, sh->w2_codes, sh->w2_scales};
+    for (const void* p : sp)
+      if (T > 0 && (!p || !aligned16(p)))
+        return fail(W4A8_ERR_INVALID_ARG, "shared expert pointers must be non-NULL and 16-byte aligned");
+  }
   if (H <= 0 || I <= 0 || H % kGroup || I % kGroup)
     return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld and I = %lld must be positive multiples of 128",
                 static_cast<long long>(H), static_cast<long long>(I));
@@ -433,7 +584,8 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
     if (!p) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
     if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   }
-  const size_t need = w4a8_moe_workspace_size(T, H, I, E, k);
+  const size_t need = sh ? w4a8_moe_shared_workspace_size(T, H, I, E, k, sh->I)
+                         : w4a8_moe_workspace_size(T, H, I, E, k);
   if (workspace_bytes < need)
     return fail(W4A8_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu", workspace_bytes, need);
   DeviceInfo di;
@@ -442,6 +594,8 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
 
   Carver c(workspace);
   ForwardBufs b = carve_forward(c, T, H, I, E, k);
+  SharedBufs sb{};
+  if (sh) sb = carve_shared(c, T, H, sh->I, true);
   void* const* ev = nullptr;
   if (aux) {
     auto pick = [](auto* user, auto* ws) { return user ? user : ws; };
@@ -523,6 +677,14 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
     if (err != cudaSuccess) return cuda_fail(err, what); \
   } while (0)
 
+  // the shared expert first: it reads only the hidden states, and the combine
+  // adds its output
+  if (sh) {
+    if (w4a8_status st = shared_forward_impl(hidden_bf16, sh->w13_codes, sh->w13_scales,
+                                             sh->w2_codes, sh->w2_scales, T, H, sh->I, sb.y, sb,
+                                             sh->aux, di, s))
+      return st;
+  }
   // routing first: the activation quantiser writes each token's codes to its
   // segment rows as well, so both GEMMs read contiguous activation tiles
   W4A8_STEP(record(2), "cudaEventRecord");
@@ -596,7 +758,8 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   W4A8_STEP(record(9), "cudaEventRecord");
 
   W4A8_STEP(record(10), "cudaEventRecord");
-  W4A8_STEP(launch_combine(b.y, b.row_of, b.topk_w, T, H, k, out_bf16, di.sms, s),
+  W4A8_STEP(launch_combine(b.y, b.row_of, b.topk_w, T, H, k, out_bf16, di.sms, s,
+                           sh ? sb.y : nullptr),
             "combine launch");
   W4A8_STEP(record(11), "cudaEventRecord");
 #undef W4A8_STEP
@@ -669,6 +832,96 @@ w4a8_status w4a8_prepare_experts_channel_b200(const int32_t* packed, int64_t E, 
   cudaError_t err = launch_nibble_row_sum(packed, R, K / 8, nibble_sums, di.sms, s);
   if (err == cudaSuccess) err = launch_repack_int4_b200(packed, nwords, packed_out, di.sms, s);
   return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "prepare_experts_channel launch");
+}
+
+w4a8_status w4a8_quant_fp8_block(const void* w_bf16, int64_t R, int64_t K, uint8_t* codes,
+                                 float* scales, void* stream) {
+  if (R < 0 || K < 0) return fail(W4A8_ERR_INVALID_ARG, "R = %lld, K = %lld",
+                                  static_cast<long long>(R), static_cast<long long>(K));
+  if (R % kGroup || K % kGroup)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "R = %lld and K = %lld must be multiples of 128",
+                static_cast<long long>(R), static_cast<long long>(K));
+  if (R == 0 || K == 0) return W4A8_OK;
+  if (R / kGroup > 65535) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "R / 128 exceeds 65535");
+  if (!w_bf16 || !codes || !scales) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(scales))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_quant_fp8_block(w_bf16, R, K, codes, scales,
+                                           static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "quant_fp8_block launch");
+}
+
+w4a8_status w4a8_quant_act_fp8_group(const void* x_bf16, int64_t T, int64_t H, uint8_t* codes,
+                                     float* scales, void* stream) {
+  if (T < 0 || H <= 0) return fail(W4A8_ERR_INVALID_ARG, "T = %lld, H = %lld",
+                                   static_cast<long long>(T), static_cast<long long>(H));
+  if (H % kGroup) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld is not a multiple of 128",
+                              static_cast<long long>(H));
+  if (T == 0) return W4A8_OK;
+  if (!x_bf16 || !codes || !scales) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_act_quant_group(x_bf16, nullptr, T, H, codes, scales, di.sms,
+                                           static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "quant_act_fp8_group launch");
+}
+
+size_t w4a8_shared_expert_workspace_size(int64_t T, int64_t H, int64_t I) {
+  if (T < 0 || H <= 0 || I <= 0) return 0;
+  Carver c(nullptr);
+  carve_shared(c, T, H, I, false);
+  return c.off + 256;
+}
+
+w4a8_status w4a8_shared_expert_forward(const void* hidden_bf16, const uint8_t* w13_codes,
+                                       const float* w13_scales, const uint8_t* w2_codes,
+                                       const float* w2_scales, int64_t T, int64_t H, int64_t I,
+                                       float* y, void* workspace, size_t workspace_bytes,
+                                       const w4a8_shared_aux* aux, void* stream) {
+  if (w4a8_status st = check_shared_shape(T, H, I)) return st;
+  if (T == 0) return W4A8_OK;
+  const void* ptrs[] = {hidden_bf16, w13_codes, w13_scales, w2_codes, w2_scales, y, workspace};
+  for (const void* p : ptrs) {
+    if (!p) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  const size_t need = w4a8_shared_expert_workspace_size(T, H, I);
+  if (workspace_bytes < need)
+    return fail(W4A8_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu", workspace_bytes, need);
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  Carver c(workspace);
+  const SharedBufs b = carve_shared(c, T, H, I, false);
+  return shared_forward_impl(hidden_bf16, w13_codes, w13_scales, w2_codes, w2_scales, T, H, I, y,
+                             b, aux, di, static_cast<cudaStream_t>(stream));
+}
+
+size_t w4a8_moe_shared_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k,
+                                      int64_t I_shared) {
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || I_shared <= 0) return 0;
+  Carver c(nullptr);
+  carve_forward(c, T, H, I, E, k);
+  carve_shared(c, T, H, I_shared, true);
+  return c.off + 256;
+}
+
+w4a8_status w4a8_moe_forward_shared(const void* hidden_bf16, const float* logits,
+                                    const int32_t* w13_packed, const void* w13_scales,
+                                    const int32_t* w2_packed, const void* w2_scales,
+                                    const uint8_t* ws13_codes, const float* ws13_scales,
+                                    const uint8_t* ws2_codes, const float* ws2_scales,
+                                    int64_t T, int64_t H, int64_t I, int64_t I_shared, int32_t E,
+                                    int32_t k, void* out_bf16, void* workspace,
+                                    size_t workspace_bytes, const w4a8_moe_aux* aux,
+                                    const w4a8_shared_aux* shared_aux, void* stream) {
+  const SharedExpert sh{ws13_codes, ws13_scales, ws2_codes, ws2_scales, I_shared, shared_aux};
+  return moe_forward_impl(hidden_bf16, logits, w13_packed, w13_scales, w2_packed, w2_scales, T, H,
+                          I, E, k, out_bf16, workspace, workspace_bytes, aux, stream, nullptr,
+                          &sh);
 }
 
 }  // extern "C"

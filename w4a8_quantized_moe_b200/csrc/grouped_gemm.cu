@@ -139,9 +139,11 @@ struct Shape {
   static constexpr __host__ __device__ int tile_sc_bytes(int G) { return 256 * G; }
   // tile_prefix and expert_offsets, [E + 1] int32 each
   static constexpr __host__ __device__ int table_bytes(int E) { return (8 * (E + 1) + 15) & ~15; }
-  static constexpr int smem_bytes(bool gate_up, int G, int E) {
-    return 1024 + WStages * kWStageBytes + BStages * kBStageBytes +
-           EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G)) + kTileScBufs * tile_sc_bytes(G) +
+  // f8w: E4M3 weights (128 B per row and group, no tile-scale buffers)
+  static constexpr int smem_bytes(bool gate_up, int G, int E, bool f8w = false) {
+    return 1024 + WStages * (f8w ? 2 * kWStageBytes : kWStageBytes) + BStages * kBStageBytes +
+           EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G)) +
+           (f8w ? 0 : kTileScBufs * tile_sc_bytes(G)) +
            table_bytes(E) + kNumBars * 8 + 16;
   }
 };
@@ -157,6 +159,8 @@ using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 3, 3, 1, 4, 16, 2, 1, 1>;
 using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 3, 2, 1, 2, 16, 2, 1, 1>;
 using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
 using PrefillTileCorr = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 2>;
+// E4M3-weight (FP8 block) shape: A from shared memory, no converter warps
+using F8Block = Shape<kTileNPrefill, 4, 4, 1, 3, 0, 4, 16, 2, 1, 0>;
 // INT8 per-channel shapes: one accumulator per tile, single MMA issuer
 using I8Decode  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 1, 1, 0>;
 using I8Decode2 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;  // 4 tiles x 2 chains
@@ -238,7 +242,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
   }
 }
 
-template <class S, bool kGateUp, bool kI8>
+template <class S, bool kGateUp, bool kI8, bool kF8W>
 __global__ void __launch_bounds__(S::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
                         const __grid_constant__ CUtensorMap tmap_act,
@@ -253,14 +257,17 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sW = smem;
-  uint8_t* sB = sW + kWStages * kWStageBytes;
+  // W stage: packed INT4 [128 rows x 64 B], or E4M3 weights [128 rows x 128 B]
+  constexpr int kWBytes = kF8W ? 2 * kWStageBytes : kWStageBytes;
+  constexpr int kTileScTotal = kF8W ? 0 : S::kTileScBufs;
+  uint8_t* sB = sW + kWStages * kWBytes;
   const int G = a.K / kGroup;
   // per epilogue set: [sU (gate/up only)][sS]
   constexpr int kUpPerSet = kGateUp ? kUpBytes : 0;
   const int set_bytes = kUpPerSet + S::sum_bytes(G);
   uint8_t* sSet = sB + kBStages * kBStageBytes;
   uint8_t* sT = sSet + S::kEpiSets * set_bytes;
-  int* sTP = reinterpret_cast<int*>(sT + S::kTileScBufs * S::tile_sc_bytes(G));
+  int* sTP = reinterpret_cast<int*>(sT + kTileScTotal * S::tile_sc_bytes(G));
   int* sEO = sTP + (a.E + 1);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sTP) + S::table_bytes(a.E));
   uint64_t* wfull = bars;                 // [kWStages] packed weights landed
@@ -279,7 +286,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   // FP8: one commit per group releases the A slot, B stage and accumulator when
   // the three rings have one size.  INT8: one accumulator per tile, so only
   // the A and B rings can share a barrier.
-  constexpr bool kUniAll = S::kUnified && !kI8;
+  constexpr bool kUniAll = S::kUnified && !kI8 && !kF8W;
   constexpr bool kUniAB = kI8 ? (kASlots == kBStages) : kUniAll;
   if constexpr (kUniAB) bempty = aempty;
   if constexpr (kUniAll) dfull = aempty;
@@ -298,7 +305,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kWStages; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 4);
+      mbar_init(&wempty[s], kF8W ? 1 : 4);  // E4M3 weights: released by the MMA commit
     }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&bfull[s], 1);
@@ -374,7 +381,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
         const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
         const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
-        if constexpr (!kI8) {  // the tile's weight scales: box [G groups x 128 (or 2 x 64) rows] of bf16
+        if constexpr (!kI8 && !kF8W) {  // the tile's weight scales: box [G groups x 128 (or 2 x 64) rows] of bf16
           const int tb = nt % S::kTileScBufs;
           const uint32_t tph = (nt / S::kTileScBufs) & 1;
           if (!mbar_wait(&tempty[tb], tph ^ 1, abort_flag, tmo)) break;
@@ -392,9 +399,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           const int s = it % kWStages;
           const uint32_t ph = (it / kWStages) & 1;
           if (!mbar_wait(&wempty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
-          const uint32_t dW = smem_u32(sW + s * kWStageBytes);
-          mbar_arrive_expect_tx(&wfull[s], kWStageBytes);
-          if (kGateUp) {
+          const uint32_t dW = smem_u32(sW + s * kWBytes);
+          mbar_arrive_expect_tx(&wfull[s], kWBytes);
+          if constexpr (kF8W) {  // E4M3 rows: 128 B per group, boxes of 64 (gate/up) or 128 rows
+            tma_load_2d(dW, &tmap_w, &wfull[s], g * kGroup, wy0);
+            if (kGateUp) tma_load_2d(dW + kWBytes / 2, &tmap_w, &wfull[s], g * kGroup, wy1);
+          } else if (kGateUp) {
             tma_load_2d(dW, &tmap_w, &wfull[s], g * 64, wy0);
             tma_load_2d(dW + kWStageBytes / 2, &tmap_w, &wfull[s], g * 64, wy1);
           } else {
@@ -406,7 +416,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       // The latest fill of every stage must have landed before the CTA exits.
       for (int i = (it > kWStages ? it - kWStages : 0); i < it; ++i)
         mbar_wait_drain(&wfull[i % kWStages], (i / kWStages) & 1, tmo);
-      if (!kI8)
+      if (!kI8 && !kF8W)
         for (int i = (nt > S::kTileScBufs ? nt - S::kTileScBufs : 0); i < nt; ++i)
           mbar_wait_drain(&tfull[i % S::kTileScBufs], (i / S::kTileScBufs) & 1, tmo);
     }
@@ -490,6 +500,46 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           tc_commit(&aempty[as]);
           if constexpr (!kUniAB) tc_commit(&bempty[sb]);
           if (g + kChains >= G) tc_commit(&dfull[dcur]);  // this chain's last group of the tile
+        }
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, tmo);
+      }
+    } else if constexpr (kF8W) {
+      // E4M3 weights: A straight from the W stage in shared memory (K-major,
+      // 128-byte swizzle, the layout of the activation stages); the commit
+      // releases the W stage, the activation stage and the accumulator
+      if (lane == 0) {
+        int cur = -1;
+        uint32_t idesc = 0;
+        for (int it = mw; it < n_groups; it += S::kMmaWarps) {
+          const int tl = it / G;
+          if (tl != cur) {
+            cur = tl;
+            const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest,
+                                               blockIdx.x + tl * gridDim.x);
+            idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
+          }
+          const int ws = it % kWStages;
+          const uint32_t phw = (it / kWStages) & 1;
+          const int sb = it % kBStages;
+          const uint32_t phb = (it / kBStages) & 1;
+          const int d = it % kDBufs;
+          const uint32_t phd = (it / kDBufs) & 1;
+          if (!mbar_wait(&dempty[d], phd ^ 1, abort_flag, tmo) ||
+              !mbar_wait(&bfull[sb], phb, abort_flag, tmo) ||
+              !mbar_wait(&wfull[ws], phw, abort_flag, tmo))
+            break;
+          tc_fence_after();
+          const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sW + ws * kWBytes));
+          const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + sb * kBStageBytes));
+          const uint32_t dt = tmem + kTmemD + d * kTileN;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // K = 32 E4M3 = 32 B of each operand row
+            mma_f8_ss(dt, adesc + static_cast<uint64_t>(kk * 2),
+                      bdesc + static_cast<uint64_t>(kk * 2), idesc, kk > 0 ? 1u : 0u);
+          tc_commit(&dfull[d]);
+          tc_commit(&wempty[ws]);
+          tc_commit(&bempty[sb]);
         }
         tc_commit(drain);
         mbar_wait_drain(drain, 0, tmo);
@@ -583,6 +633,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     __syncwarp();
   } else if (warp < S::kConvWarps) {
     // ------------------------------------------------------------ INT4 -> E4M3 converters
+    // (E4M3 weights need none: these warps have no role then)
+    if constexpr (!kF8W) {
     const int quad = warp & 3;
     const int set = warp >> 2;                      // converts groups it % kConvSets == set
     const int m = quad * 32 + lane;                 // weight row of the tile = TMEM lane
@@ -677,6 +729,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       for (int it = set; it < n_groups; it += S::kConvSets)
         if (!convert(it, it)) break;
     }
+    }  // !kF8W
   } else if (warp < S::kWarpW) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - S::kConvWarps;
@@ -712,7 +765,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         float v = 0.0f;
         if (j < t.n_valid) {
           const int64_t r = t.row0 + j;
-          v = kGateUp ? __ldg(a.act_scale + __ldg(a.row_tokens + r)) : __ldg(a.act_scale + r);
+          if constexpr (kF8W) v = 1.0f;  // scales are per group, applied in the promotion
+          else v = kGateUp ? __ldg(a.act_scale + __ldg(a.row_tokens + r)) : __ldg(a.act_scale + r);
         }
         ts[i] = v;
       }
@@ -782,8 +836,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kBatch; ++i) {
             const int j = j0 + q * kTok + b0 + i;
-            key[i] = j < t.n_valid ? (kGateUp ? __ldg(a.row_tokens + t.row0 + j)
-                                              : static_cast<int>(t.row0 + j))
+            key[i] = j < t.n_valid ? ((kGateUp && !kF8W) ? __ldg(a.row_tokens + t.row0 + j)
+                                                         : static_cast<int>(t.row0 + j))
                                    : -1;
           }
           float v0[kBatch], v1[kBatch];
@@ -805,7 +859,15 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       }
       if (S::kEpiOffset && !mbar_wait(my_sfull, phs, abort_flag, tmo)) break;
       const int tb = ntile % S::kTileScBufs;
-      if (!mbar_wait(&tfull[tb], (ntile / S::kTileScBufs) & 1, abort_flag, tmo)) break;
+      if (!kF8W && !mbar_wait(&tfull[tb], (ntile / S::kTileScBufs) & 1, abort_flag, tmo)) break;
+      // E4M3 weights: one float32 scale per 128-row block and group, this row's
+      // block of [rows / 128, G] (gate rows, then up rows from half_rows on)
+      const float* wblk_sc = nullptr;
+      if constexpr (kF8W) {
+        const int blk = kGateUp ? (m < 64 ? t.mb / 2 : a.half_rows / kBM + t.mb / 2) : t.mb;
+        wblk_sc = static_cast<const float*>(a.wscale) + static_cast<int64_t>(blk) * G;
+      }
+      float sw_next = kF8W ? __ldg(wblk_sc) : 0.0f;
       const __nv_bfloat16* sTm =
           reinterpret_cast<const __nv_bfloat16*>(sT + tb * S::tile_sc_bytes(G)) + sc_off;
       if (S::kEpiSets > 1 && ntile > 0 &&
@@ -819,7 +881,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       // units: the G groups, then (offset mode 2) the correction sum_g s_g S_g,
       // which enters with the factor -8
       for (int g = 0; g < units_per_tile; ++g) {
-        const float sg = g < G ? __bfloat162float(sTm[g * kScStride]) : 0.0f;
+        const float sw = sw_next;                 // E4M3 weights: this group's block scale
+        if (kF8W && g + 1 < G) sw_next = __ldg(wblk_sc + g + 1);
+        const float sg = (!kF8W && g < G) ? __bfloat162float(sTm[g * kScStride]) : 0.0f;
         const float f = g < G ? sg * 512.0f : -8.0f;
         const float2 s512x2 = make_float2(f, f);
         const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
@@ -837,6 +901,16 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < kLdCols; i += 4) {
               const int o = (c * kLdCols + i) / 2;
+              if constexpr (kF8W) {  // acc += (s_w * s_a[column]) * D
+                const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
+                acc2[o] = __ffma2_rn(make_float2(sw * s4.x, sw * s4.y),
+                                     make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                     acc2[o]);
+                acc2[o + 1] = __ffma2_rn(
+                    make_float2(sw * s4.z, sw * s4.w),
+                    make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), acc2[o + 1]);
+                continue;
+              }
               acc2[o] = __ffma2_rn(
                   s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
               acc2[o + 1] = __ffma2_rn(
@@ -868,7 +942,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         if (S::kEpiOffset) mbar_arrive(my_sempty);
-        mbar_arrive(&tempty[tb]);
+        if (!kF8W) mbar_arrive(&tempty[tb]);
         if (S::kEpiSets > 1) mbar_arrive(loopdone);
       }
       }  // FP8
@@ -912,14 +986,16 @@ __global__ void __launch_bounds__(S::kThreads, 1)
                              smem_u32(sU + (j0 + jj) * 64 + q * 32), 128);
           }
           bulk_commit();
+          if constexpr (!kF8W) {  // E4M3-weight layers requantise h per 128-group later
 #pragma unroll
-          for (int jj = 0; jj < kEpiN; ++jj) acc[jj] = jj < n_here ? fabsf(acc[jj]) : 0.0f;
-          // per-column max over this warp's 32 rows: lane l ends with column l
+            for (int jj = 0; jj < kEpiN; ++jj) acc[jj] = jj < n_here ? fabsf(acc[jj]) : 0.0f;
+            // per-column max over this warp's 32 rows: lane l ends with column l
 #pragma unroll
-          for (int b = 0; b < kEpiN / 32; ++b) {
-            const float hm = column_max32(acc, b * 32, lane);
-            const int j = j0 + b * 32 + lane;
-            if (j < t.n_valid) atomicMax(a.row_amax + t.row0 + j, __float_as_uint(hm));
+            for (int b = 0; b < kEpiN / 32; ++b) {
+              const float hm = column_max32(acc, b * 32, lane);
+              const int j = j0 + b * 32 + lane;
+              if (j < t.n_valid) atomicMax(a.row_amax + t.row0 + j, __float_as_uint(hm));
+            }
           }
           bulk_wait_read_all();                     // sU may be refilled after this
           __syncwarp();
@@ -949,26 +1025,26 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in limit of sm_100
 
-template <class S, bool kGateUp, bool kI8 = false>
+template <class S, bool kGateUp, bool kI8 = false, bool kF8W = false>
 cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
                          const CUtensorMap& tmap_sc, const CUtensorMap& tmap_gs,
                          const GemmArgs& a, int num_ctas, cudaStream_t s) {
-  static_assert(S::smem_bytes(kGateUp, kMaxGroups, kMaxExperts) <= kMaxSmemPerBlock,
+  static_assert(S::smem_bytes(kGateUp, kMaxGroups, kMaxExperts, kF8W) <= kMaxSmemPerBlock,
                 "shared memory");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev >= 64 || !attr_set[dev]) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<S, kGateUp, kI8>,
+    err = cudaFuncSetAttribute(grouped_gemm_kernel<S, kGateUp, kI8, kF8W>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               S::smem_bytes(kGateUp, kMaxGroups, kMaxExperts));
+                               S::smem_bytes(kGateUp, kMaxGroups, kMaxExperts, kF8W));
     if (err != cudaSuccess) return err;
     if (dev < 64) attr_set[dev] = true;
   }
-  const int smem = S::smem_bytes(kGateUp, a.K / kGroup, a.E);
-  grouped_gemm_kernel<S, kGateUp, kI8><<<num_ctas, S::kThreads, smem, s>>>(tmap_w, tmap_act,
-                                                                           tmap_sc, tmap_gs, a);
+  const int smem = S::smem_bytes(kGateUp, a.K / kGroup, a.E, kF8W);
+  grouped_gemm_kernel<S, kGateUp, kI8, kF8W><<<num_ctas, S::kThreads, smem, s>>>(
+      tmap_w, tmap_act, tmap_sc, tmap_gs, a);
   return cudaGetLastError();
 }
 
@@ -1065,6 +1141,19 @@ cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap&
                    : launch_shape<I8Decode, false, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s);
   return gate_up ? launch_shape<I8Prefill, true, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s)
                  : launch_shape<I8Prefill, false, true>(tmap_w, tmap_act, tmap_w, tmap_act, a, num_ctas, s);
+}
+
+cudaError_t launch_fp8_block_gemm(bool gate_up, const CUtensorMap& tmap_w,
+                                  const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
+                                  cudaStream_t s) {
+  if (a.K % kGroup || a.K / kGroup > kMaxGroups || a.K <= 0 || a.n_rows % kBM ||
+      (gate_up && a.half_rows % kBM))
+    return cudaErrorInvalidValue;
+  // the tile-scale and sum-part maps are unused in this mode
+  return gate_up ? launch_shape<F8Block, true, false, true>(tmap_w, tmap_act, tmap_w, tmap_act, a,
+                                                            num_ctas, s)
+                 : launch_shape<F8Block, false, false, true>(tmap_w, tmap_act, tmap_w, tmap_act,
+                                                             a, num_ctas, s);
 }
 
 cudaError_t read_and_clear_device_error(int* value) {

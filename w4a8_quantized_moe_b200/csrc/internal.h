@@ -65,8 +65,21 @@ cudaError_t launch_pack_int4_channel(const void* w, int64_t R, int64_t K, int32_
 // sums[r] = sum of the 2 * 4 * words_per_row stored nibbles of row r.
 cudaError_t launch_nibble_row_sum(const int32_t* packed, int64_t R, int64_t words_per_row,
                                   int32_t* sums, int num_sms, cudaStream_t s);
+// y_shared (nullable): [T, H] float32 added to each token's routed sum.
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
-                           int64_t H, int k, void* out, int num_sms, cudaStream_t s);
+                           int64_t H, int k, void* out, int num_sms, cudaStream_t s,
+                           const float* y_shared = nullptr);
+// FP8 block weights: bf16 [R, K] -> E4M3 codes [R, K] + float32 scales
+// [R / 128, K / 128], scale = absmax / 448 per 128 x 128 block.
+cudaError_t launch_quant_fp8_block(const void* w, int64_t R, int64_t K, uint8_t* codes,
+                                   float* scales, cudaStream_t s);
+// Per-row, per-128-group E4M3 activations from bf16 (x_bf16) or float32 (x_f32)
+// input: codes [T, H], scales [T, H / 128].
+cudaError_t launch_act_quant_group(const void* x_bf16, const float* x_f32, int64_t T, int64_t H,
+                                   uint8_t* codes, float* scales, int num_sms, cudaStream_t s);
+// expert_offsets {0, T} and tile prefix {0, ceil(T / tile_n)} of a dense GEMM.
+cudaError_t launch_dense_tables(int32_t* offsets, int32_t* tile_prefix, int64_t T, int tile_n,
+                                cudaStream_t s);
 
 // ---- grouped_gemm.cu
 struct GemmArgs {
@@ -110,6 +123,14 @@ bool grouped_gemm_uses_sum_parts(bool decode);
 cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap& tmap_w,
                                    const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
                                    cudaStream_t s);
+// Dense GEMM with E4M3 weights and 128 x 128 block scales (one expert, E = 1):
+// tmap_w = codes [n_rows, K] bytes, box [64 (gate/up) or 128 rows x 128 B],
+// 128-byte swizzle; wscale = float32 [n_rows / 128, K / 128]; act_gsum = the
+// activations' float32 group scales [rows, K / 128]; act_scale, row_tokens
+// and row_amax unused (null).
+cudaError_t launch_fp8_block_gemm(bool gate_up, const CUtensorMap& tmap_w,
+                                  const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
+                                  cudaStream_t s);
 // One bounded wait on an mbarrier nothing arrives on (failure-detection self-test).
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
 

@@ -569,6 +569,91 @@ __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restric
   }
 }
 
+// ---------------------------------------------------------------- FP8 block quantisers
+// Weights: one CTA per 128 x 128 block (blockIdx.y: row block, blockIdx.x:
+// column block); thread i reads rows i / 16 + 16 j (j < 8), 8 columns at
+// (i % 16) * 8.  scale = float32(absmax / 448), codes = E4M3(w / scale).
+__global__ void __launch_bounds__(256) quant_fp8_block_kernel(const __nv_bfloat16* __restrict__ w,
+                                                              int64_t K, uint8_t* __restrict__ codes,
+                                                              float* __restrict__ scales) {
+  __shared__ float red[8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kGroup + tid / 16;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kGroup + (tid % 16) * 8;
+  uint4 v[8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[j] = __ldg(reinterpret_cast<const uint4*>(w + (r0 + 16 * j) * K + c0));
+    amax = fmaxf(amax, absmax8(v[j]));
+  }
+  amax = warp_max(amax);
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float scale = __fdiv_rn(amax, 448.0f);
+  if (tid == 0) scales[static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x] = scale;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float f[8];
+    unpack8(v[j], f);
+    *reinterpret_cast<uint2*>(codes + (r0 + 16 * j) * K + c0) = quant8(f, scale);
+  }
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  unpack8(__ldg(reinterpret_cast<const uint4*>(p)), f);
+}
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// Activations (bf16 x or float32 h): one float32 scale per row and 128-wide
+// group, scale = float32(absmax / 448).  8 values per thread; the 16
+// consecutive threads of a group reduce the absmax with shuffles (whole warps
+// run every iteration; H % 128 == 0 keeps a group inside one half-warp).
+template <class TIn>
+__global__ void __launch_bounds__(256) act_quant_group_kernel(const TIn* __restrict__ x, int64_t T,
+                                                              int64_t H, uint8_t* __restrict__ codes,
+                                                              float* __restrict__ scales) {
+  const int64_t per_row = H / 8;
+  const int64_t n = T * per_row;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t n_iter = (n + stride - 1) / stride;
+  for (int64_t it = 0; it < n_iter; ++it) {
+    const int64_t i = it * stride + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const bool active = i < n;
+    float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) load8(x + i * 8, f);
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 8));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 4));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    if (active) {
+      const float scale = __fdiv_rn(amax, 448.0f);
+      *reinterpret_cast<uint2*>(codes + i * 8) = quant8(f, scale);
+      if ((i & 15) == 0) scales[i / 16] = scale;   // row-major [T, H / 128]
+    }
+  }
+}
+
+// Expert tables of a dense (one-expert) GEMM over T rows.
+__global__ void dense_tables_kernel(int32_t* offsets, int32_t* tile_prefix, int32_t T, int tile_n) {
+  if (threadIdx.x == 0) {
+    offsets[0] = 0;
+    offsets[1] = T;
+    tile_prefix[0] = 0;
+    tile_prefix[1] = (T + tile_n - 1) / tile_n;
+  }
+}
+
 // ---------------------------------------------------------------- B200 weight layout
 // Word-local nibble interleave: element j of each group of 8 moves from
 // nibble j to nibble 2j (j < 4) or 2(j - 4) + 1 (j >= 4), so that w & 0x0F0F0F0F
@@ -610,6 +695,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       const int32_t* __restrict__ row_of,
                                                       const float* __restrict__ topk_w, int64_t T,
                                                       int64_t H, int k,
+                                                      const float* __restrict__ y_shared,
                                                       __nv_bfloat16* __restrict__ out) {
   const int64_t per_row = H / 8;
   const int64_t n = T * per_row;
@@ -626,6 +712,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       acc[2] = fmaf(wj, a.z, acc[2]); acc[3] = fmaf(wj, a.w, acc[3]);
       acc[4] = fmaf(wj, b.x, acc[4]); acc[5] = fmaf(wj, b.y, acc[5]);
       acc[6] = fmaf(wj, b.z, acc[6]); acc[7] = fmaf(wj, b.w, acc[7]);
+    }
+    if (y_shared) {  // the shared expert, added after the routed slots
+      const float4* src = reinterpret_cast<const float4*>(y_shared + t * H + c * 8);
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
     uint32_t p[4];
 #pragma unroll
@@ -773,11 +865,41 @@ cudaError_t launch_nibble_row_sum(const int32_t* packed, int64_t R, int64_t word
 }
 
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
-                           int64_t H, int k, void* out, int num_sms, cudaStream_t s) {
+                           int64_t H, int k, void* out, int num_sms, cudaStream_t s,
+                           const float* y_shared) {
   if (T == 0) return cudaSuccess;
   const int grid = grid_for(T * (H / 8), 256, num_sms);
-  combine_kernel<<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k,
+  combine_kernel<<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k, y_shared,
                                       static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_fp8_block(const void* w, int64_t R, int64_t K, uint8_t* codes,
+                                   float* scales, cudaStream_t s) {
+  if (R == 0 || K == 0) return cudaSuccess;
+  if (R / kGroup > 65535) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(K / kGroup), static_cast<unsigned>(R / kGroup));
+  quant_fp8_block_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), K, codes,
+                                              scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant_group(const void* x_bf16, const float* x_f32, int64_t T, int64_t H,
+                                   uint8_t* codes, float* scales, int num_sms, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if ((x_bf16 == nullptr) == (x_f32 == nullptr)) return cudaErrorInvalidValue;
+  const int grid = grid_for(T * (H / 8), 256, num_sms);
+  if (x_bf16)
+    act_quant_group_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x_bf16), T, H, codes, scales);
+  else
+    act_quant_group_kernel<float><<<grid, 256, 0, s>>>(x_f32, T, H, codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense_tables(int32_t* offsets, int32_t* tile_prefix, int64_t T, int tile_n,
+                                cudaStream_t s) {
+  dense_tables_kernel<<<1, 32, 0, s>>>(offsets, tile_prefix, static_cast<int32_t>(T), tile_n);
   return cudaGetLastError();
 }
 

@@ -183,6 +183,18 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// D (TMEM, F32) (+)= A (SMEM descriptor, E4M3) x B (SMEM descriptor, E4M3),
+// kind::f8f6f4, K = 32.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor: kind::f16, A = B = BF16, D = F32, both K-major,
 // M = 128, N = n (multiple of 16, 16..256).
 __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32_m128(uint32_t n) {
