@@ -110,3 +110,42 @@ def test_python_binding_refuses_cpu_tensors():
     import w4a8_quantized_moe_b200 as m
     with pytest.raises(ValueError, match="CUDA"):
         m.w4a8_quant_act_fp8_per_token(torch.zeros(4, 128, dtype=torch.bfloat16))
+
+
+def test_shared_expert_entries_validate_on_the_host(L):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    # block quantiser: both dimensions multiples of 128
+    assert L.w4a8_quant_fp8_block(fake, 100, 128, fake, fake, None) == 2
+    assert L.w4a8_quant_fp8_block(fake, 128, 200, fake, fake, None) == 2
+    assert L.w4a8_quant_fp8_block(None, 0, 128, None, None, None) == 0
+    assert L.w4a8_quant_fp8_block(vp((1 << 20) + 8), 128, 128, fake, fake, None) == 1
+    # group activation quantiser
+    assert L.w4a8_quant_act_fp8_group(fake, -1, 128, fake, fake, None) == 1
+    assert L.w4a8_quant_act_fp8_group(fake, 4, 100, fake, fake, None) == 2
+    assert L.w4a8_quant_act_fp8_group(None, 0, 128, None, None, None) == 0
+    # workspace sizes: host arithmetic, the combined layer needs both parts
+    T, H, I = 64, 6144, 2048
+    ws = L.w4a8_shared_expert_workspace_size(T, H, I)
+    assert ws >= T * H + T * (H // 128) * 4 + T * I * 4 + T * I + T * (I // 128) * 4
+    assert L.w4a8_shared_expert_workspace_size(-1, H, I) == 0
+    both = L.w4a8_moe_shared_workspace_size(T, H, I, 256, 8, I)
+    assert both >= L.w4a8_moe_workspace_size(T, H, I, 256, 8) + ws + T * H * 4 - 4096
+    # the expert alone: shapes, NULL, workspace, empty input
+    w = [fake] * 5
+    assert L.w4a8_shared_expert_forward(*w, 4, 256, 100, fake, fake, 1 << 40, None, None) == 2
+    assert L.w4a8_shared_expert_forward(*w, 4, 200, 128, fake, fake, 1 << 40, None, None) == 2
+    assert L.w4a8_shared_expert_forward(fake, None, fake, fake, fake, 4, 256, 128, fake, fake,
+                                        1 << 40, None, None) == 1
+    assert L.w4a8_shared_expert_forward(*w, 4, 256, 128, fake, fake, 64, None, None) == 4
+    assert L.w4a8_shared_expert_forward(None, None, None, None, None, 0, 256, 128, None, None, 0,
+                                        None, None) == 0
+    # the combined layer: the shared expert's width is checked, and its weights
+    routed = [fake] * 6
+    shared = [fake] * 4
+    assert L.w4a8_moe_forward_shared(*routed, *shared, 4, 256, 256, 100, 8, 2, fake, fake,
+                                     1 << 40, None, None, None) == 2
+    assert L.w4a8_moe_forward_shared(*routed, None, fake, fake, fake, 4, 256, 256, 128, 8, 2,
+                                     fake, fake, 1 << 40, None, None, None) == 1
+    assert L.w4a8_moe_forward_shared(*routed, *shared, 4, 256, 256, 128, 8, 2, fake, fake, 1024,
+                                     None, None, None) == 4
