@@ -138,3 +138,18 @@ def test_layer_with_shared_expert_full_size_sampled(ci):
     e_out = rel_fro(f64(out[torch.as_tensor(toks, device=dev)]), res["out"])
     print(f"\n[{cfg.name} + shared] sampled tokens {toks.tolist()} out rel-Frobenius {e_out:.2e}")
     assert e_out <= 2e-3
+
+
+def test_shared_expert_zero_tokens_and_bad_shapes():
+    dev = torch.device("cuda")
+    w13 = torch.zeros(256, 256, dtype=torch.bfloat16, device=dev)
+    w2 = torch.zeros(256, 128, dtype=torch.bfloat16, device=dev)
+    sh = w4.SharedExpertFP8.from_bf16(w13, w2)
+    y = sh(torch.zeros(0, 256, dtype=torch.bfloat16, device=dev))
+    assert y.shape == (0, 256)
+    # all-zero weights: every block scale is 0 and the output is exactly 0
+    y = sh(torch.randn(5, 256, device=dev).to(torch.bfloat16))
+    w4.w4a8_check_device_error()
+    assert torch.count_nonzero(y) == 0
+    with pytest.raises(w4.W4A8Error, match="UNSUPPORTED_SHAPE"):
+        w4.w4a8_quant_fp8_block(torch.zeros(100, 128, dtype=torch.bfloat16, device=dev))
