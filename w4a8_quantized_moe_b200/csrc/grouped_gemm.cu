@@ -53,11 +53,13 @@
 // TMEM by the converter warps) with the rows' group sums (three bf16 parts
 // each, written by the activation quantisers), accumulated like one more group.
 //
-// Two shapes of the same kernel: a decode shape (32-token tiles, 8 A slots,
-// 8 accumulators, 3 converter sets, 16 weight stages) for batches with few
-// tokens per expert, where pipeline depth hides the MMA and TMEM latencies,
-// and a prefill shape (128-token tiles) where each converted weight tile
-// feeds more tokens.
+// Two families of shapes of the same kernel: decode shapes (32-token tiles,
+// 8 groups in flight, 12-16 weight stages) for batches with few tokens per
+// expert, where pipeline depth hides the MMA and TMEM latencies, and prefill
+// shapes (128-token tiles) where each converted weight tile feeds more tokens.
+// The decode shapes pair the groups: one A slot, activation stage and
+// accumulator hold two consecutive groups, so each barrier round trip and MMA
+// commit serves two groups (the tensor-core issue rate sets the decode speed).
 //
 // Every wait is bounded (see ptx.cuh); a timed-out CTA drains its own
 // in-flight copies and MMAs, frees its TMEM and exits.
@@ -81,7 +83,7 @@ constexpr int kWStageBytes = kBM * kGroup / 2;      // 8 KB of packed INT4
 constexpr uint32_t kTmemCols = 512;
 
 template <int TileN, int WStages, int BStages, int ASlots, int DBufs, int ConvSets,
-          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetMode>
+          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetMode, int Pair = 0>
 struct Shape {
   static constexpr int kTileN = TileN;
   static constexpr int kWStages = WStages;
@@ -104,6 +106,11 @@ struct Shape {
   static constexpr bool kOffsetInMma = OffsetMode == 1;
   static constexpr bool kOffsetTile = OffsetMode == 2;
   static constexpr bool kEpiOffset = OffsetMode == 0;
+  // Paired groups: each ring element (A slot, activation stage, accumulator)
+  // holds two consecutive K groups, so every barrier wait, arrival and MMA
+  // commit is shared by two groups.  K / 128 must be even.
+  static constexpr bool kPair = Pair != 0;
+  static constexpr int kGPU = kPair ? 2 : 1;              // groups per ring element
   static constexpr int kEpiPerSet = 4 * EpiPerQuad;
   static constexpr int kEpiWarps = kEpiPerSet * EpiSets;
   static constexpr int kWarpW = kConvWarps + kEpiWarps;   // TMA: packed weights
@@ -113,16 +120,20 @@ struct Shape {
   static constexpr bool kUnified = ASlots == BStages && BStages == DBufs;
   static constexpr int kThreads = 32 * ((kWarpB + 1 + 3) / 4 * 4);
   static constexpr int kEpiN = TileN / EpiPerQuad;        // columns per epilogue warp
-  static constexpr int kBStageBytes = TileN * kGroup;
+  static constexpr int kBStageBytes = TileN * kGroup * kGPU;
   static constexpr int kUpBytes = 64 * TileN * 4;         // up-projection exchange
   static constexpr int kSumLd = kEpiN + 4;                // padded: 4-way bank spread on stores
   static constexpr int kTileScBufs = 2;                   // tile weight-scale buffers
-  static constexpr uint32_t kTmemA = 0;                   // A slots: 32 columns each
-  static constexpr uint32_t kTmemConst = ASlots * 32;     // E4M3 -2^-6 in every byte (offset MMAs)
-  static constexpr uint32_t kTmemD = kTmemConst + (kOffsetInMma ? 32 : 0);  // TileN columns each
+  static constexpr uint32_t kACols = 32 * kGPU;           // TMEM columns per A slot
+  static constexpr uint32_t kDCols = TileN * kGPU;        // TMEM columns per accumulator
+  static constexpr uint32_t kTmemA = 0;                   // A slots
+  static constexpr uint32_t kTmemConst = ASlots * kACols; // E4M3 -2^-6 in every byte (offset MMAs)
+  static constexpr uint32_t kTmemD = kTmemConst + (kOffsetInMma ? 32 : 0);  // accumulators
   static constexpr int kNumBars = 2 * WStages + 2 * BStages + 2 * ASlots + 2 * DBufs + 3 +
                                   2 * EpiSets * (1 + EpiPerQuad) + 2 * kTileScBufs + 1;
-  static_assert(kTmemD + DBufs * TileN <= kTmemCols, "TMEM budget exceeded");
+  static_assert(kTmemD + DBufs * kDCols <= kTmemCols, "TMEM budget exceeded");
+  static_assert(!kPair || (kEpiOffset && kUnified && ConvSets == 1),
+                "paired groups: epilogue offset, unified rings, one converter set");
   static_assert(kEpiN % 32 == 0 && kEpiN % LdCols == 0 && (LdCols == 16 || LdCols == 32),
                 "epilogue load width");
   static_assert(TileN % 16 == 0 && TileN <= 256, "MMA N");
@@ -149,12 +160,15 @@ struct Shape {
 };
 
 // Shapes.  By default each projection takes the shape measured fastest for it;
-// W4A8_GEMM_DECODE_SHAPE = 1..3 / W4A8_GEMM_PREFILL_SHAPE = 1..4 force one for both.
+// W4A8_GEMM_DECODE_SHAPE = 1..5 / W4A8_GEMM_PREFILL_SHAPE = 1..4 force one for both
+// (decode 5: the paired shapes, gate/up and down).
 //                            TileN        W   B  A  D cvt epi/q ld mma sets offset mode
 using DecodeOneSet  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;
 using DecodeTwoSets = Shape<kTileNDecode, 12, 8, 8, 8, 1, 1, 32, 2, 2, 0>;
 using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2, 0>;
 using DecodeTileCorr = Shape<kTileNDecode, 16, 8, 8, 7, 1, 1, 32, 2, 1, 2>;
+using DecodePair = Shape<kTileNDecode, 16, 4, 4, 4, 1, 1, 32, 2, 1, 0, 1>;  // 2 groups per element
+using DecodePairTwoSets = Shape<kTileNDecode, 12, 4, 4, 4, 1, 1, 32, 2, 2, 0, 1>;
 using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 3, 3, 1, 4, 16, 2, 1, 1>;
 using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 3, 2, 1, 2, 16, 2, 1, 1>;
 using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
@@ -368,8 +382,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   const int Gp = (G + 15) & ~15;
   const int KC = 3 * Gp;
   const int kNC = S::kOffsetTile ? (KC + 63) / 64 : 0;
-  const int ab_per_tile = G + kNC;                       // A slot / B stage steps
-  const int units_per_tile = G + (S::kOffsetTile ? 1 : 0);  // accumulators
+  constexpr int kGPU = S::kGPU;                          // groups per ring element
+  const int ab_per_tile = G / kGPU + kNC;                // A slot / B stage steps
+  const int units_per_tile = G / kGPU + (S::kOffsetTile ? 1 : 0);  // accumulators
   const int n_units = my_tiles * units_per_tile;
 
   if (warp == S::kWarpW) {
@@ -432,18 +447,26 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       const int n_ops = t.n_mma >> 4;
       const uint32_t tx = t.n_mma * kGroup;
       const int32_t y0 = static_cast<int32_t>(t.row0) + 16 * lane;
-      // G stages of codes, then (per-tile correction) kNC stages of the bf16
-      // group-sum parts, 128 bytes of each row per stage
+      // G stages of codes (kGPU groups per stage, each in its own kTileN-row
+      // half), then (per-tile correction) kNC stages of the bf16 group-sum
+      // parts, 128 bytes of each row per stage
       for (int g = 0; g < ab_per_tile; ++g) {
         const int s = it % kBStages;
         const uint32_t ph = (it / kBStages) & 1;
         if (!mbar_wait(&bempty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
         const uint32_t dB = smem_u32(sB + s * kBStageBytes);
-        if (lane == 0) mbar_arrive_expect_tx(&bfull[s], tx);
+        const bool codes = g * kGPU < G;
+        if (lane == 0) mbar_arrive_expect_tx(&bfull[s], codes ? kGPU * tx : tx);
         __syncwarp();
         if (lane < n_ops) {
-          if (g < G) tma_load_2d(dB + lane * 16 * kGroup, &tmap_act, &bfull[s], g * kGroup, y0);
-          else tma_load_2d(dB + lane * 16 * kGroup, &tmap_gs, &bfull[s], (g - G) * 128, y0);
+          if (codes) {
+#pragma unroll
+            for (int h = 0; h < kGPU; ++h)
+              tma_load_2d(dB + h * (kTileN * kGroup) + lane * 16 * kGroup, &tmap_act, &bfull[s],
+                          (g * kGPU + h) * kGroup, y0);
+          } else {
+            tma_load_2d(dB + lane * 16 * kGroup, &tmap_gs, &bfull[s], (g - G) * 128, y0);
+          }
         }
         ++it;
       }
@@ -604,19 +627,26 @@ __global__ void __launch_bounds__(S::kThreads, 1)
              !mbar_wait(&afull[as], pha, abort_flag, tmo)))
           break;
         tc_fence_after();
-        const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + sb * kBStageBytes));
-        const uint32_t dt = tmem + kTmemD + d * kTileN;
-        const uint32_t at = tmem + kTmemA + as * 32;
+        const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB + sb * kBStageBytes));
+        const uint32_t dt0 = tmem + kTmemD + d * S::kDCols;
+        const uint32_t at0 = tmem + kTmemA + as * S::kACols;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = 32 E4M3 per MMA: 8 TMEM columns, 32 B of smem
-          mma_f8_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                    kk > 0 ? 1u : 0u);
-          if constexpr (S::kOffsetInMma) {
-            // D += sum_k a_k * (-2^-6) over the same 32 k (A = the constant TMEM
-            // columns): after each pair D holds 2^-9 * sum a * q of the slices so
-            // far, so the offset cancels at the magnitude of a 32-element partial
-            // sum, not of the whole group
-            mma_f8_ts(dt, tmem + S::kTmemConst, bdesc + static_cast<uint64_t>(kk * 2), idesc, 1u);
+        for (int h = 0; h < kGPU; ++h) {  // the element's groups: own A columns, B half, accumulator
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(h * (kTileN * kGroup / 16));
+          const uint32_t dt = dt0 + h * kTileN;
+          const uint32_t at = at0 + h * 32;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // K = 32 E4M3 per MMA: 8 TMEM columns, 32 B of smem
+            mma_f8_ts(dt, at + kk * 8, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                      kk > 0 ? 1u : 0u);
+            if constexpr (S::kOffsetInMma) {
+              // D += sum_k a_k * (-2^-6) over the same 32 k (A = the constant TMEM
+              // columns): after each pair D holds 2^-9 * sum a * q of the slices so
+              // far, so the offset cancels at the magnitude of a 32-element partial
+              // sum, not of the whole group
+              mma_f8_ts(dt, tmem + S::kTmemConst, bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                        1u);
+            }
           }
         }
         if constexpr (kUniAll) {
@@ -650,16 +680,18 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
     }
-    // one weight group: W stage wit -> A slot ait
-    auto convert = [&](int wit, int ait) -> bool {
+    // one weight group: W stage wit -> group h of A slot ait (the slot is
+    // claimed with its first group and published after its last)
+    auto convert = [&](int wit, int ait, int h) -> bool {
+      const bool first = h == 0, last = h == kGPU - 1;
       const int s = wit % kWStages;
       const uint32_t ph = (wit / kWStages) & 1;
       const int as = ait % kASlots;
       const uint32_t pha = (ait / kASlots) & 1;
       const bool rw = mbar_test_wait(&wfull[s], ph);   // both polls in flight at once
-      const bool ra = mbar_test_wait(&aempty[as], pha ^ 1);
+      const bool ra = !first || mbar_test_wait(&aempty[as], pha ^ 1);
       if (!(rw && ra) && (!mbar_wait(&wfull[s], ph, abort_flag, tmo) ||
-                          !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo)))
+                          (first && !mbar_wait(&aempty[as], pha ^ 1, abort_flag, tmo))))
         return false;
       tc_fence_after();
       const uint32_t row = smem_u32(sW + s * kWStageBytes) + m * 64;
@@ -676,11 +708,13 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&wempty[s]);       // the stage's bytes are in registers
-      tmem_st_32x32b_x32(tmem + lane_base + kTmemA + as * 32, r);
+      tmem_st_32x32b_x32(tmem + lane_base + kTmemA + as * S::kACols + h * 32, r);
       tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[as]);
+      if (last) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[as]);
+      }
       return true;
     };
     if constexpr (S::kOffsetTile) {
@@ -693,7 +727,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       bool ok = true;
       for (int nt = 0; ok && nt < my_tiles; ++nt) {
         for (int g = 0; g < G; ++g)
-          if (!convert(nt * G + g, ait++)) { ok = false; break; }
+          if (!convert(nt * G + g, ait++, 0)) { ok = false; break; }
         if (!ok) break;
         const int tb = nt % S::kTileScBufs;
         if (!mbar_wait(&tfull[tb], (nt / S::kTileScBufs) & 1, abort_flag, tmo)) break;
@@ -726,8 +760,11 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         if (lane == 0) mbar_arrive(&tempty[tb]);
       }
     } else {
-      for (int it = set; it < n_groups; it += S::kConvSets)
-        if (!convert(it, it)) break;
+      // ring element ue holds groups kGPU * ue .. kGPU * ue + kGPU - 1
+      bool ok = true;
+      for (int ue = set; ok && ue < n_units; ue += S::kConvSets)
+        for (int h = 0; h < kGPU; ++h)
+          if (!convert(ue * kGPU + h, ue, h)) { ok = false; break; }
     }
     }  // !kF8W
   } else if (warp < S::kWarpW) {
@@ -880,46 +917,50 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       uint32_t phd = (it / kDBufs) & 1;
       // units: the G groups, then (offset mode 2) the correction sum_g s_g S_g,
       // which enters with the factor -8
-      for (int g = 0; g < units_per_tile; ++g) {
-        const float sw = sw_next;                 // E4M3 weights: this group's block scale
-        if (kF8W && g + 1 < G) sw_next = __ldg(wblk_sc + g + 1);
-        const float sg = (!kF8W && g < G) ? __bfloat162float(sTm[g * kScStride]) : 0.0f;
-        const float f = g < G ? sg * 512.0f : -8.0f;
-        const float2 s512x2 = make_float2(f, f);
-        const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
-        const float* sg_row = sSl + g * kSumLd;
+      for (int u = 0; u < units_per_tile; ++u) {
         if (!mbar_wait(&dfull[d], phd, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t taddr = tmem + lane_base + kTmemD + d * kTileN + j0;
 #pragma unroll
-        for (int c = 0; c < kEpiN / kLdCols; ++c) {
-          if (j0 + c * kLdCols < t.n_mma) {
-            uint32_t v[kLdCols];
-            if constexpr (kLdCols == 32) tmem_ld_32x32b_x32(taddr + c * 32, v);
-            else tmem_ld_32x32b_x16(taddr + c * 16, v);
-            tmem_wait_ld();
+        for (int h = 0; h < kGPU; ++h) {  // the accumulator's groups
+          const int g = u * kGPU + h;
+          const float sw = sw_next;                 // E4M3 weights: this group's block scale
+          if (kF8W && g + 1 < G) sw_next = __ldg(wblk_sc + g + 1);
+          const float sg = (!kF8W && g < G) ? __bfloat162float(sTm[g * kScStride]) : 0.0f;
+          const float f = g < G ? sg * 512.0f : -8.0f;
+          const float2 s512x2 = make_float2(f, f);
+          const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
+          const float* sg_row = sSl + g * kSumLd;
+          const uint32_t taddr = tmem + lane_base + kTmemD + d * S::kDCols + h * kTileN + j0;
 #pragma unroll
-            for (int i = 0; i < kLdCols; i += 4) {
-              const int o = (c * kLdCols + i) / 2;
-              if constexpr (kF8W) {  // acc += (s_w * s_a[column]) * D
-                const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
-                acc2[o] = __ffma2_rn(make_float2(sw * s4.x, sw * s4.y),
-                                     make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
-                                     acc2[o]);
+          for (int c = 0; c < kEpiN / kLdCols; ++c) {
+            if (j0 + c * kLdCols < t.n_mma) {
+              uint32_t v[kLdCols];
+              if constexpr (kLdCols == 32) tmem_ld_32x32b_x32(taddr + c * 32, v);
+              else tmem_ld_32x32b_x16(taddr + c * 16, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < kLdCols; i += 4) {
+                const int o = (c * kLdCols + i) / 2;
+                if constexpr (kF8W) {  // acc += (s_w * s_a[column]) * D
+                  const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
+                  acc2[o] = __ffma2_rn(make_float2(sw * s4.x, sw * s4.y),
+                                       make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                       acc2[o]);
+                  acc2[o + 1] = __ffma2_rn(
+                      make_float2(sw * s4.z, sw * s4.w),
+                      make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), acc2[o + 1]);
+                  continue;
+                }
+                acc2[o] = __ffma2_rn(
+                    s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
                 acc2[o + 1] = __ffma2_rn(
-                    make_float2(sw * s4.z, sw * s4.w),
-                    make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), acc2[o + 1]);
-                continue;
-              }
-              acc2[o] = __ffma2_rn(
-                  s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
-              acc2[o + 1] = __ffma2_rn(
-                  s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
-                  acc2[o + 1]);
-              if constexpr (S::kEpiOffset) {  // remove the +8 offset: - 8 s_g S_g
-                const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
-                acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
-                acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
+                    s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
+                    acc2[o + 1]);
+                if constexpr (S::kEpiOffset) {  // remove the +8 offset: - 8 s_g S_g
+                  const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
+                  acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
+                  acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
+                }
               }
             }
           }
@@ -1089,11 +1130,16 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
   if (decode) {
     // gate/up (48 groups per tile at H = 6144) runs best with one epilogue set
     // and a deep weight ring; down (16 groups per tile) with two epilogue sets,
-    // whose tile finalize then overlaps the other set's groups
-    const int d = dshape != 0 ? dshape : (gate_up ? 1 : 2);
+    // whose tile finalize then overlaps the other set's groups.  Both pair the
+    // groups (two per ring element) when K / 128 is even.
+    const bool even = (a.K / kGroup) % 2 == 0;
+    const int d = dshape != 0 ? dshape : (even ? 5 : (gate_up ? 1 : 2));
     if (d == 1) return launch_either<DecodeOneSet>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     if (d == 3) return launch_either<DecodeTwoCvt>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     if (d == 4) return launch_either<DecodeTileCorr>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
+    if (d == 5 && (a.K / kGroup) % 2 == 0)
+      return gate_up ? launch_either<DecodePair>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s)
+                     : launch_either<DecodePairTwoSets>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     return launch_either<DecodeTwoSets>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
   }
   const int p = prefill_shape();
