@@ -279,7 +279,7 @@ def bench_reference(args, cfg, rank):
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
                 impl="reference",
                 config=dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
-                            sample_tokens_per_step=len(s.tokens)),
+                            variant=args.variant, sample_tokens_per_step=len(s.tokens)),
                 cpu_baseline=dict(value=value, unit="tokens/s", cores=s.cores, kind="oracle",
                                   sample=s.describe(tot / args.steps)),
                 e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0,
