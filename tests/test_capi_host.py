@@ -149,3 +149,17 @@ def test_shared_expert_entries_validate_on_the_host(L):
                                      fake, fake, 1 << 40, None, None, None) == 1
     assert L.w4a8_moe_forward_shared(*routed, *shared, 4, 256, 256, 128, 8, 2, fake, fake, 1024,
                                      None, None, None) == 4
+
+
+def test_binding_checks_shared_expert_arguments_before_any_cuda_call():
+    import torch
+    import w4a8_quantized_moe_b200 as m
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        m.w4a8_quant_fp8_block(torch.zeros(128, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        m.w4a8_quant_act_fp8_group(x)
+    w13c = torch.zeros(256, 256, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        m.w4a8_shared_expert_forward(x, w13c, torch.zeros(2, 2), torch.zeros(256, 128,
+                                     dtype=torch.uint8), torch.zeros(2, 1))
