@@ -44,18 +44,19 @@ have no pin beyond those of their parts.
 """
 from .numerics import (bf16_bits_to_f64, f64_to_bf16_bits, bf16_round, f32_round,
                        e4m3_decode, e4m3_encode, E4M3_MAX)
-from .quant import (rtn_quantize_int4, mse_clip_quantize_int4, CLIP_RATIOS, pack_uint4b8,
+from .quant import (rtn_quantize_int4, mse_clip_quantize_int4, mse_clip_candidates,
+                    MSE_ERR_REL_BOUND, CLIP_RATIOS, pack_uint4b8,
                     unpack_uint4b8, dequantize_int4, quant_act_fp8_per_token,
                     quant_act_int8_per_token, rtn_quantize_int4_channel)
-from .moe import route_topk, permute_by_expert, moe_forward, ExpertStore
+from .moe import route_topk, permute_by_expert, moe_forward, expert_forward, ExpertStore
 from .shared import (quant_fp8_block, dequant_fp8_block, quant_act_fp8_group,
                      dequant_act_fp8_group, shared_expert_forward)
 
 __all__ = ["bf16_bits_to_f64", "f64_to_bf16_bits", "bf16_round", "f32_round",
            "e4m3_decode", "e4m3_encode", "E4M3_MAX", "rtn_quantize_int4",
-           "mse_clip_quantize_int4", "CLIP_RATIOS",
+           "mse_clip_quantize_int4", "mse_clip_candidates", "MSE_ERR_REL_BOUND", "CLIP_RATIOS",
            "pack_uint4b8", "unpack_uint4b8", "dequantize_int4",
            "quant_act_fp8_per_token", "quant_act_int8_per_token", "route_topk", "permute_by_expert",
-           "moe_forward", "ExpertStore", "rtn_quantize_int4_channel", "quant_fp8_block",
+           "moe_forward", "expert_forward", "ExpertStore", "rtn_quantize_int4_channel", "quant_fp8_block",
            "dequant_fp8_block", "quant_act_fp8_group", "dequant_act_fp8_group",
            "shared_expert_forward"]

@@ -31,6 +31,8 @@ all-zero codes.
 """
 from __future__ import annotations
 
+from fractions import Fraction
+
 import numpy as np
 
 from .numerics import bf16_round, f32_round, e4m3_encode, E4M3_MAX
@@ -64,37 +66,32 @@ def rtn_quantize_int4(w, group: int = GROUP):
 CLIP_RATIOS = np.array([np.float32((100.0 - 3.0 * i) / 100.0) for i in range(11)],
                        dtype=np.float32)
 
-
-def _squared_error_fixed_order(d):
-    """Sum of d**2 over the last axis (128 = 32 x 4) in float64, in one fixed
-    order: each run of 4 consecutive values summed in sequence, then the 32
-    partial sums combined by five pairwise (xor 16, 8, 4, 2, 1) exchanges.
-    The pages do not say how the MSE is accumulated; fixing the order makes the
-    arg-min below a deterministic function of the inputs, which the kernel
-    reproduces operation for operation."""
-    sq = d * d
-    p = sq[..., 0::4] + sq[..., 1::4]
-    p = p + sq[..., 2::4]
-    p = p + sq[..., 3::4]
-    lanes = np.arange(32)
-    for off in (16, 8, 4, 2, 1):
-        p = p + p[..., lanes ^ off]
-    return p[..., 0]
+# Relative bound on |e_float - e_exact| for one candidate's squared error over a
+# group of 128, e_float computed below in float64 in any summation order.  Each
+# term fl(fl(w - q s)^2) is within (1 + u)^3 - 1 < 3.0001 u of the exact square
+# (q s is exact: a 4-bit integer times a bf16 scale; one rounding for the
+# difference, one for the square; u = 2^-53); summing 128 nonnegative terms in
+# any order adds at most (1 + u)^127 - 1 < 127.001 u.  2^-45 = 256 u covers both.
+MSE_ERR_REL_BOUND = 2.0 ** -45
 
 
-def mse_clip_quantize_int4(w, group: int = GROUP):
-    """Symmetric INT4 with the per-group MSE clip search (model card,
-    "quantisation method": for each group of 128, 11 shrink ratios of the
-    scale from 1.00 to 0.70 are tried and the MSE-optimal scale is kept).
+def _exact_group_error(wrow, qrow, s) -> Fraction:
+    """Sum over the group of (w - q s)^2 in exact rational arithmetic."""
+    sf = Fraction(float(s))
+    return sum(((Fraction(float(w)) - int(q) * sf) ** 2 for w, q in zip(wrow, qrow)),
+               Fraction(0))
 
-    For each ratio r (float32 ``CLIP_RATIOS``, tried from 1.00 down):
-      s_r = bf16(float32(float32(absmax * r) / 7));
-      q_r = clamp(round_half_even(float32(w / s_r)), -8, 7), 0 where s_r = 0;
-      e_r = sum over the group of (w - q_r * s_r)**2 in float64 (fixed order,
-            ``_squared_error_fixed_order``).
-    The first ratio with the smallest e_r is kept (ties keep the larger
-    scale).  r = 1.00 is exactly ``rtn_quantize_int4``.  With r < 1 the code
-    -8 becomes reachable.  Returns ``(q, s)`` as ``rtn_quantize_int4`` does.
+
+def mse_clip_candidates(w, group: int = GROUP):
+    """The 11 candidates of the per-group MSE clip search and their errors.
+
+    For each ratio r_i (float32 ``CLIP_RATIOS``, i = 0 .. 10):
+      s_i = bf16(float32(float32(absmax * r_i) / 7));
+      q_i = clamp(round_half_even(float32(w / s_i)), -8, 7), 0 where s_i = 0;
+      e_i = sum over the group of (w - q_i * s_i)^2, computed in float64; it is
+            within ``MSE_ERR_REL_BOUND * e_i`` of the exact value.
+    Returns ``(q [11, R, K] int8, s [11, R, K // group] float64 holding bf16
+    values, e [11, R, K // group] float64)``.
     """
     w = np.asarray(w, dtype=np.float64)
     R, K = w.shape
@@ -102,20 +99,57 @@ def mse_clip_quantize_int4(w, group: int = GROUP):
         raise ValueError("group must be 128 and divide K")
     wg = w.reshape(R, K // group, group)
     amax = np.abs(wg).max(axis=2)
-    best_e = np.full(amax.shape, np.inf)
-    best_q = np.zeros(wg.shape)
-    best_s = np.zeros(amax.shape)
+    qs, ss, es = [], [], []
     for r in CLIP_RATIOS:
         s = bf16_round(f32_round(f32_round(amax * np.float64(r)) / 7.0))
         with np.errstate(divide="ignore", invalid="ignore"):
             q = np.clip(np.rint(f32_round(wg / s[..., None])), -8, 7)
         q = np.where(s[..., None] == 0.0, 0.0, q)
-        e = _squared_error_fixed_order(wg - q * s[..., None])
-        take = e < best_e
-        best_e = np.where(take, e, best_e)
-        best_s = np.where(take, s, best_s)
-        best_q = np.where(take[..., None], q, best_q)
-    return best_q.astype(np.int8).reshape(R, K), best_s
+        d = wg - q * s[..., None]
+        es.append(np.sum(d * d, axis=2))
+        qs.append(q.astype(np.int8).reshape(R, K))
+        ss.append(s)
+    return np.stack(qs), np.stack(ss), np.stack(es)
+
+
+def mse_clip_quantize_int4(w, group: int = GROUP):
+    """Symmetric INT4 with the per-group MSE clip search (model card,
+    "quantisation method": for each group of 128, 11 shrink ratios of the
+    scale from 1.00 to 0.70 are tried and the MSE-optimal scale is kept).
+
+    The candidates are those of ``mse_clip_candidates``.  The kept candidate
+    is the one with the least EXACT squared error; among exact ties the first
+    (largest) ratio.  The float64 errors decide wherever they are further
+    apart than their error bound; candidates that stay within the bound of the
+    least error are compared in rational arithmetic.  r = 1.00 is exactly
+    ``rtn_quantize_int4``; with r < 1 the code -8 becomes reachable.  Returns
+    ``(q, s)`` as ``rtn_quantize_int4`` does.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    R, K = w.shape
+    q_all, s_all, e_all = mse_clip_candidates(w, group)
+    G = K // group
+    B = MSE_ERR_REL_BOUND
+    # a candidate whose scale equals an earlier candidate's is the same candidate
+    dup = np.zeros(e_all.shape, dtype=bool)
+    for i in range(1, 11):
+        dup[i] = np.any(s_all[:i] == s_all[i][None], axis=0)
+    e_cmp = np.where(dup, np.inf, e_all)
+    lo = e_cmp * (1.0 - B)                       # exact error is within [lo, hi]
+    hi = e_cmp * (1.0 + B)
+    best_hi = hi.min(axis=0)
+    contenders = lo <= best_hi[None]             # [11, R, G]: could be the minimum
+    choice = np.argmin(e_cmp, axis=0)            # decided where one contender remains
+    wg = w.reshape(R, G, group)
+    qg = q_all.reshape(11, R, G, group)
+    for r, g in zip(*np.nonzero(contenders.sum(axis=0) > 1)):
+        cands = np.nonzero(contenders[:, r, g])[0]
+        exact = [_exact_group_error(wg[r, g], qg[i, r, g], s_all[i, r, g]) for i in cands]
+        first_min = min(range(len(cands)), key=lambda j: exact[j])   # first of the exact minima
+        choice[r, g] = cands[first_min]
+    q = np.take_along_axis(qg, choice[None, ..., None], axis=0)[0].reshape(R, K)
+    s = np.take_along_axis(s_all, choice[None], axis=0)[0]
+    return q.astype(np.int8), s
 
 
 def rtn_quantize_int4_channel(w):

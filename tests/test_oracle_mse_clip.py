@@ -105,3 +105,64 @@ def test_gaussian_reconstruction_error_drops_like_the_pages_report():
     q, s = oracle.mse_clip_quantize_int4(w)
     rel = np.linalg.norm(w - oracle.dequantize_int4(oracle.pack_uint4b8(q), s)) / np.linalg.norm(w)
     assert 0.095 < rel < 0.107, rel
+
+
+def _exact_errors(group: np.ndarray):
+    """Exact squared error of each of the 11 candidates, built independently
+    (numpy float32 scale route, torch bf16 conversion, rational sums)."""
+    g32 = group.astype(np.float32)
+    amax = np.float32(np.abs(g32).max())
+    out = []
+    for i in range(11):
+        r = np.float32((100.0 - 3.0 * i) / 100.0)
+        s = np.float32(_bf16_torch(np.float32(np.float32(amax * r) / np.float32(7.0))))
+        q = np.zeros(128) if s == 0 else np.clip(np.rint((g32 / s).astype(np.float32)), -8, 7)
+        out.append((float(s), sum((Fraction(float(w)) - int(qq) * Fraction(float(s))) ** 2
+                                  for w, qq in zip(g32, q))))
+    return out
+
+
+def test_float_errors_within_the_stated_bound():
+    # the float64 candidate errors stay within MSE_ERR_REL_BOUND of the exact
+    # sums, on Gaussian, heavy-tailed, subnormal-heavy and outlier groups
+    rng = np.random.default_rng(21)
+    rows = [rng.normal(0, 0.02, 256), rng.standard_t(2, 256) * 0.01,
+            rng.normal(0, 1e-39, 256), np.where(rng.random(256) < 0.02, 3.0, 1e-3)]
+    w = oracle.bf16_round(np.stack(rows))
+    q_all, s_all, e_all = oracle.mse_clip_candidates(w)
+    for r in range(w.shape[0]):
+        for g in range(2):
+            exact = _exact_errors(w[r, g * 128:(g + 1) * 128])
+            for i, (s, ex) in enumerate(exact):
+                assert s_all[i, r, g] == s
+                assert abs(Fraction(float(e_all[i, r, g])) - ex) <= \
+                    Fraction(oracle.MSE_ERR_REL_BOUND) * ex
+
+
+# Sparse groups in which two DISTINCT candidate scales give exactly the same
+# squared error (found by a seeded search over groups of 1-3 nonzero bf16
+# values): ((position, value) pairs, the tied candidate indices).  The rule
+# keeps the first of the exact minima, i.e. the larger ratio.
+EXACT_TIES = [
+    ([(34, "-0x1.ea00000000000p-2"), (47, "-0x1.cc00000000000p-3")], (4, 5)),
+    ([(127, "-0x1.3800000000000p-3"), (123, "-0x1.4200000000000p-3")], (0, 5)),
+    ([(53, "-0x1.f000000000000p-2"), (79, "0x1.6a00000000000p-1")], (0, 1)),
+    ([(79, "-0x1.0a00000000000p-5"), (15, "-0x1.f000000000000p-1"),
+      (75, "0x1.0000000000000p+0")], (0, 1)),
+    ([(123, "-0x1.9400000000000p-1"), (9, "-0x1.8400000000000p-1"),
+      (89, "0x1.4e00000000000p-5")], (1, 5)),
+]
+
+
+@pytest.mark.parametrize("case", range(len(EXACT_TIES)))
+def test_exact_ties_keep_the_larger_ratio(case):
+    vals, (i, j) = EXACT_TIES[case]
+    g = np.zeros(128)
+    for pos, hx in vals:
+        g[pos] = float.fromhex(hx)
+    exact = _exact_errors(g)
+    assert exact[i][0] != exact[j][0]                  # two different scales ...
+    assert exact[i][1] == exact[j][1]                  # ... with the same exact error
+    assert exact[i][1] == min(e for _, e in exact)     # and it is the least
+    q, s = oracle.mse_clip_quantize_int4(g[None])
+    assert s[0, 0] == exact[i][0]
