@@ -112,9 +112,36 @@ def _silu(x):
     return x / (1.0 + np.exp(-x))
 
 
+def expert_forward(x_deq, expert, act_format: str = "fp8"):
+    """One expert on the dequantised activation rows ``x_deq`` (float64 [n, H]):
+    gate/up GEMM, SwiGLU, requantisation of h per row, down GEMM.
+
+    ``expert`` = ``(w13_packed, s13, w2_packed, s2)``.  Returns ``(h [n, I],
+    h codes [n, I], h scales [n], Y [n, H])``.
+    """
+    quant, decode = _act_codec(act_format)
+    w13p, s13, w2p, s2 = expert
+    I = w13p.shape[0] // 2
+    H_ = w13p.shape[1] * 8
+    G = x_deq @ dequantize_int4(w13p, s13, group=H_ // s13.shape[1]).T   # [n, 2I]
+    h = _silu(G[:, :I]) * G[:, I:]
+    hc, hs = quant(h)
+    hd = hs[:, None] * decode(hc)
+    Ye = hd @ dequantize_int4(w2p, s2, group=I // s2.shape[1]).T        # [n, H]
+    return h, hc, hs, Ye
+
+
+def _act_codec(act_format: str):
+    if act_format == "fp8":
+        return quant_act_fp8_per_token, e4m3_decode
+    if act_format == "int8":
+        return quant_act_int8_per_token, lambda c: np.asarray(c, dtype=np.float64)
+    raise ValueError(f"unknown act_format {act_format!r}")
+
+
 def moe_forward(hidden, logits, experts: Sequence, k: int,
                 tokens: Optional[np.ndarray] = None, hidden_of_tokens=None,
-                act_format: str = "fp8", shared=None):
+                act_format: str = "fp8", shared=None, expert_map=None):
     """The whole layer for all tokens, or for the token subset ``tokens``.
 
     ``hidden``: float64 [T, H] (bf16 values); ``logits``: float32 [T, E];
@@ -132,6 +159,10 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
     w2_codes, w2_scales)``; its ``shared_expert_forward`` result for the rows
     of ``tokens`` is returned under ``shared`` and its ``y`` is added to the
     routed sum before the bf16 rounding.
+
+    ``expert_map``: optional ``f(tasks, act_format) -> results`` that evaluates
+    ``expert_forward`` for each ``(e, x_deq rows)`` task in order (e.g. in
+    worker processes); by default each task runs here on ``experts[e]``.
 
     Returns a dict with ``topk_ids``, ``topk_w``, ``expert_offsets``,
     ``sorted_token_ids``, ``row_of``, ``act_codes`` / ``act_scales`` (rows of
@@ -151,12 +182,7 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
                                                                          dtype=np.float64)
     H = x_rows.shape[1]
 
-    if act_format == "fp8":
-        quant, decode = quant_act_fp8_per_token, e4m3_decode
-    elif act_format == "int8":
-        quant, decode = quant_act_int8_per_token, lambda c: np.asarray(c, dtype=np.float64)
-    else:
-        raise ValueError(f"unknown act_format {act_format!r}")
+    quant, decode = _act_codec(act_format)
     codes, a_scale = quant(x_rows)
     x_deq = a_scale[:, None] * decode(codes)               # exact: 24-bit x <= 8-bit significands
 
@@ -165,20 +191,17 @@ def moe_forward(hidden, logits, experts: Sequence, k: int,
     inter_h: Dict[int, np.ndarray] = {}
     inter_codes: Dict[int, np.ndarray] = {}
     inter_scales: Dict[int, float] = {}
+    tasks = []
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         rows = need_rows[(need_rows >= lo) & (need_rows < hi)]
-        if rows.size == 0:
-            continue
-        w13p, s13, w2p, s2 = experts[e]
-        I = w13p.shape[0] // 2
-        X = x_deq[[pos[int(sorted_tok[r])] for r in rows]]  # [n, H]
-        H_ = w13p.shape[1] * 8
-        G = X @ dequantize_int4(w13p, s13, group=H_ // s13.shape[1]).T   # [n, 2I]
-        h = _silu(G[:, :I]) * G[:, I:]
-        hc, hs = quant(h)
-        hd = hs[:, None] * decode(hc)
-        Ye = hd @ dequantize_int4(w2p, s2, group=I // s2.shape[1]).T     # [n, H]
+        if rows.size:
+            tasks.append((e, rows, x_deq[[pos[int(sorted_tok[r])] for r in rows]]))
+    if expert_map is None:
+        results = [expert_forward(X, experts[e], act_format) for e, _, X in tasks]
+    else:
+        results = expert_map([(e, X) for e, _, X in tasks], act_format)
+    for (e, rows, _), (h, hc, hs, Ye) in zip(tasks, results):
         for i, r in enumerate(rows):
             Y[int(r)] = Ye[i]
             inter_h[int(r)] = h[i]

@@ -4,6 +4,7 @@ import torch
 
 import oracle
 import workloads
+from oracle_pool import repack_b200, unrepack_b200  # noqa: F401 (re-exported)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
@@ -20,17 +21,6 @@ def rel_fro(a, b) -> float:
     b = np.asarray(b, np.float64)
     den = np.linalg.norm(b)
     return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
-
-
-def repack_b200(packed: np.ndarray) -> np.ndarray:
-    """Expected word layout of w4a8_prepare_experts_b200, from the header's definition:
-    nibble j of each word moves to nibble 2j (j < 4) or 2(j - 4) + 1 (j >= 4)."""
-    w = np.asarray(packed).view(np.uint32).astype(np.uint64)
-    r = np.zeros_like(w)
-    for j in range(8):
-        dst = 2 * j if j < 4 else 2 * (j - 4) + 1
-        r |= ((w >> np.uint64(4 * j)) & np.uint64(0xF)) << np.uint64(4 * dst)
-    return r.astype(np.uint32).view(np.int32).reshape(np.shape(packed))
 
 
 def e4m3_ordinal(codes: np.ndarray) -> np.ndarray:
@@ -72,3 +62,56 @@ def aux_buffers(T, H, I, E, k, device="cuda"):
         inter_scales=torch.empty(A, dtype=torch.float32, device=device),
         y_rows=torch.empty(A, H, dtype=torch.float32, device=device),
     )
+
+
+def assert_mse_clip_choice(packed: np.ndarray, scale_bits: np.ndarray, w: np.ndarray) -> int:
+    """Check a clip-search quantisation (the pages' word layout [R, K/8] and bf16
+    scale bits [R, K/128]) against the oracle's candidates for the float64
+    weights ``w`` [R, K].  Every group must hold one of its 11 candidates (codes
+    and scale); where that candidate is not the oracle's exact choice it must
+    be within the float64 summation bound of the least error (a near tie that
+    a different, equally valid, summation order may resolve the other way).
+    Returns the number of such groups."""
+    B = oracle.MSE_ERR_REL_BOUND
+    R, K = w.shape
+    G = K // 128
+    q_all, s_all, e_all = oracle.mse_clip_candidates(w)
+    q_o, s_o = oracle.mse_clip_quantize_int4(w)
+    q_g = oracle.unpack_uint4b8(packed).reshape(R, G, 128)
+    s_g = oracle.bf16_bits_to_f64(scale_bits).reshape(R, G)
+    same = (s_g == s_o) & np.all(q_g == q_o.reshape(R, G, 128), axis=2)
+    e_best = np.take_along_axis(e_all, np.argmin(e_all, axis=0)[None], axis=0)[0]
+    n_ties = 0
+    for r, g in zip(*np.nonzero(~same)):
+        match = [i for i in range(11) if s_all[i, r, g] == s_g[r, g]
+                 and np.array_equal(q_all[i, r].reshape(G, 128)[g], q_g[r, g])]
+        assert match, f"group ({r}, {g}) holds none of the 11 candidates"
+        i = match[0]
+        assert e_all[i, r, g] * (1 - B) <= e_best[r, g] * (1 + B), \
+            f"group ({r}, {g}): candidate {i} is not within the error bound of the minimum"
+        n_ties += 1
+    return n_ties
+
+
+
+TILE_WIDTHS = (32, 128)     # token rows per grouped-GEMM tile: decode and prefill shapes
+
+
+def boundary_rows(offsets: np.ndarray, n_segments: int = 3) -> np.ndarray:
+    """Segment rows on tile boundaries of the largest segments (the first and last row of
+    the first tile, a middle tile, the last full tile and the partial last tile,
+    for each tile width)."""
+    counts = np.diff(offsets.astype(np.int64))
+    rows = set()
+    for e in np.argsort(-counts, kind="stable")[:n_segments]:
+        lo, n = int(offsets[e]), int(counts[e])
+        if n == 0:
+            continue
+        for width in TILE_WIDTHS:
+            tiles = -(-n // width)
+            full = n // width
+            for t in {0, tiles // 2, max(full - 1, 0), tiles - 1}:
+                first = lo + t * width
+                last = min(lo + (t + 1) * width, lo + n) - 1
+                rows.update((first, last))
+    return np.array(sorted(rows), dtype=np.int64)

@@ -15,7 +15,8 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
-from gpu_helpers import aux_buffers, bf16_bits, codes_agree, f64, rel_fro, small_case, repack_b200
+from gpu_helpers import (assert_mse_clip_choice, aux_buffers, bf16_bits, codes_agree, f64,
+                         rel_fro, repack_b200, small_case, unrepack_b200)
 
 pytestmark = pytest.mark.gpu
 
@@ -39,9 +40,16 @@ def run_and_compare(cfg, hidden, logits, w13, w2, check_rows=None, mse_clip=Fals
     store = _store(w13, w2, mse_clip)
     res = oracle.moe_forward(f64(hidden), logits.numpy(), store, k)
 
-    # packed weights (bit-exact)
+    # packed weights (bit-exact; with the clip search, near ties within the
+    # float64 summation bound may take either tied candidate)
     for e in range(E):
         p13, s13, p2, s2 = store[e]
+        if mse_clip:
+            for wq, packed, scales in ((w13[e], layer.w13_packed[e], layer.w13_scales[e]),
+                                       (w2[e], layer.w2_packed[e], layer.w2_scales[e])):
+                assert_mse_clip_choice(unrepack_b200(packed.cpu().numpy()),
+                                       bf16_bits(scales.t()), f64(wq))
+            continue
         assert np.array_equal(layer.w13_packed[e].cpu().numpy(), repack_b200(p13))
         assert np.array_equal(bf16_bits(layer.w13_scales[e].t()), oracle.f64_to_bf16_bits(s13))
         assert np.array_equal(layer.w2_packed[e].cpu().numpy(), repack_b200(p2))

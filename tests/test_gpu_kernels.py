@@ -9,7 +9,7 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
-from gpu_helpers import bf16_bits, f64, repack_b200
+from gpu_helpers import assert_mse_clip_choice, bf16_bits, f64, repack_b200
 
 pytestmark = pytest.mark.gpu
 
@@ -42,9 +42,11 @@ def test_pack_int4_bit_exact(R, K):
 def test_pack_int4_mse_clip_bit_exact(R, K):
     wb = _weights(R, K, R * 977 + K)
     packed, scales = w4.w4a8_pack_int4(wb.cuda(), mse_clip=True)
-    q, s = oracle.mse_clip_quantize_int4(f64(wb))
-    assert np.array_equal(packed.cpu().numpy(), oracle.pack_uint4b8(q))
-    assert np.array_equal(bf16_bits(scales), oracle.f64_to_bf16_bits(s))
+    # the kernel sums each candidate's squared error in its own float64 order;
+    # it must hold the oracle's exact choice except at near ties within the
+    # summation bound, where either tied candidate is correct
+    n_ties = assert_mse_clip_choice(packed.cpu().numpy(), bf16_bits(scales), f64(wb))
+    print(f"\n[{R}x{K}] groups resolved differently at a near tie: {n_ties}")
 
 
 def test_pack_int4_3d_and_empty():
