@@ -51,6 +51,8 @@ typedef int32_t w4a8_status;
 #define W4A8_ERR_WORKSPACE_TOO_SMALL 4  /* workspace_bytes below the *_workspace_size value */
 #define W4A8_ERR_CUDA                5  /* a CUDA runtime call or launch failed */
 #define W4A8_ERR_DEVICE_TIMEOUT      6  /* a bounded in-kernel wait ran out (reported later) */
+#define W4A8_ERR_DEVICE_INDEX        7  /* an index read on the device was out of range; the
+                                           access was skipped (reported later) */
 
 /* Number of timed stages of w4a8_moe_forward (see w4a8_moe_aux.stage_events). */
 #define W4A8_NUM_STAGES 6
@@ -68,7 +70,9 @@ W4A8_API const char* w4a8_last_error(void);
  * w4a8_check_device_error - report and clear the device error latch.
  * Synchronises `stream`, then returns W4A8_ERR_DEVICE_TIMEOUT if any kernel of
  * this library on the current device gave up a bounded wait since the last
- * check, W4A8_ERR_CUDA if the stream holds a CUDA error, else W4A8_OK.
+ * check, W4A8_ERR_DEVICE_INDEX if a kernel found an index out of range (an
+ * expert id outside [-1, E) given to w4a8_moe_forward_experts) and skipped
+ * it, W4A8_ERR_CUDA if the stream holds a CUDA error, else W4A8_OK.
  */
 W4A8_API w4a8_status w4a8_check_device_error(void* stream);
 
@@ -119,6 +123,9 @@ W4A8_API w4a8_status w4a8_pack_int4(const void* w_bf16, int64_t R, int64_t K, in
  *         pairwise combinations of the 32 partial sums (element index xor 16,
  *         8, 4, 2, 1 runs);
  * and the smallest i with the least e_i is kept (i = 0 is w4a8_pack_int4).
+ * Each e_i is within 2^-45 e_i of the exact squared error, so the kept
+ * candidate is the exact MSE minimiser unless two candidates' exact errors
+ * lie within that bound of each other (a near tie, where either is kept).
  * With r < 1 the code -8 occurs.  Arguments and errors as w4a8_pack_int4.
  */
 W4A8_API w4a8_status w4a8_pack_int4_mse_clip(const void* w_bf16, int64_t R, int64_t K,
@@ -208,12 +215,11 @@ W4A8_API w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int3
  * (The pages have no counterpart: this is a calling convention of this
  * library, not a step of the method.)
  *
- * Why: some callers may not call cudaMalloc where they route tokens - code
- * running while a CUDA graph is being captured (an allocation there breaks
- * the capture or is not replayed), runtimes and plugin interfaces that give a
- * kernel only its planned inputs and outputs and no scratch, and paths whose
- * device memory budget is fixed in advance.  This call takes no workspace and
- * calls no cudaMalloc, cudaFree or other allocating routine.
+ * Why: some callers may not call cudaMalloc where they route tokens -
+ * runtimes and plugin interfaces that give a kernel only its planned inputs
+ * and outputs and no scratch, and paths whose device memory budget is fixed in
+ * advance.  This call takes no workspace and calls no cudaMalloc, cudaFree or
+ * other allocating routine.
  *
  * Scratch: a file-scope device array of 528,388 bytes (2 * 65536 + 1025
  * int32) that every device which loads the library holds until the process
@@ -221,7 +227,9 @@ W4A8_API w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int3
  * E = 256, or T <= 16384 with E = 1024); larger problems get
  * W4A8_ERR_UNSUPPORTED_SHAPE and should use w4a8_moe_route_permute.
  * Set-up: the first call on each device looks up the array's device address
- * with that device current; make that first call before any stream capture.
+ * with that device current and keeps it; make that first call before any
+ * stream capture.  cudaDeviceReset discards the array, so after a reset of a
+ * device the kept address is stale and this call must not be used on it.
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents.  The histogram part is zeroed by each call on `stream`
  * and the rest is rewritten before it is read, but calls that overlap on the
@@ -448,6 +456,80 @@ W4A8_API w4a8_status w4a8_moe_forward_shared(
     const float* ws2_scales, int64_t T, int64_t H, int64_t I, int64_t I_shared, int32_t E,
     int32_t k, void* out_bf16, void* workspace, size_t workspace_bytes, const w4a8_moe_aux* aux,
     const w4a8_shared_aux* shared_aux, void* stream);
+
+/*
+ * Expert parallelism: the layer split by expert over G ranks (GLM-5.3-W4A8
+ * model card, "performance" table: TP8+EP and 2 x (TP4+EP); "deployment": the
+ * W4A8 checkpoint must run with expert parallelism).  Rank g owns a contiguous
+ * range of experts.  One step: every rank quantises its own tokens
+ * (w4a8_quant_act_fp8_per_token) and routes them (w4a8_moe_route_topk); the
+ * ranks all-gather the E4M3 codes, token scales, expert ids and weights (the
+ * dispatch); each rank runs w4a8_moe_forward_experts on the gathered tokens
+ * for its own experts, giving float32 partial sums; the ranks reduce-scatter
+ * (sum) the partial sums back to the tokens' owners (the combine), and each
+ * rounds its tokens once to bf16 (w4a8_cast_f32_bf16).  The collectives are
+ * the caller's (NCCL); these calls only compute.
+ */
+
+/*
+ * w4a8_moe_route_topk - the top-k step of w4a8_moe_route_permute alone: the
+ * same ids (ties to the lower expert id) and softmax-renormalised weights,
+ * without the permutation.  Arguments and errors as w4a8_moe_route_permute;
+ * no workspace.
+ */
+W4A8_API w4a8_status w4a8_moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
+                                         int32_t* topk_ids, float* topk_w, void* stream);
+
+/*
+ * w4a8_moe_experts_workspace_size - bytes of scratch w4a8_moe_forward_experts
+ * needs for T (gathered) tokens and e_count local experts.
+ */
+W4A8_API size_t w4a8_moe_experts_workspace_size(int64_t T, int64_t H, int64_t I,
+                                                int32_t e_count, int32_t k);
+
+/*
+ * w4a8_moe_forward_experts - steps 3-6 of w4a8_moe_forward for the experts
+ * e_begin .. e_begin + e_count - 1 only, from activations already quantised
+ * and tokens already routed; the combine writes float32 sums instead of bf16:
+ *
+ *   partial_out[t] = sum over the slots j of token t whose expert is local,
+ *                    in slot order, of topk_w[t, j] * Y[t, j]
+ *
+ * (0 for a token with no local slot).  Summed over ranks whose ranges cover
+ * [0, E) and rounded to bf16, this is w4a8_moe_forward's output up to the
+ * float32 summation order.  The permutation is the stable counting sort of
+ * w4a8_moe_route_permute restricted to the local experts.
+ *
+ *   act_codes     [T, H] uint8 E4M3 codes (w4a8_quant_act_fp8_per_token)
+ *   act_scales    [T] float32 token scales
+ *   topk_ids      [T, k] int32 expert ids in [0, E), or -1 for an empty
+ *                 slot (a padding token); any other id sets the device latch
+ *                 (W4A8_ERR_DEVICE_INDEX at the next w4a8_check_device_error)
+ *                 and its slot is skipped
+ *   topk_w        [T, k] float32 routing weights
+ *   T, H, I, E, k as w4a8_moe_forward (T = all ranks' tokens)
+ *   e_begin, e_count  0 <= e_begin, 1 <= e_count, e_begin + e_count <= E
+ *   w13_packed, w13_scales, w2_packed, w2_scales
+ *                 the LOCAL experts only, laid out as for w4a8_moe_forward
+ *                 ([e_count, 2I, H / 8], [e_count, H / 128, 2I], ...)
+ *   partial_out   [T, H] float32, written
+ *   workspace     >= w4a8_moe_experts_workspace_size(T, H, I, e_count, k) bytes
+ */
+W4A8_API w4a8_status w4a8_moe_forward_experts(
+    const uint8_t* act_codes, const float* act_scales, const int32_t* topk_ids,
+    const float* topk_w, int64_t T, int64_t H, int64_t I, int32_t E, int32_t k, int32_t e_begin,
+    int32_t e_count, const int32_t* w13_packed, const void* w13_scales, const int32_t* w2_packed,
+    const void* w2_scales, float* partial_out, void* workspace, size_t workspace_bytes,
+    void* stream);
+
+/*
+ * w4a8_cast_f32_bf16 - out = bf16(x), round to nearest even: the single bf16
+ * rounding of the expert-parallel combine, after the partial sums are reduced.
+ *
+ *   x         [n] float32;  n >= 0, n % 8 == 0 (0: no-op)
+ *   out_bf16  [n] bf16, written
+ */
+W4A8_API w4a8_status w4a8_cast_f32_bf16(const float* x, int64_t n, void* out_bf16, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

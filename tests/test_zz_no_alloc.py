@@ -1,6 +1,6 @@
 """w4a8_moe_route_permute_noalloc, the routing entry point for callers that
-cannot allocate device memory when they route (graph capture, plugin
-interfaces that pass only planned buffers, fixed memory budgets).  It keeps
+cannot allocate device memory when they route (plugin interfaces that pass
+only planned buffers, fixed device memory budgets).  It keeps
 its scratch in a static device array instead of a caller workspace; its
 outputs must equal those of w4a8_moe_route_permute, on consecutive calls that
 reuse the same scratch.

@@ -20,7 +20,9 @@ __all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_ab
            "w4a8_moe_route_permute_noalloc", "w4a8_moe_workspace_size",
            "w4a8_moe_forward", "w4a8_check_device_error", "W4A8MoELayer",
            "w4a8_quant_fp8_block", "w4a8_quant_act_fp8_group", "w4a8_shared_expert_forward",
-           "w4a8_moe_forward_shared", "SharedExpertFP8", "SHARED_STAGE_NAMES"]
+           "w4a8_moe_forward_shared", "SharedExpertFP8", "SHARED_STAGE_NAMES",
+           "w4a8_moe_route_topk", "w4a8_moe_experts_workspace_size", "w4a8_moe_forward_experts",
+           "w4a8_cast_f32_bf16"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a8.so")
 NUM_STAGES = 6
@@ -85,6 +87,11 @@ def _declare(L):
         "w4a8_moe_shared_workspace_size": (sz, [i64, i64, i64, i32, i32, i64]),
         "w4a8_moe_forward_shared": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
                                           i64, i32, i32, vp, vp, sz, vp, vp, vp]),
+        "w4a8_moe_route_topk": (i32, [vp, i64, i32, i32, vp, vp, vp]),
+        "w4a8_moe_experts_workspace_size": (sz, [i64, i64, i64, i32, i32]),
+        "w4a8_moe_forward_experts": (i32, [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
+                                           vp, vp, vp, vp, vp, vp, sz, vp]),
+        "w4a8_cast_f32_bf16": (i32, [vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -646,3 +653,88 @@ class W4A8MoELayerShared(W4A8MoELayer):
                                        self.w2_packed, self.w2_scales, self.shared.weights,
                                        self.k, out=out, workspace=self.workspace(hidden.shape[0]),
                                        **kw)
+
+
+# ---------------------------------------------------------------- expert parallelism
+
+def w4a8_moe_route_topk(logits: torch.Tensor, k: int, topk_ids: Optional[torch.Tensor] = None,
+                        topk_w: Optional[torch.Tensor] = None):
+    """Top-k ids and softmax-renormalised weights only: (int32 [T, k], float32 [T, k])."""
+    _need(logits, "logits", torch.float32, 2)
+    T, E = logits.shape
+    dev = logits.device
+    if topk_ids is None:
+        topk_ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    _need(topk_ids, "topk_ids", torch.int32, 2)
+    _need(topk_w, "topk_w", torch.float32, 2)
+    if topk_ids.shape != (T, k) or topk_w.shape != (T, k):
+        raise ValueError("topk_ids / topk_w must be [T, k]")
+    _check("w4a8_moe_route_topk",
+           lib().w4a8_moe_route_topk(_p(logits), T, E, k, _p(topk_ids), _p(topk_w),
+                                     _stream(dev)))
+    return topk_ids, topk_w
+
+
+def w4a8_moe_experts_workspace_size(T: int, H: int, I: int, e_count: int, k: int) -> int:
+    return int(lib().w4a8_moe_experts_workspace_size(T, H, I, e_count, k))
+
+
+def w4a8_moe_forward_experts(act_codes: torch.Tensor, act_scales: torch.Tensor,
+                             topk_ids: torch.Tensor, topk_w: torch.Tensor, E: int, e_begin: int,
+                             w13_packed: torch.Tensor, w13_scales: torch.Tensor,
+                             w2_packed: torch.Tensor, w2_scales: torch.Tensor,
+                             out: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The local experts' share of the layer (expert parallelism): float32
+    partial sums [T, H] over the slots routed to experts e_begin ..
+    e_begin + e_count - 1, whose prepared weights ``w13_*`` / ``w2_*`` hold
+    those experts only (see include/w4a8.h)."""
+    _need(act_codes, "act_codes", torch.uint8, 2)
+    _need(act_scales, "act_scales", torch.float32, 1)
+    _need(topk_ids, "topk_ids", torch.int32, 2)
+    _need(topk_w, "topk_w", torch.float32, 2)
+    _need(w13_packed, "w13_packed", torch.int32, 3)
+    _need(w13_scales, "w13_scales", torch.bfloat16, 3)
+    _need(w2_packed, "w2_packed", torch.int32, 3)
+    _need(w2_scales, "w2_scales", torch.bfloat16, 3)
+    T, H = act_codes.shape
+    k = topk_ids.shape[1]
+    e_count = w13_packed.shape[0]
+    I = w2_packed.shape[2] * 8
+    if act_scales.shape != (T,) or topk_ids.shape[0] != T or topk_w.shape != (T, k) or \
+            w13_packed.shape != (e_count, 2 * I, H // 8) or \
+            w2_packed.shape != (e_count, H, I // 8) or \
+            w13_scales.shape != (e_count, H // 128, 2 * I) or \
+            w2_scales.shape != (e_count, I // 128, H):
+        raise ValueError("inconsistent shapes: codes [T,H], scales [T], ids/w [T,k], local "
+                         "w13 [e,2I,H/8], w2 [e,H,I/8], scales group-major")
+    dev = act_codes.device
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, 2)
+    need = w4a8_moe_experts_workspace_size(T, H, I, e_count, k)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("w4a8_moe_forward_experts",
+           lib().w4a8_moe_forward_experts(
+               _p(act_codes), _p(act_scales), _p(topk_ids), _p(topk_w), T, H, I, E, k, e_begin,
+               e_count, _p(w13_packed), _p(w13_scales), _p(w2_packed), _p(w2_scales), _p(out),
+               _p(workspace), workspace.numel(), _stream(dev)))
+    return out
+
+
+def w4a8_cast_f32_bf16(x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """bf16 copy of float32 ``x`` (round to nearest even); numel % 8 == 0."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.float32 or \
+            not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    if out.shape != x.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or \
+            not out.is_cuda:
+        raise ValueError("out must be a contiguous bf16 CUDA tensor of x's shape")
+    _check("w4a8_cast_f32_bf16",
+           lib().w4a8_cast_f32_bf16(_p(x), x.numel(), _p(out), _stream(x.device)))
+    return out

@@ -296,6 +296,7 @@ const char* w4a8_status_string(w4a8_status s) {
     case W4A8_ERR_WORKSPACE_TOO_SMALL: return "W4A8_ERR_WORKSPACE_TOO_SMALL";
     case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
     case W4A8_ERR_DEVICE_TIMEOUT: return "W4A8_ERR_DEVICE_TIMEOUT";
+    case W4A8_ERR_DEVICE_INDEX: return "W4A8_ERR_DEVICE_INDEX";
     default: return "W4A8_ERR_UNKNOWN";
   }
 }
@@ -308,8 +309,12 @@ w4a8_status w4a8_check_device_error(void* stream) {
   int v = 0;
   err = read_and_clear_device_error(&v);
   if (err != cudaSuccess) return cuda_fail(err, "reading the device error latch");
-  if (v != 0)
+  if (v & kDeviceErrorTimeout)
     return fail(W4A8_ERR_DEVICE_TIMEOUT, "a bounded in-kernel wait ran out (latch 0x%x)", v);
+  if (v & kDeviceErrorIndex)
+    return fail(W4A8_ERR_DEVICE_INDEX,
+                "an index read on the device was out of range; the access was skipped (latch 0x%x)",
+                v);
   return W4A8_OK;
 }
 
@@ -922,6 +927,186 @@ w4a8_status w4a8_moe_forward_shared(const void* hidden_bf16, const float* logits
   return moe_forward_impl(hidden_bf16, logits, w13_packed, w13_scales, w2_packed, w2_scales, T, H,
                           I, E, k, out_bf16, workspace, workspace_bytes, aux, stream, nullptr,
                           &sh);
+}
+
+// ---------------------------------------------------------------- expert parallelism
+
+w4a8_status w4a8_moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
+                                int32_t* topk_ids, float* topk_w, void* stream) {
+  if (w4a8_status st = check_route_args(logits, T, E, k)) return st;
+  if (T == 0) return W4A8_OK;
+  if (!topk_ids || !topk_w) return fail(W4A8_ERR_INVALID_ARG, "NULL output pointer");
+  if (!aligned16(topk_ids) || !aligned16(topk_w))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_route_topk(logits, T, E, k, topk_ids, topk_w,
+                                      static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "route_topk launch");
+}
+
+size_t w4a8_moe_experts_workspace_size(int64_t T, int64_t H, int64_t I, int32_t e_count,
+                                       int32_t k) {
+  if (T < 0 || H <= 0 || I <= 0 || e_count < 1 || k < 1) return 0;
+  Carver c(nullptr);
+  carve_forward(c, T, H, I, e_count, k);
+  return c.off + 256;
+}
+
+w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_scales,
+                                     const int32_t* topk_ids, const float* topk_w, int64_t T,
+                                     int64_t H, int64_t I, int32_t E, int32_t k,
+                                     int32_t e_begin, int32_t e_count,
+                                     const int32_t* w13_packed, const void* w13_scales,
+                                     const int32_t* w2_packed, const void* w2_scales,
+                                     float* partial_out, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (T < 0) return fail(W4A8_ERR_INVALID_ARG, "T = %lld < 0", static_cast<long long>(T));
+  if (E < 1 || E > kMaxExperts)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "E = %d outside [1, %d]", E, kMaxExperts);
+  if (k < 1 || k > E || k > kMaxTopK)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "k = %d outside [1, min(E, %d)]", k, kMaxTopK);
+  if (e_begin < 0 || e_count < 1 || e_begin + static_cast<int64_t>(e_count) > E)
+    return fail(W4A8_ERR_INVALID_ARG, "expert range [%d, %d + %d) is not inside [0, %d)", e_begin,
+                e_begin, e_count, E);
+  if (T * static_cast<int64_t>(k) > INT32_MAX)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "T * k exceeds 2^31 - 1");
+  if (H <= 0 || I <= 0 || H % kGroup || I % kGroup)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld and I = %lld must be positive multiples of 128",
+                static_cast<long long>(H), static_cast<long long>(I));
+  if (H / kGroup > kMaxGroups || I / kGroup > kMaxGroups)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld, I = %lld: at most %d groups of 128 per row",
+                static_cast<long long>(H), static_cast<long long>(I), kMaxGroups);
+  if (static_cast<int64_t>(e_count) * 2 * I > INT32_MAX || static_cast<int64_t>(e_count) * H > INT32_MAX)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "e_count * rows exceeds 2^31 - 1");
+  if (T == 0) return W4A8_OK;
+  const void* ptrs[] = {act_codes, act_scales, topk_ids, topk_w, w13_packed, w13_scales,
+                        w2_packed, w2_scales, partial_out, workspace};
+  for (const void* p : ptrs) {
+    if (!p) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+    if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  }
+  const size_t need = w4a8_moe_experts_workspace_size(T, H, I, e_count, k);
+  if (workspace_bytes < need)
+    return fail(W4A8_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu", workspace_bytes, need);
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  int* latch = nullptr;
+  if (cudaError_t err = device_error_latch(&latch)) return cuda_fail(err, "device error latch");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  Carver c(workspace);
+  ForwardBufs b = carve_forward(c, T, H, I, e_count, k);
+  const int64_t A = T * k;   // rows of the buffers: every slot could be local
+  // the shape by the expected local load, which is the whole layer's per-expert load
+  const bool decode = A <= static_cast<int64_t>(kDecodeTokensPerExpert) * E;
+  const int tile_n = grouped_gemm_tile_n(decode);
+  const bool parts = grouped_gemm_uses_sum_parts(decode);
+
+  CUtensorMap tw1, ta1, tw2, ta2, ts1, ts2, tg1, tg2;
+  if (w4a8_status st = encode_u8_2d(&tw1, w13_packed, static_cast<uint64_t>(H / 2),
+                                    static_cast<uint64_t>(e_count) * 2 * I, 64, 64,
+                                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ta1, b.perm_codes, static_cast<uint64_t>(H),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&tw2, w2_packed, static_cast<uint64_t>(I / 2),
+                                    static_cast<uint64_t>(e_count) * H, 64, 128,
+                                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ta2, b.inter_codes, static_cast<uint64_t>(I),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&tg1, b.act_parts, static_cast<uint64_t>(2 * sum_parts_ld(H)),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&tg2, b.inter_parts,
+                                    static_cast<uint64_t>(2 * sum_parts_ld(I)),
+                                    static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ts1, w13_scales, static_cast<uint64_t>(2 * I) * 2,
+                                    static_cast<uint64_t>(e_count) * (H / kGroup), 128,
+                                    static_cast<uint32_t>(H / kGroup), CU_TENSOR_MAP_SWIZZLE_NONE))
+    return st;
+  if (w4a8_status st = encode_u8_2d(&ts2, w2_scales, static_cast<uint64_t>(H) * 2,
+                                    static_cast<uint64_t>(e_count) * (I / kGroup), 256,
+                                    static_cast<uint32_t>(I / kGroup), CU_TENSOR_MAP_SWIZZLE_NONE))
+    return st;
+
+  cudaError_t err = cudaSuccess;
+#define W4A8_STEP(call, what)                              \
+  do {                                                     \
+    err = (call);                                          \
+    if (err != cudaSuccess) return cuda_fail(err, what);   \
+  } while (0)
+  // the local experts' segments of all T tokens; rows_total = expert_offsets[e_count]
+  W4A8_STEP(launch_route_local(topk_ids, T, E, k, e_begin, e_count, b.expert_offsets,
+                               b.sorted_token_ids, b.row_of, b.route.block_counts,
+                               b.route.block_base, b.route.tile_prefix, tile_n, b.row_amax, latch,
+                               di.sms, s),
+            "local routing launch");
+  const int32_t* rows_total = b.expert_offsets + e_count;
+  W4A8_STEP(launch_ep_gather(act_codes, H, b.sorted_token_ids, rows_total, A, b.perm_codes,
+                             parts ? nullptr : b.act_gsum, parts ? b.act_parts : nullptr, di.sms, s),
+            "dispatch gather launch");
+
+  GemmArgs g1{};
+  g1.K = static_cast<int>(H);
+  g1.n_rows = static_cast<int>(2 * I);
+  g1.half_rows = static_cast<int>(I);
+  g1.E = e_count;
+  g1.expert_offsets = b.expert_offsets;
+  g1.tile_prefix = b.route.tile_prefix;
+  g1.row_tokens = b.sorted_token_ids;
+  g1.act_scale = act_scales;
+  g1.act_gsum = b.act_gsum;
+  g1.wscale = w13_scales;
+  g1.out = b.h;
+  g1.out_ld = I;
+  g1.row_amax = b.row_amax;
+  g1.act_rows = T;
+  g1.timeout_ns = wait_timeout_ns();
+  g1.nb_fastest = tile_order_nb_fastest(decode);
+  W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
+            "gate/up GEMM launch");
+  W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales,
+                               parts ? nullptr : b.inter_gsum, di.sms, s, nullptr,
+                               parts ? b.inter_parts : nullptr, rows_total),
+            "intermediate quant launch");
+  GemmArgs g2 = g1;
+  g2.K = static_cast<int>(I);
+  g2.n_rows = static_cast<int>(H);
+  g2.half_rows = 0;
+  g2.row_tokens = nullptr;
+  g2.act_scale = b.inter_scales;
+  g2.act_gsum = b.inter_gsum;
+  g2.wscale = w2_scales;
+  g2.out = b.y;
+  g2.out_ld = H;
+  g2.row_amax = nullptr;
+  g2.act_rows = A;
+  W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),
+            "down GEMM launch");
+  W4A8_STEP(launch_combine(b.y, b.row_of, topk_w, T, H, k, nullptr, di.sms, s, nullptr,
+                           partial_out),
+            "partial combine launch");
+#undef W4A8_STEP
+  return W4A8_OK;
+}
+
+w4a8_status w4a8_cast_f32_bf16(const float* x, int64_t n, void* out_bf16, void* stream) {
+  if (n < 0) return fail(W4A8_ERR_INVALID_ARG, "n = %lld < 0", static_cast<long long>(n));
+  if (n % 8) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "n = %lld is not a multiple of 8",
+                         static_cast<long long>(n));
+  if (n == 0) return W4A8_OK;
+  if (!x || !out_bf16) return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(x) || !aligned16(out_bf16))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_cast_bf16(x, n, out_bf16, di.sms, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "cast launch");
 }
 
 }  // extern "C"

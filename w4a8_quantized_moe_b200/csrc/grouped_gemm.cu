@@ -71,6 +71,7 @@
 #include <cstdlib>
 
 #include "internal.h"
+#define W4A8_OWNS_DEVICE_ERROR_LATCH 1
 #include "ptx.cuh"
 
 namespace w4a8 {
@@ -1200,6 +1201,10 @@ cudaError_t launch_fp8_block_gemm(bool gate_up, const CUtensorMap& tmap_w,
                                                             num_ctas, s)
                  : launch_shape<F8Block, false, false, true>(tmap_w, tmap_act, tmap_w, tmap_act,
                                                              a, num_ctas, s);
+}
+
+cudaError_t device_error_latch(int** latch) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(latch), g_device_error);
 }
 
 cudaError_t read_and_clear_device_error(int* value) {

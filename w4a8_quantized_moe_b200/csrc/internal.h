@@ -16,6 +16,10 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxGroups = 64;     // K / 128 per GEMM (K <= 8192)
 
+// Bits of the device error latch.
+constexpr int kDeviceErrorTimeout = 1;  // a bounded in-kernel wait ran out
+constexpr int kDeviceErrorIndex = 2;    // an index was out of range (the access was skipped)
+
 inline int64_t route_blocks(int64_t T) { return (T + kRouteTok - 1) / kRouteTok; }
 // Three-part group sums (per-tile offset correction): one part spans Gp =
 // K / 128 groups rounded up to 16 columns; a row holds the three parts and is
@@ -48,11 +52,33 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                          int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
                          cudaStream_t s);
+// Top-k and weights only (no histogram, no permutation).
+cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
+                              float* topk_w, cudaStream_t s);
+// Expert parallelism: the permutation of given ids restricted to the E_loc
+// experts e_lo .. e_lo + E_loc - 1 of E_all (segments, offsets and tile prefix
+// over the local experts only; row_of = -1 for other experts' slots).  Ids
+// outside [-1, E_all) set kDeviceErrorIndex in *latch and are skipped.
+cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, int k, int e_lo,
+                               int E_loc, int32_t* expert_offsets, int32_t* sorted_token_ids,
+                               int32_t* row_of, int32_t* block_counts, int32_t* block_base,
+                               int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
+                               int* latch, int num_sms, cudaStream_t s);
+// Segment row r < *rows_total (device) receives the codes of token
+// sorted_token_ids[r]; the group sums go to gsum [T, H / 128] by token, or to
+// the row's three-part sums (sum_parts, [max_rows, sum_parts_ld(H)]).
+cudaError_t launch_ep_gather(const uint8_t* codes, int64_t H, const int32_t* sorted_token_ids,
+                             const int32_t* rows_total, int64_t max_rows, uint8_t* perm,
+                             float* gsum, uint16_t* sum_parts, int num_sms, cudaStream_t s);
+// bf16 = round-to-nearest-even(x), n a multiple of 8.
+cudaError_t launch_cast_bf16(const float* x, int64_t n, void* out, int num_sms, cudaStream_t s);
 // sum_parts (nullable): [A, sum_parts_ld(I)] bf16 as for launch_act_quant.
+// rows_dev (nullable): device-side row count (min with A) when only the
+// device knows it.
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, float* gsum, int num_sms,
                                cudaStream_t s, int32_t* int8_row_sum = nullptr,
-                               uint16_t* sum_parts = nullptr);
+                               uint16_t* sum_parts = nullptr, const int32_t* rows_dev = nullptr);
 // packed uint4b8 words -> the word-local nibble interleave the grouped GEMM reads.
 cudaError_t launch_repack_int4_b200(const int32_t* in, int64_t nwords, int32_t* out, int num_sms,
                                     cudaStream_t s);
@@ -66,9 +92,11 @@ cudaError_t launch_pack_int4_channel(const void* w, int64_t R, int64_t K, int32_
 cudaError_t launch_nibble_row_sum(const int32_t* packed, int64_t R, int64_t words_per_row,
                                   int32_t* sums, int num_sms, cudaStream_t s);
 // y_shared (nullable): [T, H] float32 added to each token's routed sum.
+// partial_f32 (nullable): write the float32 sum over the slots with a row
+// (row_of >= 0) there instead of the bf16 output (expert parallelism).
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
                            int64_t H, int k, void* out, int num_sms, cudaStream_t s,
-                           const float* y_shared = nullptr);
+                           const float* y_shared = nullptr, float* partial_f32 = nullptr);
 // FP8 block weights: bf16 [R, K] -> E4M3 codes [R, K] + float32 scales
 // [R / 128, K / 128], scale = absmax / 448 per 128 x 128 block.
 cudaError_t launch_quant_fp8_block(const void* w, int64_t R, int64_t K, uint8_t* codes,
@@ -133,5 +161,9 @@ cudaError_t launch_fp8_block_gemm(bool gate_up, const CUtensorMap& tmap_w,
                                   cudaStream_t s);
 // One bounded wait on an mbarrier nothing arrives on (failure-detection self-test).
 cudaError_t launch_wait_timeout_selftest(uint64_t timeout_ns, cudaStream_t s);
+// Device address (current device) of the library's one error latch, for
+// kernels outside grouped_gemm.cu: they atomicOr kDeviceErrorIndex into it.
+// w4a8_check_device_error() reads and clears it.
+cudaError_t device_error_latch(int** latch);
 
 }  // namespace w4a8

@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;  // warp-uniform
   const float* lt = logits + t * E;
-  int32_t* counts = block_counts + (t / kRouteTok) * E;
+  int32_t* counts = block_counts ? block_counts + (t / kRouteTok) * E : nullptr;
   float v[NV];
   uint32_t taken = 0;
 #pragma unroll
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     if (lane == j) {
       myv = bv;
       topk_ids[t * k + j] = bi;
-      atomicAdd(counts + bi, 1);
+      if (block_counts) atomicAdd(counts + bi, 1);
     }
     if (j == 0) v0 = bv;
   }
@@ -479,8 +479,11 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
 // bits below it in its own chunk's mask.
 constexpr int kScatterWarps = kRouteTok / 32;
 
+// Only experts e_lo .. e_lo + E - 1 get segments (E = the segment count; the
+// whole layer passes e_lo = 0): an assignment to any other expert gets
+// row_of = -1 and no row (expert parallelism: the experts of other ranks).
 __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
-    const int32_t* __restrict__ topk_ids, int64_t T, int E, int k,
+    const int32_t* __restrict__ topk_ids, int64_t T, int E, int k, int e_lo,
     const int32_t* __restrict__ block_base, int32_t* __restrict__ sorted_token_ids,
     int32_t* __restrict__ row_of, uint32_t* __restrict__ row_amax) {
   extern __shared__ uint32_t mask[];  // [kScatterWarps][E]
@@ -491,10 +494,12 @@ __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
   const bool valid = t < T;
   int ids[kMaxTopK];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) ids[j] = (valid && j < k) ? __ldg(topk_ids + t * k + j) : 0;
+  for (int j = 0; j < kMaxTopK; ++j)
+    ids[j] = (valid && j < k) ? __ldg(topk_ids + t * k + j) - e_lo : -1;
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j)
-    if (valid && j < k) atomicOr(&mask[warp * E + ids[j]], 1u << lane);
+    if (static_cast<unsigned>(ids[j]) < static_cast<unsigned>(E))
+      atomicOr(&mask[warp * E + ids[j]], 1u << lane);
   __syncthreads();
   const uint32_t lt_mask = (1u << lane) - 1u;
   const int32_t* base = block_base + static_cast<int64_t>(blockIdx.x) * E;
@@ -502,6 +507,10 @@ __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
   for (int j = 0; j < kMaxTopK; ++j) {
     if (valid && j < k) {
       const int e = ids[j];
+      if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
+        row_of[t * k + j] = -1;
+        continue;
+      }
       int rank = __popc(mask[warp * E + e] & lt_mask);
       for (int w = 0; w < warp; ++w) rank += __popc(mask[w * E + e]);
       const int row = base[e] + rank;
@@ -509,6 +518,90 @@ __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
       sorted_token_ids[row] = static_cast<int32_t>(t);
       if (row_amax) row_amax[row] = 0u;
     }
+  }
+}
+
+// Histogram of given expert ids for the experts e_lo .. e_lo + E_loc - 1 into
+// block_counts[token / kRouteTok][e - e_lo] (thread per assignment; the
+// launcher zeroes the counts).  An id outside [0, E_all) other than -1 (no
+// expert) is a caller error: it raises the device latch's index bit and is
+// left out.
+__global__ void __launch_bounds__(256) route_ids_hist_kernel(const int32_t* __restrict__ topk_ids,
+                                                             int64_t T, int k, int E_all, int e_lo,
+                                                             int E_loc,
+                                                             int32_t* __restrict__ block_counts,
+                                                             int* __restrict__ latch) {
+  const int64_t n = T * k;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int e = __ldg(topk_ids + i);
+    if (e < -1 || e >= E_all) {
+      atomicOr(latch, kDeviceErrorIndex);
+      continue;
+    }
+    const int le = e - e_lo;
+    if (e >= 0 && static_cast<unsigned>(le) < static_cast<unsigned>(E_loc))
+      atomicAdd(block_counts + (i / k / kRouteTok) * E_loc + le, 1);
+  }
+}
+
+// Expert-parallel dispatch: segment row r (r < expert_offsets[E_loc], read on
+// the device) receives the E4M3 codes of token sorted_token_ids[r]; the sums
+// of the E4M3 values of its 128-wide groups go to gsum [T, H / 128] (by token;
+// several rows of one token write the same values) or, for the shapes that
+// remove the nibble offset once per tile, to the row's three bf16 parts.
+// One warp per row, 16 bytes per lane per step.
+__global__ void __launch_bounds__(256) ep_gather_kernel(const uint8_t* __restrict__ codes,
+                                                        int64_t H,
+                                                        const int32_t* __restrict__ sorted_token_ids,
+                                                        const int32_t* __restrict__ rows_total,
+                                                        uint8_t* __restrict__ perm,
+                                                        float* __restrict__ gsum,
+                                                        uint16_t* __restrict__ parts) {
+  const int lane = threadIdx.x & 31;
+  const int64_t A = __ldg(rows_total);
+  const int64_t nchunk = H / 16;                 // 16-byte chunks; 8 per 128-wide group
+  const int G = static_cast<int>(H / kGroup);
+  const int gp = (G + 15) / 16 * 16;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < A;
+       r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t t = __ldg(sorted_token_ids + r);
+    const uint4* src = reinterpret_cast<const uint4*>(codes + t * H);
+    uint4* dst = reinterpret_cast<uint4*>(perm + r * H);
+    for (int64_t base = 0; base < nchunk; base += 32) {   // warp-uniform trip count
+      const int64_t c = base + lane;
+      float part = 0.0f;
+      if (c < nchunk) {
+        const uint4 v = __ldg(src + c);
+        dst[c] = v;
+        part = sum8_e4m3(make_uint2(v.x, v.y)) + sum8_e4m3(make_uint2(v.z, v.w));
+      }
+      part += __shfl_xor_sync(kFull, part, 4);
+      part += __shfl_xor_sync(kFull, part, 2);
+      part += __shfl_xor_sync(kFull, part, 1);
+      if (c < nchunk && (c & 7) == 0) {
+        if (gsum) gsum[t * G + (c >> 3)] = part;
+        if (parts) store_sum_parts(parts + r * sum_parts_ld(H), part, static_cast<int>(c >> 3), G, gp);
+      }
+    }
+  }
+}
+
+// float32 -> bf16, round to nearest even, 8 values per thread.
+__global__ void __launch_bounds__(256) cast_bf16_kernel(const float* __restrict__ x, int64_t n8,
+                                                        __nv_bfloat16* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(x) + 2 * i);
+    const float4 b = __ldg(reinterpret_cast<const float4*>(x) + 2 * i + 1);
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t p[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+      p[q] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    reinterpret_cast<uint4*>(out)[i] = make_uint4(p[0], p[1], p[2], p[3]);
   }
 }
 
@@ -525,11 +618,16 @@ __global__ void __launch_bounds__(256) inter_quant_kernel(const float* __restric
                                                           float* __restrict__ scales,
                                                           float* __restrict__ gsum,
                                                           int32_t* __restrict__ row_sum,
-                                                          uint16_t* __restrict__ parts) {
+                                                          uint16_t* __restrict__ parts,
+                                                          const int32_t* __restrict__ rows_dev) {
   const int64_t per_row = I / 16;
   const bool want_sums = !kInt8 && (gsum || parts);
   const int G = static_cast<int>(I / kGroup);
   const int gp = (G + 15) / 16 * 16;
+  if (rows_dev) {  // the row count is known only on the device (expert parallelism)
+    const int64_t a_dev = __ldg(rows_dev);
+    A = a_dev < A ? a_dev : A;
+  }
   const int64_t n = A * per_row;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t n_iter = (n + stride - 1) / stride;
@@ -691,12 +789,16 @@ __global__ void __launch_bounds__(256) transpose_scales_kernel(const uint16_t* _
 
 // ---------------------------------------------------------------- combine
 // out[t, c..c+7] = bf16(sum_j w[t, j] * Y[row_of[t, j], c..c+7]) in slot order.
+// kPartial: the float32 sum over the slots with a row (row_of >= 0: this
+// rank's experts) instead, for the expert-parallel combine.
+template <bool kPartial>
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y,
                                                       const int32_t* __restrict__ row_of,
                                                       const float* __restrict__ topk_w, int64_t T,
                                                       int64_t H, int k,
                                                       const float* __restrict__ y_shared,
-                                                      __nv_bfloat16* __restrict__ out) {
+                                                      __nv_bfloat16* __restrict__ out,
+                                                      float* __restrict__ out_f32) {
   const int64_t per_row = H / 8;
   const int64_t n = T * per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -705,6 +807,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < k; ++j) {
       const int64_t r = __ldg(row_of + t * k + j);
+      if (kPartial && r < 0) continue;
       const float wj = __ldg(topk_w + t * k + j);
       const float4* src = reinterpret_cast<const float4*>(y + r * H + c * 8);
       const float4 a = __ldg(src), b = __ldg(src + 1);
@@ -719,13 +822,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
-    uint32_t p[4];
+    if constexpr (kPartial) {
+      float4* dst = reinterpret_cast<float4*>(out_f32 + t * H + c * 8);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    } else {
+      uint32_t p[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-      p[q] = *reinterpret_cast<const uint32_t*>(&b2);
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+        p[q] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(out + t * H + c * 8) = make_uint4(p[0], p[1], p[2], p[3]);
     }
-    *reinterpret_cast<uint4*>(out + t * H + c * 8) = make_uint4(p[0], p[1], p[2], p[3]);
   }
 }
 
@@ -803,14 +912,77 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || nblk == 0) return err;
   const size_t smem = static_cast<size_t>(kScatterWarps) * E * sizeof(uint32_t);
-  route_scatter_kernel<<<nblk, kRouteTok, smem, s>>>(topk_ids, T, E, k, block_base,
+  route_scatter_kernel<<<nblk, kRouteTok, smem, s>>>(topk_ids, T, E, k, 0, block_base,
                                                      sorted_token_ids, row_of, row_amax_to_zero);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
+                              float* topk_w, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int64_t grid = (T + 7) / 8;
+  const int nv = (E + 31) / 32;
+  if (nv <= 1)
+    route_topk_kernel<1><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, nullptr);
+  else if (nv <= 2)
+    route_topk_kernel<2><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, nullptr);
+  else if (nv <= 4)
+    route_topk_kernel<4><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, nullptr);
+  else if (nv <= 8)
+    route_topk_kernel<8><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, nullptr);
+  else if (nv <= 16)
+    route_topk_kernel<16><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, nullptr);
+  else
+    route_topk_kernel<32><<<grid, 256, 0, s>>>(logits, T, E, k, topk_ids, topk_w, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, int k, int e_lo,
+                               int E_loc, int32_t* expert_offsets, int32_t* sorted_token_ids,
+                               int32_t* row_of, int32_t* block_counts, int32_t* block_base,
+                               int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
+                               int* latch, int num_sms, cudaStream_t s) {
+  const int64_t nblk = route_blocks(T);
+  if (nblk > 0) {
+    cudaError_t err = cudaMemsetAsync(block_counts, 0,
+                                      static_cast<size_t>(nblk) * E_loc * sizeof(int32_t), s);
+    if (err != cudaSuccess) return err;
+    route_ids_hist_kernel<<<grid_for(T * k, 256, num_sms), 256, 0, s>>>(
+        topk_ids, T, k, E_all, e_lo, E_loc, block_counts, latch);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E_loc, tile_n, block_base,
+                                       expert_offsets, tile_prefix);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || nblk == 0) return err;
+  const size_t smem = static_cast<size_t>(kScatterWarps) * E_loc * sizeof(uint32_t);
+  route_scatter_kernel<<<nblk, kRouteTok, smem, s>>>(topk_ids, T, E_loc, k, e_lo, block_base,
+                                                     sorted_token_ids, row_of, row_amax_to_zero);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_gather(const uint8_t* codes, int64_t H, const int32_t* sorted_token_ids,
+                             const int32_t* rows_total, int64_t max_rows, uint8_t* perm,
+                             float* gsum, uint16_t* sum_parts, int num_sms, cudaStream_t s) {
+  if (max_rows == 0) return cudaSuccess;
+  ep_gather_kernel<<<grid_for(max_rows * 32, 256, num_sms), 256, 0, s>>>(
+      codes, H, sorted_token_ids, rows_total, perm, gsum, sum_parts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cast_bf16(const float* x, int64_t n, void* out, int num_sms, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8) return cudaErrorInvalidValue;
+  cast_bf16_kernel<<<grid_for(n / 8, 256, num_sms), 256, 0, s>>>(
+      x, n / 8, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }
 
 cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t A, int64_t I,
                                uint8_t* codes, float* scales, float* gsum, int num_sms,
-                               cudaStream_t s, int32_t* int8_row_sum, uint16_t* sum_parts) {
+                               cudaStream_t s, int32_t* int8_row_sum, uint16_t* sum_parts,
+                               const int32_t* rows_dev) {
   if (A == 0) return cudaSuccess;
   const int grid = grid_for(A * (I / 16), 256, num_sms);
   if (int8_row_sum) {
@@ -818,10 +990,10 @@ cudaError_t launch_inter_quant(const float* h, const uint32_t* row_amax, int64_t
     if (err != cudaSuccess) return err;
     if (sum_parts) return cudaErrorInvalidValue;
     inter_quant_kernel<true><<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, nullptr,
-                                                  int8_row_sum, nullptr);
+                                                  int8_row_sum, nullptr, rows_dev);
   } else {
     inter_quant_kernel<false><<<grid, 256, 0, s>>>(h, row_amax, A, I, codes, scales, gsum,
-                                                   nullptr, sum_parts);
+                                                   nullptr, sum_parts, rows_dev);
   }
   return cudaGetLastError();
 }
@@ -866,11 +1038,15 @@ cudaError_t launch_nibble_row_sum(const int32_t* packed, int64_t R, int64_t word
 
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int64_t T,
                            int64_t H, int k, void* out, int num_sms, cudaStream_t s,
-                           const float* y_shared) {
+                           const float* y_shared, float* partial_f32) {
   if (T == 0) return cudaSuccess;
   const int grid = grid_for(T * (H / 8), 256, num_sms);
-  combine_kernel<<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k, y_shared,
-                                      static_cast<__nv_bfloat16*>(out));
+  if (partial_f32)
+    combine_kernel<true><<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k, nullptr, nullptr,
+                                              partial_f32);
+  else
+    combine_kernel<false><<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k, y_shared,
+                                               static_cast<__nv_bfloat16*>(out), nullptr);
   return cudaGetLastError();
 }
 

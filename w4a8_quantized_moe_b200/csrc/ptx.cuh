@@ -1,5 +1,5 @@
 // ptx.cuh - thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers, TMA (tiled and gather4), tcgen05 tensor memory and MMA.
+// mbarriers, tiled TMA loads, tcgen05 tensor memory and MMA.
 // Every wait here is bounded: it gives up after a deadline, raises the
 // CTA's abort flag and the device error latch, and returns false.
 #pragma once
@@ -9,10 +9,18 @@
 
 namespace w4a8 {
 
-// Device error latch (bit 0: a bounded wait ran out), one per translation
-// unit that includes this header; the unit that launches the waiting kernels
+// The library's one device error latch (bit 0: a bounded wait ran out; bit 1:
+// a caller-supplied or routing-derived index was out of range).  Without
+// relocatable device code a __device__ variable belongs to one translation
+// unit, so this header holds the definition and may be included by exactly one
+// unit, grouped_gemm.cu, which defines W4A8_OWNS_DEVICE_ERROR_LATCH first.
+// Kernels of other units reach the same latch through the pointer
+// device_error_latch() (internal.h) returns; read_and_clear_device_error()
 // reads and clears it for w4a8_check_device_error().
-static __device__ int g_device_error = 0;
+#ifndef W4A8_OWNS_DEVICE_ERROR_LATCH
+#error "ptx.cuh defines the device error latch: include it only from grouped_gemm.cu"
+#endif
+__device__ int g_device_error = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -2,11 +2,10 @@
 // callers that cannot allocate device memory.
 //
 // Some callers may not call cudaMalloc or any allocating routine at the point
-// where they route tokens: code running while a CUDA graph is being captured
-// (an allocation there fails the capture or is not replayed), runtimes and
-// plugin interfaces that hand a kernel only its pre-planned input and output
-// buffers and no scratch, and latency-critical paths whose memory budget is
-// fixed up front.  This entry point takes only inputs and outputs; its
+// where they route tokens: runtimes and plugin interfaces that hand a kernel
+// only its pre-planned input and output buffers and no scratch, and
+// latency-critical paths whose device memory budget is fixed up front.  This
+// entry point takes only inputs and outputs; its
 // scratch (per-block expert histograms, their scanned bases and the GEMM tile
 // prefix) lives in the file-scope device array below, which every device that
 // loads the library holds until the process exits.
@@ -38,7 +37,10 @@ int32_t* g_scratch_ptr[64] = {};
 
 // Device address of g_route_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in; the kernels need the address the
-// runtime reports for the current device, looked up once per device.
+// runtime reports for the current device, looked up once per device and kept
+// for the life of the process.  cudaDeviceReset discards the device's copy of
+// the array, so the kept address is stale afterwards: a process that resets a
+// device must not call w4a8_moe_route_permute_noalloc on it again.
 w4a8_status scratch_for_current_device(int32_t** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
