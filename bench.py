@@ -3,12 +3,17 @@
 One step = one ``w4a8_moe_forward`` (activation quantisation, routing +
 permutation, gate/up grouped GEMM + SwiGLU, intermediate requantisation, down
 grouped GEMM, combine) over one batch of synthetic tokens.  Prints one JSON
-line.  ``--impl reference`` times the CPU oracle instead (the only other
-place this script runs ``oracle/``).
+line: the headline workload (decode, 64 tokens, by default) and, on one GPU,
+a ``per_config`` entry for every workload.  ``--impl reference`` times the
+CPU oracle instead (the only other place this script runs ``oracle/``).
 
-Multi-GPU: one process per GPU (torchrun); each rank runs its own batch
-through its own copy of the experts (data parallel, no collective on the data
-path): weak scaling, value = all ranks' tokens / max-over-ranks time.
+Multi-GPU: one process per GPU (torchrun).  ``--parallel ep`` (the default
+for more than one GPU): expert parallelism -- each rank holds E / N of the
+experts and its own batch of tokens; the step all-gathers the quantised
+tokens, runs each rank's experts on them and reduce-scatters the partial
+sums (NCCL).  ``--parallel replicas``: every rank holds all experts and runs
+its own batch with no collective on the data path.  Both are weak scaling:
+value = all ranks' tokens / max-over-ranks time.
 """
 from __future__ import annotations
 
@@ -33,6 +38,10 @@ METRIC = "MoE-layer tokens/s on 1 B200 + % of HBM (decode) / FP8-peak (prefill) 
 DEFAULT_CONFIG = workloads.CONFIGS[1].name
 KERNELS_PER_STEP = 8   # act_quant, route topk/scan/scatter, gemm1, inter_quant, gemm2, combine
 SHARED_KERNELS_PER_STEP = 5   # tables, input group quant, gate/up GEMM, h group quant, down GEMM
+# expert-parallel step: act quant, top-k, then local hist/scan/scatter, gather,
+# gemm1, inter_quant, gemm2, partial combine, and the final bf16 cast
+EP_KERNELS_PER_STEP = 11
+SEGMENT_BINS = [(0, 0), (1, 8), (9, 32), (33, 128), (129, 512), (513, 2048), (2049, 1 << 31)]
 
 
 def peaks():
@@ -110,16 +119,19 @@ class ClockSampler:
         return out
 
 
-def build_layer(cfg, device, w4, variant: str = "w4a8"):
-    """Pack every expert's seeded bf16 weights on the device and lay them out for the GEMMs (not timed)."""
-    E, H, I = cfg.E, cfg.H, cfg.I
+def build_layer(cfg, device, w4, variant: str = "w4a8", experts=None):
+    """Pack the seeded bf16 weights of every expert (or of the range ``experts`` =
+    (begin, count), for one expert-parallel rank) on the device and lay them out
+    for the GEMMs (not timed)."""
+    H, I = cfg.H, cfg.I
+    e0, E = experts if experts is not None else (0, cfg.E)
     if variant == "channel-int8":
         p13 = torch.empty(E, 2 * I, H // 8, dtype=torch.int32, device=device)
         s13 = torch.empty(E, 2 * I, dtype=torch.bfloat16, device=device)
         p2 = torch.empty(E, H, I // 8, dtype=torch.int32, device=device)
         s2 = torch.empty(E, H, dtype=torch.bfloat16, device=device)
         for e in range(E):
-            w13, w2 = workloads.gen_expert_weights(cfg, e, device=device)
+            w13, w2 = workloads.gen_expert_weights(cfg, e0 + e, device=device)
             w4.w4a8_pack_int4_channel(w13, packed=p13[e], scales=s13[e])
             w4.w4a8_pack_int4_channel(w2, packed=p2[e], scales=s2[e])
         p13, n13 = w4.w4a8_prepare_experts_channel_b200(p13, packed_out=p13)
@@ -131,7 +143,7 @@ def build_layer(cfg, device, w4, variant: str = "w4a8"):
     p2 = torch.empty(E, H, I // 8, dtype=torch.int32, device=device)
     s2 = torch.empty(E, H, I // 128, dtype=torch.bfloat16, device=device)
     for e in range(E):
-        w13, w2 = workloads.gen_expert_weights(cfg, e, device=device)
+        w13, w2 = workloads.gen_expert_weights(cfg, e0 + e, device=device)
         w4.w4a8_pack_int4(w13, packed=p13[e], scales=s13[e])
         w4.w4a8_pack_int4(w2, packed=p2[e], scales=s2[e])
     p13, s13g = w4.w4a8_prepare_experts_b200(p13, s13, packed_out=p13)
@@ -210,8 +222,67 @@ def shared_work(cfg):
     return s1, s2
 
 
+def layer_work(cfg, counts, variant: str = "w4a8"):
+    """Algorithmic bytes and FLOPs of the whole layer (one step): the HBM bytes
+    of every active expert's weights and scales, the hidden states and logits
+    read, the output written, and the intermediates that cross HBM between the
+    kernels (h written and read as float32, its codes, the float32 Y rows
+    written and read); FLOPs 6 A H I."""
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    A = T * k
+    active = int(np.count_nonzero(counts))
+    if variant == "channel-int8":
+        per_expert = 2 * I * H // 2 + 2 * I * 6 + H * I // 2 + H * 6
+    else:
+        per_expert = 2 * I * H // 2 + 2 * I * (H // 128) * 2 + H * I // 2 + H * (I // 128) * 2
+    nbytes = (active * per_expert + T * H * 2 + T * E * 4 + T * H * 2 + A * I * (4 + 4 + 1)
+              + A * H * 4 * 2)
+    return dict(bytes=nbytes, flops=6 * A * H * I)
+
+
+def segment_histogram(counts):
+    """Segment sizes (tokens per expert) in bins, with the active count and the maximum."""
+    c = np.asarray(counts, dtype=np.int64)
+    bins = {(f"{lo}" if lo == hi else f"{lo}-{hi}" if hi < (1 << 31) else f">={lo}"):
+            int(np.count_nonzero((c >= lo) & (c <= hi))) for lo, hi in SEGMENT_BINS}
+    return dict(bins=bins, active=int(np.count_nonzero(c)), max=int(c.max(initial=0)),
+                experts=int(c.size))
+
+
+def input_digest(hidden: torch.Tensor, logits: torch.Tensor) -> str:
+    """sha256 of the generated hidden-state and logit bytes, as the oracle sees them."""
+    h = hashlib.sha256()
+    for t in (hidden, logits):
+        h.update(t.contiguous().view(torch.uint8).cpu().numpy().tobytes())
+    return h.hexdigest()
+
+
+def roofline(work, ms, prefill: bool, pk, kernel=None, traffic=None):
+    """Achieved / peak for ``work`` (dict with bytes and flops) done in ``ms``:
+    HBM bytes against the measured copy bandwidth for decode-shaped batches,
+    FLOPs against the FP8 dense rate (2 x the measured bf16 GEMM rate, the
+    nominal FP8 / bf16 ratio) for prefill-shaped ones."""
+    if prefill:
+        achieved = work["flops"] / (ms / 1e3) / 1e12
+        peak, peak_sus = 2.0 * pk["bf16"], 2.0 * pk["bf16_sus"]
+        out = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
+                   frac=achieved / peak, frac_of_sustained=achieved / peak_sus,
+                   peak_source=f"{pk['src']} bf16 GEMM burst x 2 (FP8 dense); sustained x 2 = "
+                               f"{peak_sus:.1f}")
+    else:
+        achieved = work["bytes"] / (ms / 1e3) / 1e9
+        out = dict(bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
+                   frac=achieved / pk["hbm"], peak_source=f"{pk['src']} HBM copy")
+    if kernel is not None:
+        out["kernel"] = kernel
+        out["traffic"] = traffic
+    return out
+
+
 class OracleSample:
     """The CPU oracle on a seeded sample of tokens, experts quantised up front."""
+
+    MAX_ROWS = 256
 
     def __init__(self, cfg, n_tokens: int, seed_tokens: int = 7, variant: str = "w4a8"):
         import oracle
@@ -226,10 +297,14 @@ class OracleSample:
         self.cores = self.cores or os.cpu_count()
         f = lambda t: oracle.bf16_bits_to_f64(t.contiguous().view(torch.int16).numpy()
                                               .view(np.uint16))
-        self.hidden = f(workloads.gen_hidden(cfg))
-        self.logits = workloads.gen_logits(cfg).numpy()
+        # the tokens are drawn from the first rows of the workload's generator
+        # (same recipe; generating all T rows on the host would dominate)
+        self.rows = min(cfg.T, self.MAX_ROWS)
+        self.hidden = f(workloads.gen_hidden(cfg, T=self.rows))
+        self.logits = workloads.gen_logits(cfg, T=self.rows).numpy()
         rng = np.random.default_rng(seed_tokens)
-        self.tokens = np.sort(rng.choice(cfg.T, size=min(n_tokens, cfg.T), replace=False))
+        self.tokens = np.sort(rng.choice(self.rows, size=min(n_tokens, self.rows),
+                                         replace=False))
         ids, _ = oracle.route_topk(self.logits, cfg.k)
 
         def weights(e):
@@ -254,8 +329,8 @@ class OracleSample:
 
     def describe(self, dt: float) -> str:
         return (f"{len(self.tokens)} of {self.cfg.T} tokens of {self.cfg.name} per step "
-                f"(their {self.cfg.k} experts each, RTN-quantised before timing), float64 "
-                f"numpy, {dt:.2f} s per step")
+                f"(drawn from the generator's first {self.rows} rows; their {self.cfg.k} "
+                f"experts each, RTN-quantised before timing), float64 numpy, {dt:.2f} s per step")
 
 
 def cpu_baseline(cfg, n_tokens: int, variant: str = "w4a8"):
@@ -288,6 +363,185 @@ def bench_reference(args, cfg, rank):
     return 0
 
 
+def run_single(cfg, args, device, w4, cpu_tokens: int):
+    """One workload on one GPU: device-timed steps with per-stage events and
+    clock samples, then the end-to-end loop through host buffers.  Returns the
+    fields of the JSON line for this workload."""
+    layer = build_layer(cfg, device, w4, args.variant)
+    hidden = workloads.gen_hidden(cfg, device=device)
+    logits = workloads.gen_logits(cfg, device=device)
+    digest = input_digest(hidden, logits) if args.digest else None
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=device)
+    offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    shared = args.variant == "w4a8+shared"
+    n_ev = 2 * w4.NUM_STAGES + (8 if shared else 0)
+
+    def step(events=None):
+        if events:
+            # torch only reports elapsed time for events it recorded itself; the
+            # library re-records each one at its stage boundary later in the stream
+            for e in events:
+                e.record(stream)
+        kw = {}
+        if shared:
+            kw["shared_stage_events"] = events[2 * w4.NUM_STAGES:] if events else None
+            events = events[:2 * w4.NUM_STAGES] if events else None
+        layer(hidden, logits, out=out, aux={"expert_offsets": offsets}, stage_events=events, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    w4.w4a8_check_device_error(device)
+    counts = np.diff(offsets.cpu().numpy().astype(np.int64))
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    w4.w4a8_check_device_error(device)
+    ms = t_start.elapsed_time(t_end)
+    stage_ms = [statistics.mean(ev[i][2 * s_].elapsed_time(ev[i][2 * s_ + 1])
+                                for i in range(args.steps)) for s_ in range(n_ev // 2)]
+
+    # end to end through the public API: inputs copied in from pinned host
+    # memory and the output read back every step, each step waiting for its
+    # output on the host before the next one starts
+    h_host = hidden.cpu().pin_memory()
+    l_host = logits.cpu().pin_memory()
+    o_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    h_dev = torch.empty_like(hidden)
+    l_dev = torch.empty_like(logits)
+    done = torch.cuda.Event()
+
+    def e2e_step():
+        h_dev.copy_(h_host, non_blocking=True)
+        l_dev.copy_(l_host, non_blocking=True)
+        layer(h_dev, l_dev, out=out)
+        o_host.copy_(out, non_blocking=True)
+        done.record(stream)
+        done.synchronize()
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e_start.elapsed_time(e_end)
+
+    pk = peaks()
+    g1, g2, active = algorithmic_work(cfg, counts, args.variant)
+    prefill = cfg.T >= 4096
+    gi = 2 if stage_ms[2] >= stage_ms[4] else 4          # dominant kernel: the slower GEMM
+    kname = "grouped_gemm_gate_up" if gi == 2 else "grouped_gemm_down"
+    traffic_key = cfg.name if args.variant == "w4a8" else f"{cfg.name}:{args.variant}"
+    res = dict(
+        cfg=cfg, ms=ms, e2e_ms=e2e_ms, stage_ms=stage_ms, counts=counts, active=active,
+        roofline=roofline(g1 if gi == 2 else g2, stage_ms[gi], prefill, pk, kname,
+                          recorded_traffic(traffic_key, kname)),
+        roofline_layer=roofline(layer_work(cfg, counts, args.variant), ms / args.steps, prefill,
+                                pk),
+        clocks=clk.summary(), digest=digest, l2_bytes=g1["bytes"] + g2["bytes"])
+    if shared:   # the shared expert's slower GEMM against the same peak
+        s1, s2 = shared_work(cfg)
+        # stages 6..9: shared input quantisation, gate/up GEMM, requantisation, down GEMM
+        si = 1 if stage_ms[7] >= stage_ms[9] else 3
+        sw_, st_ = (s1, stage_ms[7]) if si == 1 else (s2, stage_ms[9])
+        res["shared_roofline"] = roofline(sw_, st_, prefill, pk,
+                                          "shared_gemm_gate_up" if si == 1 else "shared_gemm_down")
+    if cpu_tokens > 0:
+        res["cpu_baseline"] = cpu_baseline(cfg, cpu_tokens, args.variant)
+    del layer
+    return res
+
+
+def config_fields(cfg, res, args, world=1, parallelism="single"):
+    c = dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
+             variant=args.variant, active_experts=res["active"], parallelism=parallelism,
+             segments=segment_histogram(res["counts"]),
+             l2=("inputs larger than L2: %.2f GB of packed experts streamed per step"
+                 % (res["l2_bytes"] / 1e9)))
+    if res.get("digest"):
+        c["inputs_sha256"] = res["digest"]
+    return c
+
+
+def stage_names(w4, shared):
+    return w4.STAGE_NAMES + (w4.SHARED_STAGE_NAMES if shared else [])
+
+
+def run_expert_parallel(cfg, args, device, w4, dist, rank, world):
+    """Expert parallelism over the ranks: rank g holds experts
+    expert_partition(E, world)[g] and its own batch of cfg.T tokens."""
+    from w4a8_quantized_moe_b200.ep import ExpertParallelMoE, expert_partition
+    b, n = expert_partition(cfg.E, world)[rank]
+    local = build_layer(cfg, device, w4, experts=(b, n)) if n else None
+    weights = ((local.w13_packed, local.w13_scales, local.w2_packed, local.w2_scales)
+               if local is not None else None)
+    ep = ExpertParallelMoE(weights, cfg.E, cfg.k, b, n, cfg.H, cfg.I, tokens_per_rank=cfg.T)
+    rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)      # each rank its own batch
+    hidden = workloads.gen_hidden(rank_cfg, device=device)
+    logits = workloads.gen_logits(rank_cfg, device=device)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        ep(hidden, logits, out=out)
+    w4.w4a8_check_device_error(device)
+    # the experts this rank's share actually served (from the gathered ids)
+    gat_ids = next(iter(ep._bufs.values()))[1].ids.cpu().numpy()
+    local_counts = np.array([np.count_nonzero(gat_ids == e) for e in range(b, b + n)])
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clk:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            ep(hidden, logits, out=out)
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    dist.barrier()
+    w4.w4a8_check_device_error(device)
+    ms = t_start.elapsed_time(t_end)
+
+    h_host = hidden.cpu().pin_memory()
+    l_host = logits.cpu().pin_memory()
+    o_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    h_dev, l_dev = torch.empty_like(hidden), torch.empty_like(logits)
+    done = torch.cuda.Event()
+
+    def e2e_step():
+        h_dev.copy_(h_host, non_blocking=True)
+        l_dev.copy_(l_host, non_blocking=True)
+        ep(h_dev, l_dev, out=out)
+        o_host.copy_(out, non_blocking=True)
+        done.record(stream)
+        done.synchronize()
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(device)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e_start.elapsed_time(e_end)
+    dist.barrier()
+    return dict(ms=ms, e2e_ms=e2e_ms, local_counts=local_counts, experts=(b, n),
+                clocks=clk.summary())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -310,11 +564,18 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload with this many tokens instead (a smaller case for "
                          "profiler captures; recorded in config)")
+    ap.add_argument("--per-config", type=int, default=1,
+                    help="on one GPU, also time every other workload into per_config (0: no)")
+    ap.add_argument("--parallel", default="ep", choices=["ep", "replicas"],
+                    help="more than one GPU: expert parallelism (default) or full replicas")
+    ap.add_argument("--digest", type=int, default=1,
+                    help="log the sha256 of each workload's generated inputs (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     cfg = workloads.config_by_name(args.config)
+    custom = bool(args.experts or args.tokens)
     if args.experts:
         cfg = cfg.with_(name=f"{cfg.name}_E{args.experts}", E=args.experts,
                         forced_empty=min(cfg.forced_empty, args.experts // 16))
@@ -330,152 +591,119 @@ def main():
     import w4a8_quantized_moe_b200 as w4
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
-
-    layer = build_layer(cfg, device, w4, args.variant)
-    rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)      # each rank its own batch
-    hidden = workloads.gen_hidden(rank_cfg, device=device)
-    logits = workloads.gen_logits(rank_cfg, device=device)
-    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=device)
-    ws = layer.workspace(cfg.T)
-    offsets = torch.empty(cfg.E + 1, dtype=torch.int32, device=device)
-    stream = torch.cuda.current_stream(device)
-
+    dtype = "s8xint4-s32acc" if args.variant == "channel-int8" else "e4m3xint4-f32acc"
     shared = args.variant == "w4a8+shared"
-    n_ev = 2 * w4.NUM_STAGES + (8 if shared else 0)
 
-    def step(events=None):
-        if events:
-            # torch only reports elapsed time for events it recorded itself; the
-            # library re-records each one at its stage boundary later in the stream
-            for e in events:
-                e.record(stream)
-        kw = {}
-        if shared:
-            kw["shared_stage_events"] = events[2 * w4.NUM_STAGES:] if events else None
-            events = events[:2 * w4.NUM_STAGES] if events else None
-        layer(hidden, logits, out=out, aux={"expert_offsets": offsets}, stage_events=events, **kw)
+    if world == 1:
+        head = run_single(cfg, args, device, w4, args.cpu_tokens)
+        line = dict(
+            metric=METRIC, value=whole_job_throughput(cfg.T, 1, args.steps, head["ms"]),
+            unit="tokens/s", n_gpus=1, steps=args.steps, warmup=args.warmup,
+            ms_per_step=head["ms"] / args.steps, higher_is_better=True, scaling="weak",
+            vs_baseline=None, dtype=dtype, data="synthetic",
+            config=config_fields(cfg, head, args),
+            stage_ms={n_: round(x, 5) for n_, x in zip(stage_names(w4, shared), head["stage_ms"])},
+            roofline=head["roofline"], roofline_layer=head["roofline_layer"],
+            e2e=dict(value=whole_job_throughput(cfg.T, 1, args.steps, head["e2e_ms"]),
+                     unit="tokens/s", h2d_bytes_per_step=cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
+                     d2h_bytes_per_step=cfg.T * cfg.H * 2, host_round_trip_per_step=True),
+            gpu_launches=(KERNELS_PER_STEP + (SHARED_KERNELS_PER_STEP if shared else 0))
+            * args.steps,
+            clocks=head["clocks"])
+        if "shared_roofline" in head:
+            line["shared_roofline"] = head["shared_roofline"]
+        if "cpu_baseline" in head:
+            line["cpu_baseline"] = head["cpu_baseline"]
+        if args.per_config and not custom:
+            per = {}
+            for c in workloads.CONFIGS:
+                r = head if c.name == cfg.name else run_single(c, args, device, w4, 1)
+                torch.cuda.empty_cache()
+                per[c.name] = dict(
+                    ms_per_step=r["ms"] / args.steps,
+                    tokens_per_s=whole_job_throughput(c.T, 1, args.steps, r["ms"]),
+                    e2e_tokens_per_s=whole_job_throughput(c.T, 1, args.steps, r["e2e_ms"]),
+                    stage_ms={n_: round(x, 5) for n_, x in
+                              zip(stage_names(w4, shared), r["stage_ms"])},
+                    roofline=r["roofline"], roofline_layer=r["roofline_layer"],
+                    config=config_fields(c, r, args), clocks=r["clocks"],
+                    gpu_launches=(KERNELS_PER_STEP + (SHARED_KERNELS_PER_STEP if shared else 0))
+                    * args.steps)
+                if "cpu_baseline" in r:
+                    per[c.name]["cpu_baseline"] = r["cpu_baseline"]
+                if "shared_roofline" in r:
+                    per[c.name]["shared_roofline"] = r["shared_roofline"]
+            line["per_config"] = per
+        print(json.dumps(line), flush=True)
+        return 0
 
-    for _ in range(args.warmup):
-        step()
-    w4.w4a8_check_device_error(device)
-    counts = np.diff(offsets.cpu().numpy().astype(np.int64))
-
-    # ---------------- device-resident timing (kernel path)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-          for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize(device)
-    with ClockSampler(device) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(ev[i])
-        t_end.record(stream)
-        torch.cuda.synchronize(device)
-    if dist:
-        dist.barrier()
-    w4.w4a8_check_device_error(device)
-    ms = t_start.elapsed_time(t_end)
-    stage_ms = [statistics.mean(ev[i][2 * s].elapsed_time(ev[i][2 * s + 1])
-                                for i in range(args.steps)) for s in range(n_ev // 2)]
-
-    # ---------------- end to end through the public API, host buffers
-    h_host = hidden.cpu().pin_memory()
-    l_host = logits.cpu().pin_memory()
-    o_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
-    h_dev = torch.empty_like(hidden)
-    l_dev = torch.empty_like(logits)
-
-    def e2e_step():
-        h_dev.copy_(h_host, non_blocking=True)
-        l_dev.copy_(l_host, non_blocking=True)
-        layer(h_dev, l_dev, out=out)
-        o_host.copy_(out, non_blocking=True)
-
-    for _ in range(args.warmup):
-        e2e_step()
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(device)
-    if dist:
-        dist.barrier()
-    e_start.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e_end.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = e_start.elapsed_time(e_end)
-
-    if dist:
-        ms, e2e_ms, *stage_ms = max_over_ranks(dist, [ms, e2e_ms] + stage_ms, device)
-
-    value = whole_job_throughput(cfg.T, world, args.steps, ms)
-    e2e_value = whole_job_throughput(cfg.T, world, args.steps, e2e_ms)
-
-    pk = peaks()
-    g1, g2, active = algorithmic_work(cfg, counts, args.variant)
-    prefill = cfg.T >= 4096
-    gi = 2 if stage_ms[2] >= stage_ms[4] else 4          # dominant kernel: the slower GEMM
-    work = g1 if gi == 2 else g2
-    kname = "grouped_gemm_gate_up" if gi == 2 else "grouped_gemm_down"
-    traffic_key = cfg.name if args.variant == "w4a8" else f"{cfg.name}:{args.variant}"
-    if prefill:
-        achieved = work["flops"] / (stage_ms[gi] / 1e3) / 1e12
-        peak = 2.0 * pk["bf16_sus"]                     # FP8 = 2 x bf16 (nominal ratio)
-        roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
-                    frac=achieved / peak, traffic=recorded_traffic(traffic_key, kname), kernel=kname,
-                    peak_source=f"{pk['src']} sustained bf16 x 2")
-    else:
-        achieved = work["bytes"] / (stage_ms[gi] / 1e3) / 1e9
-        peak = pk["hbm"]
-        roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak,
-                    traffic=recorded_traffic(traffic_key, kname), kernel=kname,
-                    peak_source=f"{pk['src']} HBM copy")
-
-    line = dict(
-        metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
-        warmup=args.warmup, ms_per_step=ms / args.steps, higher_is_better=True, scaling="weak",
-        vs_baseline=None,
-        dtype="s8xint4-s32acc" if args.variant == "channel-int8" else "e4m3xint4-f32acc",
-        data="synthetic",
-        config=dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
-                    variant=args.variant, active_experts=active,
-                    parallelism=f"dp{world}" if world > 1 else "single",
-                    l2=("inputs larger than L2: %.2f GB of packed experts streamed per step"
-                        % ((g1["bytes"] + g2["bytes"]) / 1e9))),
-        stage_ms={n: round(x, 5) for n, x in
-                  zip(w4.STAGE_NAMES + (w4.SHARED_STAGE_NAMES if shared else []), stage_ms)},
-        roofline=roof,
-        e2e=dict(value=e2e_value, unit="tokens/s",
-                 h2d_bytes_per_step=cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
-                 d2h_bytes_per_step=cfg.T * cfg.H * 2),
-        gpu_launches=(KERNELS_PER_STEP + (SHARED_KERNELS_PER_STEP if shared else 0)) * args.steps,
-        clocks=clk.summary(),
-    )
-    if shared:   # the shared expert's slower GEMM against the same peak
-        s1, s2 = shared_work(cfg)
-        # stages 6..9: shared input quantisation, gate/up GEMM, requantisation, down GEMM
-        si = 1 if stage_ms[7] >= stage_ms[9] else 3
-        sw_, st_ = (s1, stage_ms[7]) if si == 1 else (s2, stage_ms[9])
-        sname = "shared_gemm_gate_up" if si == 1 else "shared_gemm_down"
-        if prefill:
-            a_ = sw_["flops"] / (st_ / 1e3) / 1e12
-            line["shared_roofline"] = dict(bound="tensor", achieved=a_, peak=roof["peak"],
-                                           unit="TFLOP/s", frac=a_ / roof["peak"], kernel=sname)
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        if args.parallel == "ep":
+            from w4a8_quantized_moe_b200.ep import expert_partition
+            if args.variant != "w4a8":
+                raise SystemExit("--parallel ep runs the w4a8 variant only")
+            r = run_expert_parallel(cfg, args, device, w4, dist, rank, world)
+            ms, e2e_ms = max_over_ranks(dist, [r["ms"], r["e2e_ms"]], device)
+            b, n = r["experts"]
+            pk = peaks()
+            T, H, I, k = cfg.T, cfg.H, cfg.I, cfg.k
+            Tg = T * world
+            per_expert = 2 * I * H // 2 + 2 * I * (H // 128) * 2 + H * I // 2 + H * (I // 128) * 2
+            A_loc = int(r["local_counts"].sum())
+            work = dict(bytes=int(np.count_nonzero(r["local_counts"])) * per_expert
+                        + Tg * H + Tg * 4 + A_loc * I * 9 + A_loc * H * 8 + Tg * H * 4,
+                        flops=6 * A_loc * H * I)
+            line = dict(
+                metric=METRIC, value=whole_job_throughput(T, world, args.steps, ms),
+                unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=ms / args.steps, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype=dtype, data="synthetic",
+                config=dict(workload=cfg.name, T=T, H=H, I=I, E=cfg.E, k=k, variant=args.variant,
+                            parallelism=f"ep{world}", tokens_per_rank=T,
+                            experts_per_rank=[n_ for _, n_ in expert_partition(cfg.E, world)],
+                            rank0_experts_served=int(np.count_nonzero(r["local_counts"])),
+                            dispatch="all-gather of E4M3 codes, scales, ids, weights (NCCL)",
+                            combine="reduce-scatter of float32 partial sums (NCCL)"),
+                roofline=roofline(work, ms / args.steps, T * world >= 4096, pk,
+                                  "ep_step (rank 0: dispatch + local experts + combine)"),
+                e2e=dict(value=whole_job_throughput(T, world, args.steps, e2e_ms),
+                         unit="tokens/s", h2d_bytes_per_step=world * (T * H * 2 + T * cfg.E * 4),
+                         d2h_bytes_per_step=world * T * H * 2, host_round_trip_per_step=True),
+                gpu_launches=EP_KERNELS_PER_STEP * args.steps, clocks=r["clocks"])
         else:
-            a_ = sw_["bytes"] / (st_ / 1e3) / 1e9
-            line["shared_roofline"] = dict(bound="hbm", achieved=a_, peak=roof["peak"],
-                                           unit="GB/s", frac=a_ / roof["peak"], kernel=sname)
-    if rank == 0 and world == 1 and args.cpu_tokens > 0:
-        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, args.variant)
-    if dist:
+            layer = build_layer(cfg, device, w4, args.variant)
+            rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)
+            hidden = workloads.gen_hidden(rank_cfg, device=device)
+            logits = workloads.gen_logits(rank_cfg, device=device)
+            out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=device)
+            stream = torch.cuda.current_stream(device)
+            for _ in range(args.warmup):
+                layer(hidden, logits, out=out)
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            dist.barrier()
+            torch.cuda.synchronize(device)
+            with ClockSampler(device) as clk:
+                t0.record(stream)
+                for _ in range(args.steps):
+                    layer(hidden, logits, out=out)
+                t1.record(stream)
+                torch.cuda.synchronize(device)
+            dist.barrier()
+            w4.w4a8_check_device_error(device)
+            (ms,) = max_over_ranks(dist, [t0.elapsed_time(t1)], device)
+            line = dict(
+                metric=METRIC, value=whole_job_throughput(cfg.T, world, args.steps, ms),
+                unit="tokens/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=ms / args.steps, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype=dtype, data="synthetic",
+                config=dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
+                            variant=args.variant, parallelism=f"replicas{world}"),
+                gpu_launches=KERNELS_PER_STEP * args.steps, clocks=clk.summary())
         dist.barrier()
+    finally:
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)

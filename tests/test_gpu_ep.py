@@ -28,6 +28,15 @@ def _share(layer, g, G):
                   layer.w2_packed[b:b + n], layer.w2_scales[b:b + n])
 
 
+def _bf16_agreement(a: torch.Tensor, b: torch.Tensor):
+    """(fraction of equal bf16 values, largest distance in bf16 steps)."""
+    def ordinal(t):
+        v = t.view(torch.int16).to(torch.int32).cpu()
+        return torch.where(v < 0, -(v & 0x7FFF), v)
+    d = (ordinal(a) - ordinal(b)).abs()
+    return float((d == 0).float().mean()), int(d.max())
+
+
 def _emulated_ep(layer, codes, scales, ids, w, G):
     total = torch.zeros(codes.shape[0], layer.H, dtype=torch.float32, device="cuda")
     for g in range(G):
@@ -56,12 +65,13 @@ def test_expert_shares_sum_to_the_layer(cfg, G):
     out = _emulated_ep(layer, aux["act_codes"], aux["act_scales"], ids, w, G)
     store = oracle.ExpertStore(cfg.E, lambda e: (f64(w13[e]), f64(w2[e])))
     res = oracle.moe_forward(f64(hidden), logits.numpy(), store, cfg.k)
-    e_layer = rel_fro(f64(out), f64(ref))
+    # the shares' float32 sums are added in another order than the layer's slot
+    # sum, so a value may land one bf16 step away where the sum sits at a midpoint
+    same, steps = _bf16_agreement(out, ref)
     e_oracle = rel_fro(f64(out), res["out"])
-    same = float((out.view(torch.int16) == ref.view(torch.int16)).float().mean())
-    print(f"\n[{cfg.name}, {G} shares] vs layer {e_layer:.2e} ({same:.4f} bit-equal), "
+    print(f"\n[{cfg.name}, {G} shares] vs layer: {same:.5f} equal, max {steps} bf16 step(s); "
           f"vs oracle {e_oracle:.2e}")
-    assert e_layer <= 1e-5 and same >= 0.99
+    assert same >= 0.999 and steps <= 1
     assert e_oracle <= 2e-3
 
 
@@ -133,8 +143,7 @@ def test_decode_workload_split_over_eight_shares():
     ref = layer(hidden, logits, aux=aux)
     out = _emulated_ep(layer, aux["act_codes"], aux["act_scales"], aux["topk_ids"],
                        aux["topk_w"], 8)
-    e_layer = rel_fro(f64(out), f64(ref))
-    same = float((out.view(torch.int16) == ref.view(torch.int16)).float().mean())
-    print(f"\n[decode, 8 shares of 32 experts, 512 tokens] vs layer {e_layer:.2e} "
-          f"({same:.4f} bit-equal)")
-    assert e_layer <= 1e-5 and same >= 0.99
+    same, steps = _bf16_agreement(out, ref)
+    print(f"\n[decode, 8 shares of 32 experts, 512 tokens] vs layer: {same:.5f} equal, "
+          f"max {steps} bf16 step(s); rel-Frobenius {rel_fro(f64(out), f64(ref)):.2e}")
+    assert same >= 0.999 and steps <= 1

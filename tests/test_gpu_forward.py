@@ -143,3 +143,26 @@ def test_forward_zero_tokens():
     out = layer(torch.zeros(0, 256, dtype=torch.bfloat16, device="cuda"),
                 torch.zeros(0, 4, device="cuda"))
     assert out.shape == (0, 256)
+
+
+def test_pages_format_goes_through_prepare():
+    # the experts as the pages store them (compressed-tensors pack-quantized
+    # words and [E, rows, K/128] scales) reach the forward only through
+    # w4a8_prepare_experts_b200: from_packed gives the layout from_bf16 gives,
+    # and the forward refuses the pages' scale layout with a message naming it
+    cfg = workloads.MoEConfig("pages_format", T=12, H=256, I=128, E=3, k=2, seed=31)
+    hidden, logits, w13, w2 = small_case(cfg)
+    p13, s13 = w4.w4a8_pack_int4(w13.cuda())
+    p2, s2 = w4.w4a8_pack_int4(w2.cuda())
+    ref = w4.W4A8MoELayer.from_bf16(w13.cuda(), w2.cuda(), cfg.k)
+    lay = w4.W4A8MoELayer.from_packed(p13, s13, p2, s2, cfg.k)
+    for a, b in ((lay.w13_packed, ref.w13_packed), (lay.w13_scales, ref.w13_scales),
+                 (lay.w2_packed, ref.w2_packed), (lay.w2_scales, ref.w2_scales)):
+        assert a.shape == b.shape and torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16
+                                                  else a, b.view(torch.int16)
+                                                  if b.dtype == torch.bfloat16 else b)
+    assert torch.equal(p13, w4.w4a8_pack_int4(w13.cuda())[0])   # not in place by default
+    out = lay(hidden.cuda(), logits.cuda())
+    assert torch.equal(out.view(torch.int16), ref(hidden.cuda(), logits.cuda()).view(torch.int16))
+    with pytest.raises(ValueError, match="w4a8_prepare_experts_b200"):
+        w4.w4a8_moe_forward(hidden.cuda(), logits.cuda(), p13, s13, p2, s2, cfg.k)

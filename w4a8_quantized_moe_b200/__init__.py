@@ -337,6 +337,10 @@ def w4a8_moe_forward(hidden: torch.Tensor, logits: torch.Tensor, w13_packed: tor
     T, H = hidden.shape
     E = logits.shape[1]
     I = w2_packed.shape[2] * 8
+    if w13_scales.shape == (E, 2 * I, H // 128) and w13_scales.shape != (E, H // 128, 2 * I):
+        raise ValueError("w13_scales is in the pack-quantized layout [E, 2I, H/128]; "
+                         "w4a8_moe_forward reads experts laid out by "
+                         "w4a8_prepare_experts_b200 (or W4A8MoELayer.from_packed)")
     if logits.shape[0] != T or w13_packed.shape != (E, 2 * I, H // 8) or \
             w2_packed.shape != (E, H, I // 8) or w13_scales.shape != (E, H // 128, 2 * I) or \
             w2_scales.shape != (E, I // 128, H):
@@ -380,8 +384,20 @@ class W4A8MoELayer:
                   mse_clip: bool = False) -> "W4A8MoELayer":
         p13, s13 = w4a8_pack_int4(w13, mse_clip=mse_clip)
         p2, s2 = w4a8_pack_int4(w2, mse_clip=mse_clip)
-        p13, s13 = w4a8_prepare_experts_b200(p13, s13, packed_out=p13)
-        p2, s2 = w4a8_prepare_experts_b200(p2, s2, packed_out=p2)
+        return cls.from_packed(p13, s13, p2, s2, k, in_place=True)
+
+    @classmethod
+    def from_packed(cls, w13_packed: torch.Tensor, w13_scales: torch.Tensor,
+                    w2_packed: torch.Tensor, w2_scales: torch.Tensor, k: int,
+                    in_place: bool = False) -> "W4A8MoELayer":
+        """A layer from experts in the pages' compressed-tensors format, as
+        ``w4a8_pack_int4`` writes it (uint4b8 words [E, rows, K/8], little-endian
+        nibbles; bf16 scales [E, rows, K/128]): ``w4a8_prepare_experts_b200``
+        lays them out for ``w4a8_moe_forward`` (in place if ``in_place``)."""
+        p13, s13 = w4a8_prepare_experts_b200(w13_packed, w13_scales,
+                                             packed_out=w13_packed if in_place else None)
+        p2, s2 = w4a8_prepare_experts_b200(w2_packed, w2_scales,
+                                           packed_out=w2_packed if in_place else None)
         return cls(p13, s13, p2, s2, k)
 
     def workspace(self, T: int) -> torch.Tensor:
