@@ -60,6 +60,17 @@ typedef int32_t w4a8_status;
 /* ABI version of this header (incremented on incompatible changes). */
 W4A8_API int32_t w4a8_abi_version(void);
 
+/*
+ * Build flags of the loaded library: bit 0 (W4A8_BUILD_DEBUG_BOUNDS) is set in
+ * the bounds-checking build (libw4a8_debug.so), whose kernels check every
+ * routing-derived index (expert offsets and tile tables, segment rows, token
+ * ids) against its buffer before use; an index out of range is skipped and
+ * reported as W4A8_ERR_DEVICE_INDEX by w4a8_check_device_error.  No
+ * counterpart on the pages: it stands in for a memory checker.
+ */
+#define W4A8_BUILD_DEBUG_BOUNDS 1
+W4A8_API int32_t w4a8_build_flags(void);
+
 /* Static text of a status code. */
 W4A8_API const char* w4a8_status_string(w4a8_status status);
 

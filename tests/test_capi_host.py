@@ -50,7 +50,20 @@ def test_status_strings_and_version(L):
     assert L.w4a8_abi_version() == 1
     assert L.w4a8_status_string(0) == b"W4A8_OK"
     assert L.w4a8_status_string(6) == b"W4A8_ERR_DEVICE_TIMEOUT"
+    assert L.w4a8_status_string(7) == b"W4A8_ERR_DEVICE_INDEX"
     assert L.w4a8_status_string(99) == b"W4A8_ERR_UNKNOWN"
+
+
+def test_release_and_bounds_checking_builds():
+    # the two builds of the same sources: same exports, and the build flag
+    # tells them apart (the debug build checks routing-derived indices)
+    from w4a8_quantized_moe_b200 import build as b
+    rel = ctypes.CDLL(b.build())
+    dbg = ctypes.CDLL(b.build(debug_bounds=True))
+    assert rel.w4a8_build_flags() == 0
+    assert dbg.w4a8_build_flags() == 1
+    for name in declared_functions():
+        assert hasattr(dbg, name), f"{name} missing from the debug build"
 
 
 def test_workspace_sizes_are_host_arithmetic(L):

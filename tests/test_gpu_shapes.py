@@ -22,7 +22,7 @@ CASES = ("tiny_workload or ragged or multi_block_segments or zipf_empty or outli
 @pytest.mark.parametrize("var,shape", [
     ("W4A8_GEMM_DECODE_SHAPE", 1), ("W4A8_GEMM_DECODE_SHAPE", 2),
     ("W4A8_GEMM_DECODE_SHAPE", 3), ("W4A8_GEMM_DECODE_SHAPE", 4),
-    ("W4A8_GEMM_DECODE_SHAPE", 5),
+    ("W4A8_GEMM_DECODE_SHAPE", 5), ("W4A8_GEMM_DECODE_SHAPE", 6),
     ("W4A8_GEMM_PREFILL_SHAPE", 1), ("W4A8_GEMM_PREFILL_SHAPE", 2),
     ("W4A8_GEMM_PREFILL_SHAPE", 3), ("W4A8_GEMM_PREFILL_SHAPE", 4),
 ], ids=lambda v: str(v))

@@ -24,7 +24,10 @@ __all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_ab
            "w4a8_moe_route_topk", "w4a8_moe_experts_workspace_size", "w4a8_moe_forward_experts",
            "w4a8_cast_f32_bf16"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4a8.so")
+# W4A8_LIBRARY=debug selects the bounds-checking build (see build.py)
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libw4a8_debug.so" if os.environ.get("W4A8_LIBRARY") == "debug"
+                        else "libw4a8.so")
 NUM_STAGES = 6
 STAGE_NAMES = ["act_quant", "route_permute", "gemm_gate_up", "inter_quant", "gemm_down",
                "combine"]
@@ -61,6 +64,7 @@ def _declare(L):
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     sig = {
         "w4a8_abi_version": (i32, []),
+        "w4a8_build_flags": (i32, []),
         "w4a8_status_string": (ctypes.c_char_p, [i32]),
         "w4a8_last_error": (ctypes.c_char_p, []),
         "w4a8_check_device_error": (i32, [vp]),
@@ -105,7 +109,8 @@ def lib():
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"{LIB_PATH} is missing; build it with "
-                               "`python -m w4a8_quantized_moe_b200.build`")
+                               "`python -m w4a8_quantized_moe_b200.build` (add "
+                               "--debug-bounds for the checking build)")
         L = ctypes.CDLL(LIB_PATH)
         _declare(L)
         _lib = L
@@ -147,6 +152,11 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
 
 def w4a8_abi_version() -> int:
     return int(lib().w4a8_abi_version())
+
+
+def w4a8_build_flags() -> int:
+    """Bit 0: the loaded library is the bounds-checking build."""
+    return int(lib().w4a8_build_flags())
 
 
 def w4a8_status_string(status: int) -> str:

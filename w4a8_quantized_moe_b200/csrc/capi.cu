@@ -287,6 +287,14 @@ extern "C" {
 
 int32_t w4a8_abi_version(void) { return 1; }
 
+int32_t w4a8_build_flags(void) {
+#if W4A8_DEBUG_BOUNDS
+  return W4A8_BUILD_DEBUG_BOUNDS;
+#else
+  return 0;
+#endif
+}
+
 const char* w4a8_status_string(w4a8_status s) {
   switch (s) {
     case W4A8_OK: return "W4A8_OK";
@@ -517,6 +525,8 @@ w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_code
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
   g1.nb_fastest = 1;
+  g1.n_seg_rows = T;
+  g1.n_tokens = T;
   const int ctas1 = static_cast<int>(std::min<int64_t>(tiles_n * (I / 64), di.sms));
   W4A8_STEP(record(2), "cudaEventRecord");
   W4A8_STEP(launch_fp8_block_gemm(true, tw1, ta1, g1, ctas1, s), "shared gate/up GEMM launch");
@@ -722,6 +732,8 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
   g1.nb_fastest = tile_order_nb_fastest(decode);
+  g1.n_seg_rows = A;
+  g1.n_tokens = T;
   g1.wsum = i8 ? i8->w13_nsum : nullptr;
   g1.act_sum = b.act_rowsum;
   W4A8_STEP(record(4), "cudaEventRecord");
@@ -754,6 +766,8 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   g2.act_rows = A;
   g2.timeout_ns = wait_timeout_ns();
   g2.nb_fastest = tile_order_nb_fastest(decode);
+  g2.n_seg_rows = A;
+  g2.n_tokens = T;
   g2.wsum = i8 ? i8->w2_nsum : nullptr;
   g2.act_sum = b.inter_rowsum;
   W4A8_STEP(record(8), "cudaEventRecord");
@@ -1047,7 +1061,7 @@ w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_
                                di.sms, s),
             "local routing launch");
   const int32_t* rows_total = b.expert_offsets + e_count;
-  W4A8_STEP(launch_ep_gather(act_codes, H, b.sorted_token_ids, rows_total, A, b.perm_codes,
+  W4A8_STEP(launch_ep_gather(act_codes, T, H, b.sorted_token_ids, rows_total, A, b.perm_codes,
                              parts ? nullptr : b.act_gsum, parts ? b.act_parts : nullptr, di.sms, s),
             "dispatch gather launch");
 
@@ -1068,6 +1082,8 @@ w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_
   g1.act_rows = T;
   g1.timeout_ns = wait_timeout_ns();
   g1.nb_fastest = tile_order_nb_fastest(decode);
+  g1.n_seg_rows = A;
+  g1.n_tokens = T;
   W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
             "gate/up GEMM launch");
   W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales,

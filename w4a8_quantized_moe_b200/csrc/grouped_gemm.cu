@@ -84,7 +84,8 @@ constexpr int kWStageBytes = kBM * kGroup / 2;      // 8 KB of packed INT4
 constexpr uint32_t kTmemCols = 512;
 
 template <int TileN, int WStages, int BStages, int ASlots, int DBufs, int ConvSets,
-          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetMode, int Pair = 0>
+          int EpiPerQuad, int LdCols, int MmaWarps, int EpiSets, int OffsetMode, int Pair = 0,
+          int Cta2 = 0>
 struct Shape {
   static constexpr int kTileN = TileN;
   static constexpr int kWStages = WStages;
@@ -112,6 +113,11 @@ struct Shape {
   // commit is shared by two groups.  K / 128 must be even.
   static constexpr bool kPair = Pair != 0;
   static constexpr int kGPU = kPair ? 2 : 1;              // groups per ring element
+  // CTA pairs (cta_group::2): a cluster of two CTAs shares each tile, M = 256
+  // weight rows, 128 in each CTA's TMEM; the tile's N token rows are split
+  // between the two CTAs' activation stages; the first CTA issues the MMAs.
+  static constexpr bool kCta2 = Cta2 != 0;
+  static constexpr int kTileNLocal = kCta2 ? TileN / 2 : TileN;  // activation rows per CTA
   static constexpr int kEpiPerSet = 4 * EpiPerQuad;
   static constexpr int kEpiWarps = kEpiPerSet * EpiSets;
   static constexpr int kWarpW = kConvWarps + kEpiWarps;   // TMA: packed weights
@@ -121,7 +127,7 @@ struct Shape {
   static constexpr bool kUnified = ASlots == BStages && BStages == DBufs;
   static constexpr int kThreads = 32 * ((kWarpB + 1 + 3) / 4 * 4);
   static constexpr int kEpiN = TileN / EpiPerQuad;        // columns per epilogue warp
-  static constexpr int kBStageBytes = TileN * kGroup * kGPU;
+  static constexpr int kBStageBytes = kTileNLocal * kGroup * kGPU;
   static constexpr int kUpBytes = 64 * TileN * 4;         // up-projection exchange
   static constexpr int kSumLd = kEpiN + 4;                // padded: 4-way bank spread on stores
   static constexpr int kTileScBufs = 2;                   // tile weight-scale buffers
@@ -135,6 +141,8 @@ struct Shape {
   static_assert(kTmemD + DBufs * kDCols <= kTmemCols, "TMEM budget exceeded");
   static_assert(!kPair || (kEpiOffset && kUnified && ConvSets == 1),
                 "paired groups: epilogue offset, unified rings, one converter set");
+  static_assert(!kCta2 || (kPair && TileN == 32),
+                "CTA pairs: the paired decode shapes (N = 32, 16 token rows per CTA)");
   static_assert(kEpiN % 32 == 0 && kEpiN % LdCols == 0 && (LdCols == 16 || LdCols == 32),
                 "epilogue load width");
   static_assert(TileN % 16 == 0 && TileN <= 256, "MMA N");
@@ -170,6 +178,9 @@ using DecodeTwoCvt  = Shape<kTileNDecode, 12, 8, 8, 8, 2, 1, 32, 2, 2, 0>;
 using DecodeTileCorr = Shape<kTileNDecode, 16, 8, 8, 7, 1, 1, 32, 2, 1, 2>;
 using DecodePair = Shape<kTileNDecode, 16, 4, 4, 4, 1, 1, 32, 2, 1, 0, 1>;  // 2 groups per element
 using DecodePairTwoSets = Shape<kTileNDecode, 12, 4, 4, 4, 1, 1, 32, 2, 2, 0, 1>;
+// the paired shapes on CTA pairs (cta_group::2, M = 256)
+using DecodePair2 = Shape<kTileNDecode, 16, 4, 4, 4, 1, 1, 32, 2, 1, 0, 1, 1>;
+using DecodePairTwoSets2 = Shape<kTileNDecode, 12, 4, 4, 4, 1, 1, 32, 2, 2, 0, 1, 1>;
 using Prefill16Epi  = Shape<kTileNPrefill, 4, 5, 3, 3, 1, 4, 16, 2, 1, 1>;
 using Prefill8Epi   = Shape<kTileNPrefill, 4, 5, 3, 2, 1, 2, 16, 2, 1, 1>;
 using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 0>;
@@ -245,6 +256,19 @@ __device__ __forceinline__ float column_max32(float (&v)[N], int off, int lane) 
   return w[0];
 }
 
+// The token a gate/up segment row reads its scale and group sums from.  The
+// debug build checks it against the token count (raising the latch's index
+// bit and reading token 0 instead); the release build trusts the permutation.
+__device__ __forceinline__ int checked_token(const GemmArgs& a, int t) {
+#if W4A8_DEBUG_BOUNDS
+  if (t < 0 || t >= a.n_tokens) {
+    atomicOr(&g_device_error, kDeviceErrorIndex);
+    return 0;
+  }
+#endif
+  return t;
+}
+
 // Wait used only while draining: ignores the abort flag, still bounded.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
                                                 uint64_t timeout_ns) {
@@ -314,8 +338,19 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mb_count = kGateUp ? a.half_rows / 64 : a.n_rows / kBM;
+  constexpr bool kCta2 = S::kCta2;
+  // CTA pairs: both CTAs of a cluster walk the same tiles (cta_x of n_cta);
+  // this CTA takes weight-row block 2 mb + crank of the pair's block mb
+  const uint32_t crank = kCta2 ? cluster_ctarank() : 0u;
+  const int cta_x = kCta2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_cta = kCta2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int mb_count = (kGateUp ? a.half_rows / 64 : a.n_rows / kBM) / (kCta2 ? 2 : 1);
   const uint64_t tmo = a.timeout_ns;
+  auto tile_at = [&](int idx) -> Tile {
+    Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, idx);
+    if (kCta2) t.mb = 2 * t.mb + static_cast<int>(crank);
+    return t;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kWStages; ++s) {
@@ -327,12 +362,13 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       if (!kUniAB) mbar_init(&bempty[s], 1);
     }
     for (int s = 0; s < kASlots; ++s) {
-      mbar_init(&afull[s], 4);
+      mbar_init(&afull[s], kCta2 ? 8 : 4);  // pairs: both CTAs' converter warps (first CTA's)
       mbar_init(&aempty[s], 1);
     }
     for (int d = 0; d < kDBufs; ++d) {
       if (!kUniAll) mbar_init(&dfull[d], kI8 ? S::kMmaWarps : 1);
-      mbar_init(&dempty[d], S::kEpiPerSet);   // each group is read by one set
+      // each group is read by one set (of both CTAs of a pair, on the first CTA's barrier)
+      mbar_init(&dempty[d], S::kEpiPerSet * (kCta2 ? 2 : 1));
     }
     for (int i = 0; i < S::kEpiSets; ++i) {
       mbar_init(&upfull[i], S::kEpiPerSet / 2);
@@ -362,19 +398,43 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     if (S::kOffsetTile) prefetch_tmap(&tmap_gs);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
+    if constexpr (kCta2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+      tmem_relinquish();
+    }
   }
   for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
     sTP[i] = __ldg(a.tile_prefix + i);
     sEO[i] = __ldg(a.expert_offsets + i);
   }
+#if W4A8_DEBUG_BOUNDS
+  // debug build: the expert tables decide every row this CTA touches; if they
+  // are not a valid segment table of the shape's tiles within the buffers,
+  // raise the latch's index bit and run no tile
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool good = sEO[0] == 0 && sTP[0] == 0 && sEO[a.E] <= a.n_seg_rows;
+    for (int e = 0; good && e < a.E; ++e) {
+      const int cnt = sEO[e + 1] - sEO[e];
+      good = cnt >= 0 && sTP[e + 1] - sTP[e] == (cnt + kTileN - 1) / kTileN;
+    }
+    if (!good) {
+      atomicOr(&g_device_error, kDeviceErrorIndex);
+      for (int e = 0; e <= a.E; ++e) sTP[e] = 0;
+    }
+  }
+#endif
   tc_fence_before();
   __syncthreads();
+  // pairs: the other CTA's barriers are initialised before anything arrives on them
+  if constexpr (kCta2) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int total = sTP[a.E] * mb_count;
-  const int my_tiles = blockIdx.x < total ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const int my_tiles = cta_x < total ? (total - cta_x + n_cta - 1) / n_cta : 0;
   const int n_groups = my_tiles * G;  // every tile has G groups
   // Per-tile correction (offset mode 2): the rows' group sums S_g come as three
   // bf16 parts, [rows][3 * Gp] with Gp = G rounded up to 16 (padding zero);
@@ -393,8 +453,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     if (lane == 0) {
       int it = 0, nt = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++nt) {
-        const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
+      for (int tile = cta_x; ok && tile < total; tile += n_cta, ++nt) {
+        const Tile t = tile_at(tile);
         const int32_t wy0 = t.e * a.n_rows + (kGateUp ? t.mb * 64 : t.mb * kBM);
         const int32_t wy1 = t.e * a.n_rows + a.half_rows + t.mb * 64;
         if constexpr (!kI8 && !kF8W) {  // the tile's weight scales: box [G groups x 128 (or 2 x 64) rows] of bf16
@@ -441,13 +501,35 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     // ------------------------------------------------------------ TMA: activation rows
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
+    for (int tile = cta_x; ok && tile < total; tile += n_cta) {
+      const Tile t = tile_at(tile);
       // the activations are in segment order: the tile's rows are contiguous,
       // loaded as 16-row boxes (rows past the tensor's end read as zero)
       const int n_ops = t.n_mma >> 4;
       const uint32_t tx = t.n_mma * kGroup;
       const int32_t y0 = static_cast<int32_t>(t.row0) + 16 * lane;
+      if constexpr (kCta2) {
+        // pairs: this CTA's 16 of the tile's 32 rows, for each group of the
+        // element; the copies of both CTAs complete on the first CTA's barrier,
+        // which the first CTA expects for both
+        const int32_t yp = static_cast<int32_t>(t.row0) + 16 * static_cast<int32_t>(crank);
+        for (int g = 0; g < ab_per_tile; ++g) {
+          const int s = it % kBStages;
+          const uint32_t ph = (it / kBStages) & 1;
+          if (!mbar_wait(&bempty[s], ph ^ 1, abort_flag, tmo)) { ok = false; break; }
+          if (lane == 0) {
+            const uint32_t dB = smem_u32(sB + s * kBStageBytes);
+            const uint32_t bar0 = mapa_shared(smem_u32(&bfull[s]), 0);
+            if (crank == 0) mbar_arrive_expect_tx(&bfull[s], 2 * kBStageBytes);
+#pragma unroll
+            for (int h = 0; h < kGPU; ++h)
+              tma_load_2d_pair(dB + h * (16 * kGroup), &tmap_act, bar0, (g * kGPU + h) * kGroup, yp);
+          }
+          __syncwarp();
+          ++it;
+        }
+        continue;
+      }
       // G stages of codes (kGPU groups per stage, each in its own kTileN-row
       // half), then (per-tile correction) kNC stages of the bf16 group-sum
       // parts, 128 bytes of each row per stage
@@ -472,7 +554,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         ++it;
       }
     }
-    if (lane == 0)
+    // (pairs: the first CTA's barriers count both CTAs' copies)
+    if (lane == 0 && crank == 0)
       for (int i = (it > kBStages ? it - kBStages : 0); i < it; ++i)
         mbar_wait_drain(&bfull[i % kBStages], (i / kBStages) & 1, tmo);
     __syncwarp();
@@ -497,8 +580,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           if (tl != cur_tile) {  // this chain's first group of the tile
             cur_tile = tl;
             first = true;
-            const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest,
-                                               blockIdx.x + tl * gridDim.x);
+            const Tile t = tile_at(cta_x + tl * n_cta);
             idesc = idesc_u8_s32_m128(static_cast<uint32_t>(t.n_mma));
             dcur = tl % kTileSlots;
             if (!mbar_wait(&dempty[dcur], ((tl / kTileSlots) & 1) ^ 1, abort_flag, tmo)) break;
@@ -539,8 +621,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           const int tl = it / G;
           if (tl != cur) {
             cur = tl;
-            const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest,
-                                               blockIdx.x + tl * gridDim.x);
+            const Tile t = tile_at(cta_x + tl * n_cta);
             idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
           }
           const int ws = it % kWStages;
@@ -568,6 +649,44 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         tc_commit(drain);
         mbar_wait_drain(drain, 0, tmo);
       }
+    } else if (kCta2 && lane == 0) {
+      // CTA pairs: the first CTA issues every MMA of the pair (M = 256, N = 32),
+      // after both CTAs' converted weights, both halves of the activation rows
+      // and both CTAs' epilogues are ready (cluster-scope waits on its own
+      // barriers); one commit signals the A slot / stage / accumulator barrier
+      // of both CTAs.  The second CTA's issuers have nothing to do.
+      if (crank == 0) {
+        const uint32_t idesc = idesc_e4m3_f32_m256(static_cast<uint32_t>(kTileN));
+        for (int it = mw; it < n_units; it += S::kMmaWarps) {
+          const int d = it % kDBufs;
+          const uint32_t phd = (it / kDBufs) & 1;
+          const int as = it % kASlots;               // unified: A slot = B stage = accumulator
+          const uint32_t pha = (it / kASlots) & 1;
+          const bool rd = mbar_test_wait_cluster(&dempty[d], phd ^ 1);
+          const bool rb = mbar_test_wait_cluster(&bfull[as], pha);
+          const bool ra = mbar_test_wait_cluster(&afull[as], pha);
+          if (!(rd && rb && ra) &&
+              (!mbar_wait_cluster(&dempty[d], phd ^ 1, abort_flag, tmo) ||
+               !mbar_wait_cluster(&bfull[as], pha, abort_flag, tmo) ||
+               !mbar_wait_cluster(&afull[as], pha, abort_flag, tmo)))
+            break;
+          tc_fence_after();
+          const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB + as * kBStageBytes));
+          const uint32_t dt0 = tmem + kTmemD + d * S::kDCols;
+          const uint32_t at0 = tmem + kTmemA + as * S::kACols;
+#pragma unroll
+          for (int h = 0; h < kGPU; ++h) {
+            const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(h * (16 * kGroup / 16));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8_ts_pair(dt0 + h * kTileN, at0 + h * 32 + kk * 8,
+                             bdesc + static_cast<uint64_t>(kk * 2), idesc, kk > 0 ? 1u : 0u);
+          }
+          tc_commit_pair_multicast(&aempty[as], static_cast<uint16_t>(0x3));
+        }
+        tc_commit_pair(drain);
+        mbar_wait_drain(drain, 0, tmo);
+      }
     } else if (lane == 0) {
       int cur = -1;
       uint32_t idesc = 0, idesc_c = 0;
@@ -578,7 +697,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const int u = it - tl * units_per_tile;
         if (tl != cur) {
           cur = tl;
-          const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, blockIdx.x + tl * gridDim.x);
+          const Tile t = tile_at(cta_x + tl * n_cta);
           idesc = idesc_e4m3_f32_m128(static_cast<uint32_t>(t.n_mma));
           idesc_c = idesc_bf16_f32_m128(static_cast<uint32_t>(t.n_mma));
         }
@@ -714,7 +833,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
       if (last) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[as]);
+        if (lane == 0) {
+          if constexpr (kCta2)  // the first CTA of the pair issues the MMAs
+            mbar_arrive_cluster(mapa_shared(smem_u32(&afull[as]), 0));
+          else
+            mbar_arrive(&afull[as]);
+        }
       }
       return true;
     };
@@ -789,9 +913,9 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     const int sc_off = kGateUp ? (m < 64 ? m : 64 * G + (m - 64)) : m;
     constexpr int kScStride = kGateUp ? 64 : 128;
     bool ok = true;
-    for (int tile = blockIdx.x + set * gridDim.x, ntile = set; ok && tile < total;
-         tile += S::kEpiSets * gridDim.x, ntile += S::kEpiSets) {
-      const Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, tile);
+    for (int tile = cta_x + set * n_cta, ntile = set; ok && tile < total;
+         tile += S::kEpiSets * n_cta, ntile += S::kEpiSets) {
+      const Tile t = tile_at(tile);
       int it = ntile * units_per_tile;              // CTA-wide index of the tile's first unit
       const uint32_t lt = ntile / S::kEpiSets;      // this set's tile count: barrier phases
       // token (gate/up) or row (down) scales of this warp's columns, lane-strided;
@@ -804,7 +928,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         if (j < t.n_valid) {
           const int64_t r = t.row0 + j;
           if constexpr (kF8W) v = 1.0f;  // scales are per group, applied in the promotion
-          else v = kGateUp ? __ldg(a.act_scale + __ldg(a.row_tokens + r)) : __ldg(a.act_scale + r);
+          else v = kGateUp ? __ldg(a.act_scale + checked_token(a, __ldg(a.row_tokens + r)))
+                           : __ldg(a.act_scale + r);
         }
         ts[i] = v;
       }
@@ -825,7 +950,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           int v = 0;
           if (j < t.n_valid) {
             const int64_t r = t.row0 + j;
-            v = kGateUp ? __ldg(a.act_sum + __ldg(a.row_tokens + r)) : __ldg(a.act_sum + r);
+            v = kGateUp ? __ldg(a.act_sum + checked_token(a, __ldg(a.row_tokens + r)))
+                        : __ldg(a.act_sum + r);
           }
           asum[i] = v;
         }
@@ -874,7 +1000,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kBatch; ++i) {
             const int j = j0 + q * kTok + b0 + i;
-            key[i] = j < t.n_valid ? ((kGateUp && !kF8W) ? __ldg(a.row_tokens + t.row0 + j)
+            key[i] = j < t.n_valid ? ((kGateUp && !kF8W) ? checked_token(a, __ldg(a.row_tokens + t.row0 + j))
                                                          : static_cast<int>(t.row0 + j))
                                    : -1;
           }
@@ -968,7 +1094,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dempty[d]);
+        if (lane == 0) {
+          if constexpr (kCta2)  // the first CTA of the pair reuses the accumulator
+            mbar_arrive_cluster(mapa_shared(smem_u32(&dempty[d]), 0));
+          else
+            mbar_arrive(&dempty[d]);
+        }
         ++it;
         if (++d == kDBufs) {  // accumulator ring position, kept incrementally
           d = 0;
@@ -1059,9 +1190,13 @@ __global__ void __launch_bounds__(S::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // pairs: the first CTA's MMAs read and write both CTAs' TMEM and the CTAs
+  // arrive on each other's barriers: neither frees or exits before both are done
+  if constexpr (kCta2) cluster_sync();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    if constexpr (kCta2) tmem_dealloc_pair(tmem, kTmemCols);
+    else tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -1085,6 +1220,22 @@ cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
     if (dev < 64) attr_set[dev] = true;
   }
   const int smem = S::smem_bytes(kGateUp, a.K / kGroup, a.E, kF8W);
+  if constexpr (S::kCta2) {  // clusters of two CTAs on SM pairs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(num_ctas & ~1), 1, 1);
+    cfg.blockDim = dim3(S::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<S, kGateUp, kI8, kF8W>, tmap_w, tmap_act,
+                              tmap_sc, tmap_gs, a);
+  }
   grouped_gemm_kernel<S, kGateUp, kI8, kF8W><<<num_ctas, S::kThreads, smem, s>>>(
       tmap_w, tmap_act, tmap_sc, tmap_gs, a);
   return cudaGetLastError();
@@ -1135,10 +1286,17 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
     // groups (two per ring element) when K / 128 is even.
     const bool even = (a.K / kGroup) % 2 == 0;
     const int d = dshape != 0 ? dshape : (even ? 5 : (gate_up ? 1 : 2));
+    // 6: the paired shapes on CTA pairs; a pair covers 128 gate (+ 128 up) or
+    // 256 down rows, so those counts must divide the rows
+    const bool pairs_fit = even && num_ctas >= 2 &&
+                           (gate_up ? a.half_rows % 128 == 0 : a.n_rows % 256 == 0);
+    if (d == 6 && pairs_fit)
+      return gate_up ? launch_either<DecodePair2>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s)
+                     : launch_either<DecodePairTwoSets2>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     if (d == 1) return launch_either<DecodeOneSet>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     if (d == 3) return launch_either<DecodeTwoCvt>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     if (d == 4) return launch_either<DecodeTileCorr>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
-    if (d == 5 && (a.K / kGroup) % 2 == 0)
+    if ((d == 5 || d == 6) && even)   // (6 without a pair fit: the same shapes on one CTA)
       return gate_up ? launch_either<DecodePair>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s)
                      : launch_either<DecodePairTwoSets>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
     return launch_either<DecodeTwoSets>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);

@@ -67,9 +67,10 @@ cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, in
 // Segment row r < *rows_total (device) receives the codes of token
 // sorted_token_ids[r]; the group sums go to gsum [T, H / 128] by token, or to
 // the row's three-part sums (sum_parts, [max_rows, sum_parts_ld(H)]).
-cudaError_t launch_ep_gather(const uint8_t* codes, int64_t H, const int32_t* sorted_token_ids,
-                             const int32_t* rows_total, int64_t max_rows, uint8_t* perm,
-                             float* gsum, uint16_t* sum_parts, int num_sms, cudaStream_t s);
+cudaError_t launch_ep_gather(const uint8_t* codes, int64_t T, int64_t H,
+                             const int32_t* sorted_token_ids, const int32_t* rows_total,
+                             int64_t max_rows, uint8_t* perm, float* gsum, uint16_t* sum_parts,
+                             int num_sms, cudaStream_t s);
 // bf16 = round-to-nearest-even(x), n a multiple of 8.
 cudaError_t launch_cast_bf16(const float* x, int64_t n, void* out, int num_sms, cudaStream_t s);
 // sum_parts (nullable): [A, sum_parts_ld(I)] bf16 as for launch_act_quant.
@@ -130,6 +131,11 @@ struct GemmArgs {
   const int32_t* wsum;            // [E, n_rows] sum over K of the stored nibbles u = q + 8
   const int32_t* act_sum;         // per token (gate/up) or row (down): sum of code + 128
   uint64_t timeout_ns;
+  // buffer bounds for the debug build's index checks (W4A8_DEBUG_BOUNDS): the
+  // segment rows of the activation / output tensors, and the tokens row_tokens
+  // may name
+  int64_t n_seg_rows;
+  int64_t n_tokens;
 };
 // decode = the shape for few tokens per expert (see grouped_gemm.cu).
 // tmap_sc: the group-major weight scales as bytes [E * K / 128, 2 * n_rows],

@@ -14,6 +14,17 @@
 
 namespace w4a8 {
 
+// Bounds checks of routing-derived indices (the debug build, compiled with
+// W4A8_DEBUG_BOUNDS=1): an index outside its buffer raises the device latch's
+// index bit and the access is skipped.  The release build compiles them out.
+#if W4A8_DEBUG_BOUNDS
+__device__ int* g_debug_latch = nullptr;
+#define W4A8_IN_BOUNDS(cond) \
+  ((cond) ? true : (atomicOr(::w4a8::g_debug_latch, ::w4a8::kDeviceErrorIndex), false))
+#else
+#define W4A8_IN_BOUNDS(cond) true
+#endif
+
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -156,7 +167,11 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
       amax = fmaxf(amax, absmax8(__ldg(row + c)));
     amax = warp_max(amax);
     if (lane == 0) red[warp] = amax;
-    if (perm && threadIdx.x < k) dst_rows[threadIdx.x] = __ldg(row_of + t * k + threadIdx.x);
+    if (perm && threadIdx.x < k) {
+      int64_t r = __ldg(row_of + t * k + threadIdx.x);
+      if (!W4A8_IN_BOUNDS(r >= 0 && r < T * k)) r = -1;
+      dst_rows[threadIdx.x] = r;
+    }
     __syncthreads();
     amax = red[0];
 #pragma unroll
@@ -179,7 +194,8 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
         const uint2 q = kInt8 ? quant8_i8(v, scale) : quant8(v, scale);
         out[c] = q;
         if (perm)  // the token's codes again at each of its k segment rows
-          for (int j = 0; j < k; ++j) reinterpret_cast<uint2*>(perm + dst_rows[j] * H)[c] = q;
+          for (int j = 0; j < k; ++j)
+            if (dst_rows[j] >= 0) reinterpret_cast<uint2*>(perm + dst_rows[j] * H)[c] = q;
         if (kInt8) isum += sum8_u8(q);
         if (want_sums) part = sum8_e4m3(q);
       }
@@ -192,7 +208,8 @@ __global__ void __launch_bounds__(kAqThreads) act_quant_kernel(const __nv_bfloat
           if (gs) gs[c >> 4] = part;
           if (parts)
             for (int j = 0; j < k; ++j)
-              store_sum_parts(parts + dst_rows[j] * sum_parts_ld(H), part, static_cast<int>(c >> 4), G, gp);
+              if (dst_rows[j] >= 0)
+                store_sum_parts(parts + dst_rows[j] * sum_parts_ld(H), part, static_cast<int>(c >> 4), G, gp);
         }
       }
     };
@@ -514,6 +531,10 @@ __global__ void __launch_bounds__(kRouteTok) route_scatter_kernel(
       int rank = __popc(mask[warp * E + e] & lt_mask);
       for (int w = 0; w < warp; ++w) rank += __popc(mask[w * E + e]);
       const int row = base[e] + rank;
+      if (!W4A8_IN_BOUNDS(row >= 0 && row < T * k)) {
+        row_of[t * k + j] = -1;
+        continue;
+      }
       row_of[t * k + j] = row;
       sorted_token_ids[row] = static_cast<int32_t>(t);
       if (row_amax) row_amax[row] = 0u;
@@ -552,7 +573,7 @@ __global__ void __launch_bounds__(256) route_ids_hist_kernel(const int32_t* __re
 // remove the nibble offset once per tile, to the row's three bf16 parts.
 // One warp per row, 16 bytes per lane per step.
 __global__ void __launch_bounds__(256) ep_gather_kernel(const uint8_t* __restrict__ codes,
-                                                        int64_t H,
+                                                        int64_t T, int64_t H,
                                                         const int32_t* __restrict__ sorted_token_ids,
                                                         const int32_t* __restrict__ rows_total,
                                                         uint8_t* __restrict__ perm,
@@ -566,6 +587,7 @@ __global__ void __launch_bounds__(256) ep_gather_kernel(const uint8_t* __restric
   for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < A;
        r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
     const int64_t t = __ldg(sorted_token_ids + r);
+    if (!W4A8_IN_BOUNDS(t >= 0 && t < T)) continue;   // warp-uniform
     const uint4* src = reinterpret_cast<const uint4*>(codes + t * H);
     uint4* dst = reinterpret_cast<uint4*>(perm + r * H);
     for (int64_t base = 0; base < nchunk; base += 32) {   // warp-uniform trip count
@@ -808,6 +830,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     for (int j = 0; j < k; ++j) {
       const int64_t r = __ldg(row_of + t * k + j);
       if (kPartial && r < 0) continue;
+      if (!W4A8_IN_BOUNDS(r >= 0 && r < T * k)) continue;
       const float wj = __ldg(topk_w + t * k + j);
       const float4* src = reinterpret_cast<const float4*>(y + r * H + c * 8);
       const float4 a = __ldg(src), b = __ldg(src + 1);
@@ -838,6 +861,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   }
 }
 
+// Debug build: point g_debug_latch at the library's device error latch (once
+// per device, before the first checked kernel).  Release build: nothing.
+cudaError_t ensure_debug_latch() {
+#if W4A8_DEBUG_BOUNDS
+  static int* done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int* latch = nullptr;
+  err = device_error_latch(&latch);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && done[dev] == latch) return cudaSuccess;
+  err = cudaMemcpyToSymbol(g_debug_latch, &latch, sizeof(latch));
+  if (err == cudaSuccess && dev < 64) done[dev] = latch;
+  return err;
+#else
+  return cudaSuccess;
+#endif
+}
+
 inline int grid_for(int64_t work_items, int threads, int num_sms, int per_sm = 8) {
   int64_t g = (work_items + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
@@ -853,6 +896,7 @@ cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes
   if (T == 0) return cudaSuccess;
   if (perm && (!row_of || k < 1 || k > kMaxTopK)) return cudaErrorInvalidValue;
   if (sum_parts && (!perm || int8_row_sum)) return cudaErrorInvalidValue;
+  if (cudaError_t err = ensure_debug_latch()) return err;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(T < cap ? T : cap);
   if (int8_row_sum)
@@ -885,6 +929,7 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                          int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
                          cudaStream_t s) {
+  if (cudaError_t err = ensure_debug_latch()) return err;
   const int64_t nblk = route_blocks(T);
   if (nblk > 0) {
     cudaError_t err = cudaMemsetAsync(block_counts, 0,
@@ -942,6 +987,7 @@ cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, in
                                int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                                int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
                                int* latch, int num_sms, cudaStream_t s) {
+  if (cudaError_t err = ensure_debug_latch()) return err;
   const int64_t nblk = route_blocks(T);
   if (nblk > 0) {
     cudaError_t err = cudaMemsetAsync(block_counts, 0,
@@ -962,12 +1008,14 @@ cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_ep_gather(const uint8_t* codes, int64_t H, const int32_t* sorted_token_ids,
-                             const int32_t* rows_total, int64_t max_rows, uint8_t* perm,
-                             float* gsum, uint16_t* sum_parts, int num_sms, cudaStream_t s) {
+cudaError_t launch_ep_gather(const uint8_t* codes, int64_t T, int64_t H,
+                             const int32_t* sorted_token_ids, const int32_t* rows_total,
+                             int64_t max_rows, uint8_t* perm, float* gsum, uint16_t* sum_parts,
+                             int num_sms, cudaStream_t s) {
   if (max_rows == 0) return cudaSuccess;
+  if (cudaError_t err = ensure_debug_latch()) return err;
   ep_gather_kernel<<<grid_for(max_rows * 32, 256, num_sms), 256, 0, s>>>(
-      codes, H, sorted_token_ids, rows_total, perm, gsum, sum_parts);
+      codes, T, H, sorted_token_ids, rows_total, perm, gsum, sum_parts);
   return cudaGetLastError();
 }
 
@@ -1040,6 +1088,7 @@ cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* t
                            int64_t H, int k, void* out, int num_sms, cudaStream_t s,
                            const float* y_shared, float* partial_f32) {
   if (T == 0) return cudaSuccess;
+  if (cudaError_t err = ensure_debug_latch()) return err;
   const int grid = grid_for(T * (H / 8), 256, num_sms);
   if (partial_f32)
     combine_kernel<true><<<grid, 256, 0, s>>>(y, row_of, topk_w, T, H, k, nullptr, nullptr,
