@@ -282,6 +282,17 @@ typedef struct w4a8_moe_aux {
 } w4a8_moe_aux;
 
 /*
+ * w4a8_moe_forward_launches - how many kernels one w4a8_moe_forward launches
+ * for T tokens, E experts and top-k: 8, or 10 when the batch averages at
+ * least 8 assignments per expert and each grouped GEMM runs as two launches
+ * ("split tiling": experts with more than 32 segment rows in 128-row tiles,
+ * the others in 32-row tiles; W4A8_SPLIT_TILES=0/1 forces it off/on).  The
+ * per-channel INT8 variant never splits (8).  Host arithmetic only; 0 for
+ * T <= 0.
+ */
+W4A8_API int32_t w4a8_moe_forward_launches(int64_t T, int32_t E, int32_t k);
+
+/*
  * w4a8_moe_workspace_size - bytes of scratch w4a8_moe_forward needs.
  */
 W4A8_API size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k);

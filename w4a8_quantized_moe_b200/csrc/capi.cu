@@ -98,14 +98,16 @@ struct RouteBufs {
   int32_t* block_counts;
   int32_t* block_base;
   int32_t* tile_prefix;
+  int32_t* tile_prefix_wide;  // split tiling: the wide-tile table
 };
 
-RouteBufs carve_route(Carver& c, int64_t T, int E) {
+RouteBufs carve_route(Carver& c, int64_t T, int E, bool wide_table = false) {
   RouteBufs b;
   const size_t n = static_cast<size_t>(route_blocks(T)) * static_cast<size_t>(E);
   b.block_counts = c.take<int32_t>(n);
   b.block_base = c.take<int32_t>(n);
   b.tile_prefix = c.take<int32_t>(static_cast<size_t>(E) + 1);
+  b.tile_prefix_wide = wide_table ? c.take<int32_t>(static_cast<size_t>(E) + 1) : nullptr;
   return b;
 }
 
@@ -140,7 +142,7 @@ ForwardBufs carve_forward(Carver& c, int64_t T, int64_t H, int64_t I, int E, int
   b.expert_offsets = c.take<int32_t>(static_cast<size_t>(E) + 1);
   b.sorted_token_ids = c.take<int32_t>(A);
   b.row_of = c.take<int32_t>(A);
-  b.route = carve_route(c, T, E);
+  b.route = carve_route(c, T, E, true);
   b.act_codes = c.take<uint8_t>(static_cast<size_t>(T) * static_cast<size_t>(H));
   b.perm_codes = c.take<uint8_t>(A * static_cast<size_t>(H));
   b.act_scales = c.take<float>(static_cast<size_t>(T));
@@ -228,6 +230,40 @@ int tile_order_nb_fastest(bool decode) {
 
 // Average tokens per expert up to which w4a8_moe_forward uses the decode shape.
 constexpr int kDecodeTokensPerExpert = 32;
+
+// Split tiling: from this many assignments per expert on average, the experts
+// with more than kTileNDecode segment rows run in the wide (prefill) tile
+// shape and the rest in the narrow (decode) shape, as two launches of each
+// grouped GEMM (a skewed batch has both kinds).  W4A8_SPLIT_TILES = 0 / 1
+// turns it off / on for every batch.
+constexpr int kSplitTokensPerExpert = 8;
+
+bool split_tiles(int64_t A, int64_t E) {
+  static const int forced = [] {
+    const char* v = std::getenv("W4A8_SPLIT_TILES");
+    return v ? std::atoi(v) : -1;
+  }();
+  // a forced shape that removes the offset once per tile needs per-row group
+  // sums that only one regime's quantisers write: no split then
+  if (grouped_gemm_uses_sum_parts(true) || grouped_gemm_uses_sum_parts(false)) return false;
+  if (forced >= 0) return forced != 0;
+  return A >= static_cast<int64_t>(kSplitTokensPerExpert) * E;
+}
+
+// Both launches of one grouped GEMM under split tiling: the narrow-tile
+// (decode) shape over the experts with tiles in a.tile_prefix, then the
+// wide-tile (prefill) shape over those in tile_prefix_wide.
+cudaError_t launch_grouped_gemm_split(bool gate_up, const CUtensorMap& tw, const CUtensorMap& ta,
+                                      const CUtensorMap& tsc, const CUtensorMap& tgs,
+                                      const GemmArgs& a, const int32_t* tile_prefix_wide,
+                                      int num_sms, cudaStream_t s) {
+  cudaError_t err = launch_grouped_gemm(gate_up, true, tw, ta, tsc, tgs, a, num_sms, s);
+  if (err != cudaSuccess) return err;
+  GemmArgs w = a;
+  w.tile_prefix = tile_prefix_wide;
+  w.nb_fastest = tile_order_nb_fastest(false);
+  return launch_grouped_gemm(gate_up, false, tw, ta, tsc, tgs, w, num_sms, s);
+}
 
 uint64_t wait_timeout_ns() {
   static uint64_t v = [] {
@@ -429,6 +465,13 @@ w4a8_status w4a8_moe_route_permute(const float* logits, int64_t T, int32_t E, in
                                  rb.tile_prefix, kTileNPrefill, nullptr,
                                  static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "route launch");
+}
+
+int32_t w4a8_moe_forward_launches(int64_t T, int32_t E, int32_t k) {
+  if (T <= 0 || E < 1 || k < 1) return 0;
+  // activation quantiser, top-k, scan, scatter, two grouped GEMMs, the
+  // requantiser and the combine; split tiling launches each GEMM twice
+  return split_tiles(T * k, E) ? 10 : 8;
 }
 
 size_t w4a8_moe_workspace_size(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k) {
@@ -637,9 +680,17 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   }
   const int64_t A = T * k;
   // Few tokens per expert (decode): narrow tiles with a deep pipeline; many
-  // (prefill): wide tiles that feed each converted weight tile to more tokens.
+  // (prefill): wide tiles that feed each converted weight tile to more tokens;
+  // in between (split): each expert by its own count.
   const bool decode = A <= static_cast<int64_t>(kDecodeTokensPerExpert) * E;
-  const int tile_n = grouped_gemm_tile_n(decode);
+  const bool split = !i8 && split_tiles(A, E);
+  const int tile_n = split ? kTileNDecode : grouped_gemm_tile_n(decode);
+  SplitTiles st;
+  if (split) {
+    st.wide_min = kTileNDecode;
+    st.tile_n_wide = kTileNPrefill;
+    st.tile_prefix_wide = b.route.tile_prefix_wide;
+  }
 
   // TMA descriptors: packed weights [E * rows, K / 2] bytes, 64-byte swizzle;
   // activation codes in segment order [A, K] bytes, 128-byte swizzle, 16-row boxes.
@@ -659,7 +710,7 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
                                     static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
   // three-part group sums as bytes [A, 2 ld], 16 rows x 128 bytes per box
-  const bool parts = !i8 && grouped_gemm_uses_sum_parts(decode);
+  const bool parts = !i8 && !split && grouped_gemm_uses_sum_parts(decode);
   if (w4a8_status st = encode_u8_2d(&tg1, b.act_parts, static_cast<uint64_t>(2 * sum_parts_ld(H)),
                                     static_cast<uint64_t>(A), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
@@ -705,7 +756,7 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   W4A8_STEP(record(2), "cudaEventRecord");
   W4A8_STEP(launch_route(logits, T, E, k, b.topk_ids, b.topk_w, b.expert_offsets,
                          b.sorted_token_ids, b.row_of, b.route.block_counts, b.route.block_base,
-                         b.route.tile_prefix, tile_n, b.row_amax, s),
+                         b.route.tile_prefix, tile_n, b.row_amax, s, st),
             "route launch");
   W4A8_STEP(record(3), "cudaEventRecord");
   W4A8_STEP(record(0), "cudaEventRecord");
@@ -737,9 +788,16 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   g1.wsum = i8 ? i8->w13_nsum : nullptr;
   g1.act_sum = b.act_rowsum;
   W4A8_STEP(record(4), "cudaEventRecord");
-  W4A8_STEP(i8 ? launch_grouped_gemm_i8(true, decode, tw1, ta1, g1, di.sms, s)
-               : launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
-            "gate/up GEMM launch");
+  if (split) {
+    g1.nb_fastest = tile_order_nb_fastest(true);
+    W4A8_STEP(launch_grouped_gemm_split(true, tw1, ta1, ts1, tg1, g1, b.route.tile_prefix_wide,
+                                        di.sms, s),
+              "gate/up GEMM launch");
+  } else {
+    W4A8_STEP(i8 ? launch_grouped_gemm_i8(true, decode, tw1, ta1, g1, di.sms, s)
+                 : launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
+              "gate/up GEMM launch");
+  }
   W4A8_STEP(record(5), "cudaEventRecord");
 
   W4A8_STEP(record(6), "cudaEventRecord");
@@ -771,9 +829,16 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
   g2.wsum = i8 ? i8->w2_nsum : nullptr;
   g2.act_sum = b.inter_rowsum;
   W4A8_STEP(record(8), "cudaEventRecord");
-  W4A8_STEP(i8 ? launch_grouped_gemm_i8(false, decode, tw2, ta2, g2, di.sms, s)
-               : launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),
-            "down GEMM launch");
+  if (split) {
+    g2.nb_fastest = tile_order_nb_fastest(true);
+    W4A8_STEP(launch_grouped_gemm_split(false, tw2, ta2, ts2, tg2, g2, b.route.tile_prefix_wide,
+                                        di.sms, s),
+              "down GEMM launch");
+  } else {
+    W4A8_STEP(i8 ? launch_grouped_gemm_i8(false, decode, tw2, ta2, g2, di.sms, s)
+                 : launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),
+              "down GEMM launch");
+  }
   W4A8_STEP(record(9), "cudaEventRecord");
 
   W4A8_STEP(record(10), "cudaEventRecord");
@@ -1014,8 +1079,15 @@ w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_
   const int64_t A = T * k;   // rows of the buffers: every slot could be local
   // the shape by the expected local load, which is the whole layer's per-expert load
   const bool decode = A <= static_cast<int64_t>(kDecodeTokensPerExpert) * E;
-  const int tile_n = grouped_gemm_tile_n(decode);
-  const bool parts = grouped_gemm_uses_sum_parts(decode);
+  const bool split = split_tiles(A, E);
+  const int tile_n = split ? kTileNDecode : grouped_gemm_tile_n(decode);
+  const bool parts = !split && grouped_gemm_uses_sum_parts(decode);
+  SplitTiles st;
+  if (split) {
+    st.wide_min = kTileNDecode;
+    st.tile_n_wide = kTileNPrefill;
+    st.tile_prefix_wide = b.route.tile_prefix_wide;
+  }
 
   CUtensorMap tw1, ta1, tw2, ta2, ts1, ts2, tg1, tg2;
   if (w4a8_status st = encode_u8_2d(&tw1, w13_packed, static_cast<uint64_t>(H / 2),
@@ -1058,7 +1130,7 @@ w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_
   W4A8_STEP(launch_route_local(topk_ids, T, E, k, e_begin, e_count, b.expert_offsets,
                                b.sorted_token_ids, b.row_of, b.route.block_counts,
                                b.route.block_base, b.route.tile_prefix, tile_n, b.row_amax, latch,
-                               di.sms, s),
+                               di.sms, s, st),
             "local routing launch");
   const int32_t* rows_total = b.expert_offsets + e_count;
   W4A8_STEP(launch_ep_gather(act_codes, T, H, b.sorted_token_ids, rows_total, A, b.perm_codes,
@@ -1084,8 +1156,15 @@ w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_
   g1.nb_fastest = tile_order_nb_fastest(decode);
   g1.n_seg_rows = A;
   g1.n_tokens = T;
-  W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
-            "gate/up GEMM launch");
+  if (split) {
+    g1.nb_fastest = tile_order_nb_fastest(true);
+    W4A8_STEP(launch_grouped_gemm_split(true, tw1, ta1, ts1, tg1, g1, b.route.tile_prefix_wide,
+                                        di.sms, s),
+              "gate/up GEMM launch");
+  } else {
+    W4A8_STEP(launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
+              "gate/up GEMM launch");
+  }
   W4A8_STEP(launch_inter_quant(b.h, b.row_amax, A, I, b.inter_codes, b.inter_scales,
                                parts ? nullptr : b.inter_gsum, di.sms, s, nullptr,
                                parts ? b.inter_parts : nullptr, rows_total),
@@ -1102,8 +1181,14 @@ w4a8_status w4a8_moe_forward_experts(const uint8_t* act_codes, const float* act_
   g2.out_ld = H;
   g2.row_amax = nullptr;
   g2.act_rows = A;
-  W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),
-            "down GEMM launch");
+  if (split) {
+    W4A8_STEP(launch_grouped_gemm_split(false, tw2, ta2, ts2, tg2, g2, b.route.tile_prefix_wide,
+                                        di.sms, s),
+              "down GEMM launch");
+  } else {
+    W4A8_STEP(launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),
+              "down GEMM launch");
+  }
   W4A8_STEP(launch_combine(b.y, b.row_of, topk_w, T, H, k, nullptr, di.sms, s, nullptr,
                            partial_out),
             "partial combine launch");

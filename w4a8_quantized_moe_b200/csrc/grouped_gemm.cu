@@ -69,6 +69,7 @@
 
 #include <cstdint>
 #include <cstdlib>
+#include <type_traits>
 
 #include "internal.h"
 #define W4A8_OWNS_DEVICE_ERROR_LATCH 1
@@ -419,7 +420,8 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     bool good = sEO[0] == 0 && sTP[0] == 0 && sEO[a.E] <= a.n_seg_rows;
     for (int e = 0; good && e < a.E; ++e) {
       const int cnt = sEO[e + 1] - sEO[e];
-      good = cnt >= 0 && sTP[e + 1] - sTP[e] == (cnt + kTileN - 1) / kTileN;
+      const int tiles = sTP[e + 1] - sTP[e];   // 0 when another launch takes the expert
+      good = cnt >= 0 && tiles >= 0 && tiles <= (cnt + kTileN - 1) / kTileN;
     }
     if (!good) {
       atomicOr(&g_device_error, kDeviceErrorIndex);
@@ -1058,38 +1060,45 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           const float2 sm8x2 = make_float2(-8.0f * sg, -8.0f * sg);
           const float* sg_row = sSl + g * kSumLd;
           const uint32_t taddr = tmem + lane_base + kTmemD + d * S::kDCols + h * kTileN + j0;
+          // one TMEM load of NC columns at chunk c, promoted into acc2
+          auto promote = [&](auto nc_tag, int c) {
+            constexpr int NC = decltype(nc_tag)::value;
+            uint32_t v[NC];
+            if constexpr (NC == 32) tmem_ld_32x32b_x32(taddr + c * kLdCols, v);
+            else tmem_ld_32x32b_x16(taddr + c * kLdCols, v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kEpiN / kLdCols; ++c) {
-            if (j0 + c * kLdCols < t.n_mma) {
-              uint32_t v[kLdCols];
-              if constexpr (kLdCols == 32) tmem_ld_32x32b_x32(taddr + c * 32, v);
-              else tmem_ld_32x32b_x16(taddr + c * 16, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < kLdCols; i += 4) {
-                const int o = (c * kLdCols + i) / 2;
-                if constexpr (kF8W) {  // acc += (s_w * s_a[column]) * D
-                  const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
-                  acc2[o] = __ffma2_rn(make_float2(sw * s4.x, sw * s4.y),
-                                       make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
-                                       acc2[o]);
-                  acc2[o + 1] = __ffma2_rn(
-                      make_float2(sw * s4.z, sw * s4.w),
-                      make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), acc2[o + 1]);
-                  continue;
-                }
-                acc2[o] = __ffma2_rn(
-                    s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
+            for (int i = 0; i < NC; i += 4) {
+              const int o = (c * kLdCols + i) / 2;
+              if constexpr (kF8W) {  // acc += (s_w * s_a[column]) * D
+                const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
+                acc2[o] = __ffma2_rn(make_float2(sw * s4.x, sw * s4.y),
+                                     make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                     acc2[o]);
                 acc2[o + 1] = __ffma2_rn(
-                    s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
-                    acc2[o + 1]);
-                if constexpr (S::kEpiOffset) {  // remove the +8 offset: - 8 s_g S_g
-                  const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
-                  acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
-                  acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
-                }
+                    make_float2(sw * s4.z, sw * s4.w),
+                    make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])), acc2[o + 1]);
+                continue;
+              }
+              acc2[o] = __ffma2_rn(
+                  s512x2, make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), acc2[o]);
+              acc2[o + 1] = __ffma2_rn(
+                  s512x2, make_float2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
+                  acc2[o + 1]);
+              if constexpr (S::kEpiOffset) {  // remove the +8 offset: - 8 s_g S_g
+                const float4 s4 = *reinterpret_cast<const float4*>(sg_row + c * kLdCols + i);
+                acc2[o] = __ffma2_rn(sm8x2, make_float2(s4.x, s4.y), acc2[o]);
+                acc2[o + 1] = __ffma2_rn(sm8x2, make_float2(s4.z, s4.w), acc2[o + 1]);
               }
             }
+          };
+#pragma unroll
+          for (int c = 0; c < kEpiN / kLdCols; ++c) {
+            // only the columns the MMA computed (a decode tile of <= 16 rows
+            // has N = 16: half of a 32-column load would be unused)
+            const int live = t.n_mma - (j0 + c * kLdCols);
+            if (kLdCols == 32 && live > 16) promote(std::integral_constant<int, kLdCols>{}, c);
+            else if (live > 0) promote(std::integral_constant<int, 16>{}, c);
           }
         }
         tc_fence_before();

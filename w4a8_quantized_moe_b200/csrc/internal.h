@@ -45,13 +45,22 @@ cudaError_t launch_act_quant(const void* x, int64_t T, int64_t H, uint8_t* codes
 // clip_search: the per-group MSE search over 11 shrink ratios instead of absmax / 7.
 cudaError_t launch_pack_int4(const void* w, int64_t R, int64_t K, int32_t* packed, void* scales,
                              bool clip_search, int num_sms, cudaStream_t s);
+// Split tiling of the grouped GEMMs: with tile_prefix_wide set, experts with
+// more than wide_min segment rows are tiled tile_n_wide rows at a time in
+// tile_prefix_wide (and get no tiles in tile_prefix), the others tile_n at a
+// time in tile_prefix only.
+struct SplitTiles {
+  int wide_min = -1;
+  int tile_n_wide = 0;
+  int32_t* tile_prefix_wide = nullptr;
+};
 // routing: top-k + per-block expert histogram; scan; stable scatter.
 // tile_prefix[e] = sum over experts e' < e of ceil(count[e'] / tile_n).
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
                          float* topk_w, int32_t* expert_offsets, int32_t* sorted_token_ids,
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                          int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
-                         cudaStream_t s);
+                         cudaStream_t s, const SplitTiles& split = SplitTiles());
 // Top-k and weights only (no histogram, no permutation).
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
                               float* topk_w, cudaStream_t s);
@@ -63,7 +72,8 @@ cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, in
                                int E_loc, int32_t* expert_offsets, int32_t* sorted_token_ids,
                                int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                                int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
-                               int* latch, int num_sms, cudaStream_t s);
+                               int* latch, int num_sms, cudaStream_t s,
+                               const SplitTiles& split = SplitTiles());
 // Segment row r < *rows_total (device) receives the codes of token
 // sorted_token_ids[r]; the group sums go to gsum [T, H / 128] by token, or to
 // the row's three-part sums (sum_parts, [max_rows, sum_parts_ld(H)]).

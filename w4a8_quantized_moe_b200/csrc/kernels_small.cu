@@ -451,11 +451,17 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh /*[32]*/, int
   return excl;
 }
 
+// Split tiling (tile_prefix_wide != nullptr): experts with more than wide_min
+// assignments get their tiles in tile_prefix_wide (tile_n_wide rows each) and
+// none in tile_prefix, the others the reverse, so that two GEMM launches of
+// different tile shapes cover disjoint experts.
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ block_counts,
                                                           int64_t nblk, int E, int tile_n,
                                                           int32_t* __restrict__ block_base,
                                                           int32_t* __restrict__ expert_offsets,
-                                                          int32_t* __restrict__ tile_prefix) {
+                                                          int32_t* __restrict__ tile_prefix,
+                                                          int wide_min, int tile_n_wide,
+                                                          int32_t* __restrict__ tile_prefix_wide) {
   __shared__ int sh[32];
   const int e = threadIdx.x;
   int running = 0;
@@ -476,7 +482,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   }
   int total = 0, total_tiles = 0;
   const int off = block_exclusive_scan(e < E ? running : 0, sh, &total);
-  const int tiles = (e < E) ? (running + tile_n - 1) / tile_n : 0;
+  const bool wide = tile_prefix_wide != nullptr && running > wide_min;
+  const int tiles = (e < E && !wide) ? (running + tile_n - 1) / tile_n : 0;
   const int toff = block_exclusive_scan(tiles, sh, &total_tiles);
   if (e < E) {
     expert_offsets[e] = off;
@@ -486,6 +493,13 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   if (e == 0) {
     expert_offsets[E] = total;
     tile_prefix[E] = total_tiles;
+  }
+  if (tile_prefix_wide != nullptr) {  // uniform: every thread takes part in the scan
+    int total_wide = 0;
+    const int wtiles = (e < E && wide) ? (running + tile_n_wide - 1) / tile_n_wide : 0;
+    const int woff = block_exclusive_scan(wtiles, sh, &total_wide);
+    if (e < E) tile_prefix_wide[e] = woff;
+    if (e == 0) tile_prefix_wide[E] = total_wide;
   }
 }
 
@@ -928,7 +942,7 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
                          float* topk_w, int32_t* expert_offsets, int32_t* sorted_token_ids,
                          int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                          int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
-                         cudaStream_t s) {
+                         cudaStream_t s, const SplitTiles& split) {
   if (cudaError_t err = ensure_debug_latch()) return err;
   const int64_t nblk = route_blocks(T);
   if (nblk > 0) {
@@ -953,7 +967,8 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int32_t* 
     if (err != cudaSuccess) return err;
   }
   route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, tile_n, block_base,
-                                       expert_offsets, tile_prefix);
+                                       expert_offsets, tile_prefix, split.wide_min,
+                                       split.tile_n_wide, split.tile_prefix_wide);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || nblk == 0) return err;
   const size_t smem = static_cast<size_t>(kScatterWarps) * E * sizeof(uint32_t);
@@ -986,7 +1001,7 @@ cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, in
                                int E_loc, int32_t* expert_offsets, int32_t* sorted_token_ids,
                                int32_t* row_of, int32_t* block_counts, int32_t* block_base,
                                int32_t* tile_prefix, int tile_n, uint32_t* row_amax_to_zero,
-                               int* latch, int num_sms, cudaStream_t s) {
+                               int* latch, int num_sms, cudaStream_t s, const SplitTiles& split) {
   if (cudaError_t err = ensure_debug_latch()) return err;
   const int64_t nblk = route_blocks(T);
   if (nblk > 0) {
@@ -999,7 +1014,8 @@ cudaError_t launch_route_local(const int32_t* topk_ids, int64_t T, int E_all, in
     if (err != cudaSuccess) return err;
   }
   route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E_loc, tile_n, block_base,
-                                       expert_offsets, tile_prefix);
+                                       expert_offsets, tile_prefix, split.wide_min,
+                                       split.tile_n_wide, split.tile_prefix_wide);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess || nblk == 0) return err;
   const size_t smem = static_cast<size_t>(kScatterWarps) * E_loc * sizeof(uint32_t);
