@@ -39,8 +39,10 @@ DEFAULT_CONFIG = workloads.CONFIGS[1].name
 KERNELS_PER_STEP = 8   # act_quant, route topk/scan/scatter, gemm1, inter_quant, gemm2, combine
 SHARED_KERNELS_PER_STEP = 5   # tables, input group quant, gate/up GEMM, h group quant, down GEMM
 # expert-parallel step: act quant, top-k, then local hist/scan/scatter, gather,
-# gemm1, inter_quant, gemm2, partial combine, and the final bf16 cast
+# gemm1, inter_quant, gemm2, partial combine, and the final bf16 cast (each
+# GEMM twice under split tiling)
 EP_KERNELS_PER_STEP = 11
+L2_BYTES = 126 * 10**6
 SEGMENT_BINS = [(0, 0), (1, 8), (9, 32), (33, 128), (129, 512), (513, 2048), (2049, 1 << 31)]
 
 
@@ -394,35 +396,48 @@ def run_single(cfg, args, device, w4, cpu_tokens: int):
     w4.w4a8_check_device_error(device)
     counts = np.diff(offsets.cpu().numpy().astype(np.int64))
 
+    # per-stage CUDA events (the stage breakdown and the dominant kernel's time)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(device)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    w4.w4a8_check_device_error(device)
+    ms_eager = t_start.elapsed_time(t_end)
+    stage_ms = [statistics.mean(ev[i][2 * s_].elapsed_time(ev[i][2 * s_ + 1])
+                                for i in range(args.steps)) for s_ in range(n_ev // 2)]
+
+    # the timed steps: the same forward captured once as a CUDA graph and
+    # replayed (the library's kernels without the per-call host work)
+    graph = w4.capture_graph(lambda: layer(hidden, logits, out=out))
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(device)
     with ClockSampler(device) as clk:
         t_start.record(stream)
         for i in range(args.steps):
-            step(ev[i])
+            graph.replay()
         t_end.record(stream)
         torch.cuda.synchronize(device)
     w4.w4a8_check_device_error(device)
     ms = t_start.elapsed_time(t_end)
-    stage_ms = [statistics.mean(ev[i][2 * s_].elapsed_time(ev[i][2 * s_ + 1])
-                                for i in range(args.steps)) for s_ in range(n_ev // 2)]
 
-    # end to end through the public API: inputs copied in from pinned host
-    # memory and the output read back every step, each step waiting for its
-    # output on the host before the next one starts
+    # end to end: inputs copied in from pinned host memory and the output read
+    # back every step, each step waiting for its output on the host before the
+    # next one starts (the graph reads the buffers the copies fill)
     h_host = hidden.cpu().pin_memory()
     l_host = logits.cpu().pin_memory()
     o_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
-    h_dev = torch.empty_like(hidden)
-    l_dev = torch.empty_like(logits)
     done = torch.cuda.Event()
 
     def e2e_step():
-        h_dev.copy_(h_host, non_blocking=True)
-        l_dev.copy_(l_host, non_blocking=True)
-        layer(h_dev, l_dev, out=out)
+        hidden.copy_(h_host, non_blocking=True)
+        logits.copy_(l_host, non_blocking=True)
+        graph.replay()
         o_host.copy_(out, non_blocking=True)
         done.record(stream)
         done.synchronize()
@@ -444,8 +459,10 @@ def run_single(cfg, args, device, w4, cpu_tokens: int):
     gi = 2 if stage_ms[2] >= stage_ms[4] else 4          # dominant kernel: the slower GEMM
     kname = "grouped_gemm_gate_up" if gi == 2 else "grouped_gemm_down"
     traffic_key = cfg.name if args.variant == "w4a8" else f"{cfg.name}:{args.variant}"
+    del graph
     res = dict(
-        cfg=cfg, ms=ms, e2e_ms=e2e_ms, stage_ms=stage_ms, counts=counts, active=active,
+        cfg=cfg, ms=ms, ms_eager=ms_eager, e2e_ms=e2e_ms, stage_ms=stage_ms, counts=counts,
+        active=active,
         roofline=roofline(g1 if gi == 2 else g2, stage_ms[gi], prefill, pk, kname,
                           recorded_traffic(traffic_key, kname)),
         roofline_layer=roofline(layer_work(cfg, counts, args.variant), ms / args.steps, prefill,
@@ -464,12 +481,25 @@ def run_single(cfg, args, device, w4, cpu_tokens: int):
     return res
 
 
+def step_launches(w4, cfg, variant: str) -> int:
+    """This library's kernel launches in one step of the variant."""
+    if variant == "channel-int8":
+        return KERNELS_PER_STEP
+    n = w4.w4a8_moe_forward_launches(cfg.T, cfg.E, cfg.k)
+    return n + (SHARED_KERNELS_PER_STEP if variant == "w4a8+shared" else 0)
+
+
 def config_fields(cfg, res, args, world=1, parallelism="single"):
+    streamed = res["l2_bytes"]
     c = dict(workload=cfg.name, T=cfg.T, H=cfg.H, I=cfg.I, E=cfg.E, k=cfg.k,
              variant=args.variant, active_experts=res["active"], parallelism=parallelism,
              segments=segment_histogram(res["counts"]),
-             l2=("inputs larger than L2: %.2f GB of packed experts streamed per step"
-                 % (res["l2_bytes"] / 1e9)))
+             l2=(("inputs larger than L2: %.2f GB of packed experts streamed per step"
+                  % (streamed / 1e9)) if streamed > L2_BYTES else
+                 ("L2-resident: %.1f MB of packed experts fit in the %d MB L2, so the HBM "
+                  "roofline fraction means nothing here" % (streamed / 1e6, L2_BYTES // 10**6))),
+             timed_as="CUDA graph replay of the forward (stage_ms from a separate eager pass "
+                      "with per-stage events, %.4f ms per step)" % (res["ms_eager"] / args.steps))
     if res.get("digest"):
         c["inputs_sha256"] = res["digest"]
     return c
@@ -607,8 +637,7 @@ def main():
             e2e=dict(value=whole_job_throughput(cfg.T, 1, args.steps, head["e2e_ms"]),
                      unit="tokens/s", h2d_bytes_per_step=cfg.T * cfg.H * 2 + cfg.T * cfg.E * 4,
                      d2h_bytes_per_step=cfg.T * cfg.H * 2, host_round_trip_per_step=True),
-            gpu_launches=(KERNELS_PER_STEP + (SHARED_KERNELS_PER_STEP if shared else 0))
-            * args.steps,
+            gpu_launches=step_launches(w4, cfg, args.variant) * args.steps,
             clocks=head["clocks"])
         if "shared_roofline" in head:
             line["shared_roofline"] = head["shared_roofline"]
@@ -627,8 +656,7 @@ def main():
                               zip(stage_names(w4, shared), r["stage_ms"])},
                     roofline=r["roofline"], roofline_layer=r["roofline_layer"],
                     config=config_fields(c, r, args), clocks=r["clocks"],
-                    gpu_launches=(KERNELS_PER_STEP + (SHARED_KERNELS_PER_STEP if shared else 0))
-                    * args.steps)
+                    gpu_launches=step_launches(w4, c, args.variant) * args.steps)
                 if "cpu_baseline" in r:
                     per[c.name]["cpu_baseline"] = r["cpu_baseline"]
                 if "shared_roofline" in r:
@@ -672,7 +700,9 @@ def main():
                 e2e=dict(value=whole_job_throughput(T, world, args.steps, e2e_ms),
                          unit="tokens/s", h2d_bytes_per_step=world * (T * H * 2 + T * cfg.E * 4),
                          d2h_bytes_per_step=world * T * H * 2, host_round_trip_per_step=True),
-                gpu_launches=EP_KERNELS_PER_STEP * args.steps, clocks=r["clocks"])
+                gpu_launches=(EP_KERNELS_PER_STEP + w4.w4a8_moe_forward_launches(
+                    T * world, cfg.E, k) - KERNELS_PER_STEP) * args.steps,
+                clocks=r["clocks"])
         else:
             layer = build_layer(cfg, device, w4, args.variant)
             rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)

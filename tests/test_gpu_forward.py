@@ -166,3 +166,27 @@ def test_pages_format_goes_through_prepare():
     assert torch.equal(out.view(torch.int16), ref(hidden.cuda(), logits.cuda()).view(torch.int16))
     with pytest.raises(ValueError, match="w4a8_prepare_experts_b200"):
         w4.w4a8_moe_forward(hidden.cuda(), logits.cuda(), p13, s13, p2, s2, cfg.k)
+
+
+def test_forward_replayed_from_a_cuda_graph():
+    # the forward on fixed buffers, captured once and replayed: bit-identical to
+    # the eager call, and a replay after new inputs are copied in computes them
+    cfg = workloads.MoEConfig("graph", T=48, H=256, I=128, E=8, k=2, seed=41, zipf_s=1.1)
+    hidden, logits, w13, w2 = small_case(cfg)
+    layer = w4.W4A8MoELayer.from_bf16(w13.cuda(), w2.cuda(), cfg.k)
+    h_dev, l_dev = hidden.cuda(), logits.cuda()
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    eager = layer(h_dev, l_dev).clone()
+    graph = w4.capture_graph(lambda: layer(h_dev, l_dev, out=out))
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    cfg2 = cfg.with_(seed=42)
+    h2, l2 = workloads.gen_hidden(cfg2), workloads.gen_logits(cfg2)
+    h_dev.copy_(h2)
+    l_dev.copy_(l2)
+    graph.replay()
+    w4.w4a8_check_device_error()
+    ref2 = layer(h2.cuda(), l2.cuda())
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))

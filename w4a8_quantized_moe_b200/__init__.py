@@ -22,12 +22,14 @@ __all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_ab
            "w4a8_quant_fp8_block", "w4a8_quant_act_fp8_group", "w4a8_shared_expert_forward",
            "w4a8_moe_forward_shared", "SharedExpertFP8", "SHARED_STAGE_NAMES",
            "w4a8_moe_route_topk", "w4a8_moe_experts_workspace_size", "w4a8_moe_forward_experts",
-           "w4a8_cast_f32_bf16"]
+           "w4a8_cast_f32_bf16", "capture_graph"]
 
-# W4A8_LIBRARY=debug selects the bounds-checking build (see build.py)
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
-                        "libw4a8_debug.so" if os.environ.get("W4A8_LIBRARY") == "debug"
-                        else "libw4a8.so")
+# W4A8_LIBRARY=debug selects the bounds-checking build (see build.py); an
+# absolute path to a .so selects that build of the library instead
+_lib_choice = os.environ.get("W4A8_LIBRARY", "")
+LIB_PATH = (_lib_choice if os.path.isabs(_lib_choice) and _lib_choice.endswith(".so") else
+            os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libw4a8_debug.so" if _lib_choice == "debug" else "libw4a8.so"))
 NUM_STAGES = 6
 STAGE_NAMES = ["act_quant", "route_permute", "gemm_gate_up", "inter_quant", "gemm_down",
                "combine"]
@@ -77,6 +79,7 @@ def _declare(L):
         "w4a8_moe_route_permute": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
         "w4a8_moe_route_permute_noalloc": (i32, [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]),
         "w4a8_moe_workspace_size": (sz, [i64, i64, i64, i32, i32]),
+        "w4a8_moe_forward_launches": (i32, [i64, i32, i32]),
         "w4a8_moe_forward": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, sz,
                                    vp, vp]),
         "w4a8_pack_int4_channel": (i32, [vp, i64, i64, vp, vp, vp]),
@@ -301,6 +304,11 @@ def w4a8_moe_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
     return int(lib().w4a8_moe_workspace_size(T, H, I, E, k))
 
 
+def w4a8_moe_forward_launches(T: int, E: int, k: int) -> int:
+    """Kernels one forward launches for these sizes (see include/w4a8.h)."""
+    return int(lib().w4a8_moe_forward_launches(T, E, k))
+
+
 _AUX_FIELDS = ["topk_ids", "topk_w", "expert_offsets", "sorted_token_ids", "row_of", "act_codes",
                "act_scales", "inter_h", "inter_codes", "inter_scales", "y_rows"]
 
@@ -370,6 +378,26 @@ def w4a8_moe_forward(hidden: torch.Tensor, logits: torch.Tensor, w13_packed: tor
                                   None if aux_struct is None else ctypes.byref(aux_struct),
                                   _stream(dev)))
     return out
+
+
+def capture_graph(fn, warmup: int = 2) -> "torch.cuda.CUDAGraph":
+    """Capture ``fn()`` -- calls of this library on fixed tensors, e.g. one
+    layer forward with its inputs, output and workspace already allocated -- as
+    a CUDA graph; ``graph.replay()`` then reruns those kernels on whatever the
+    buffers hold, without the per-call host work (argument checks, tensor-map
+    encoding, launches).  ``fn`` runs ``warmup`` times first on a side stream
+    (one-time set-up such as kernel attributes happens there, not during
+    capture).  The calls must not allocate: pass ``out`` and a workspace."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
 
 
 class W4A8MoELayer:

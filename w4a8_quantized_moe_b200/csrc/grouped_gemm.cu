@@ -1094,11 +1094,15 @@ __global__ void __launch_bounds__(S::kThreads, 1)
           };
 #pragma unroll
           for (int c = 0; c < kEpiN / kLdCols; ++c) {
-            // only the columns the MMA computed (a decode tile of <= 16 rows
-            // has N = 16: half of a 32-column load would be unused)
+            // gate/up: only the columns the MMA computed (a decode tile of <= 16
+            // rows has N = 16, and half of a 32-column load would be unused:
+            // 3 % faster at decode T=64); the down kernel measured 4 % slower
+            // that way, so it keeps the full load
             const int live = t.n_mma - (j0 + c * kLdCols);
-            if (kLdCols == 32 && live > 16) promote(std::integral_constant<int, kLdCols>{}, c);
-            else if (live > 0) promote(std::integral_constant<int, 16>{}, c);
+            if (kLdCols == 32 && (live > 16 || (!kGateUp && live > 0)))
+              promote(std::integral_constant<int, kLdCols>{}, c);
+            else if (live > 0)
+              promote(std::integral_constant<int, 16>{}, c);
           }
         }
         tc_fence_before();
