@@ -70,3 +70,39 @@ def test_committed_traffic_records_name_known_workloads():
         assert wl.split(":")[0] in names
         assert kernel in ("grouped_gemm_gate_up", "grouped_gemm_down")
         assert int(nbytes) > 0 and len(sid) == 40
+
+
+def test_layer_work_is_the_survey_decode_formula():
+    # whole-layer bytes: active experts' weights and scales, hidden in, logits
+    # in, output out, h (float32, written and read) and its codes, Y (float32,
+    # written and read); FLOPs 6 A H I
+    cfg = workloads.config_by_name("decode_t64_h6144_i2048_e256_k8")
+    counts = np.zeros(cfg.E, dtype=np.int64)
+    counts[:226] = 2
+    w = bench.layer_work(cfg, counts)
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    A = T * k
+    assert w["bytes"] == (226 * (18_874_368 + 589_824) + T * H * 2 + T * E * 4 + T * H * 2
+                          + A * I * 9 + A * H * 8)
+    assert w["flops"] == 6 * A * H * I
+
+
+def test_roofline_uses_burst_fp8_for_prefill_and_hbm_for_decode():
+    pk = dict(hbm=6000.0, bf16=1600.0, bf16_sus=1400.0, src="test")
+    r = bench.roofline(dict(bytes=6e9, flops=3.2e12), 1.0, False, pk, "k", None)
+    assert r["bound"] == "hbm" and r["achieved"] == pytest.approx(6000.0)
+    assert r["frac"] == pytest.approx(1.0) and r["kernel"] == "k" and r["traffic"] is None
+    r = bench.roofline(dict(bytes=6e9, flops=3.2e12), 1.0, True, pk)
+    assert r["bound"] == "tensor" and r["peak"] == 3200.0          # 2 x the burst bf16 rate
+    assert r["achieved"] == pytest.approx(3200.0) and r["frac"] == pytest.approx(1.0)
+    assert r["frac_of_sustained"] == pytest.approx(3200.0 / 2800.0)
+    assert "kernel" not in r
+
+
+def test_segment_histogram_bins_every_expert_once():
+    counts = np.array([0, 0, 1, 8, 9, 32, 33, 128, 129, 512, 513, 2048, 2049, 60000])
+    h = bench.segment_histogram(counts)
+    assert sum(h["bins"].values()) == len(counts) == h["experts"]
+    assert h["bins"] == {"0": 2, "1-8": 2, "9-32": 2, "33-128": 2, "129-512": 2,
+                         "513-2048": 2, ">=2049": 2}
+    assert h["active"] == 12 and h["max"] == 60000

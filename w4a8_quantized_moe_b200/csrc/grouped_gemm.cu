@@ -203,12 +203,15 @@ struct Tile {
 // (nb_fastest = 0: the weight-row blocks that share one token block are
 // neighbours) or token block fastest (nb_fastest = 1: the token blocks that
 // share one weight-row block are neighbours), so that CTAs running at the
-// same time share operands through L2.  tile_prefix and expert_offsets are
-// read from the CTA's shared copies (sTP, sEO): the binary search is a chain of
-// dependent loads.
+// same time share operands through L2.  Token block fastest re-reads all of
+// an expert's activation rows once per weight-row block, which only L2 can
+// absorb: an expert with more than nb_cap token blocks runs weight-row block
+// major whatever nb_fastest says.  tile_prefix and expert_offsets are read from
+// the CTA's shared copies (sTP, sEO): the binary search is a chain of dependent
+// loads.
 template <int TileN>
 __device__ __forceinline__ Tile decode_tile(const int* sTP, const int* sEO, int E, int mb_count,
-                                            int nb_fastest, int idx) {
+                                            int nb_fastest, int nb_cap, int idx) {
   const int nbg = idx / mb_count;  // global token block of the idx's expert range
   Tile t;
   int lo = 0, hi = E;  // tile_prefix[lo] <= nbg < tile_prefix[hi]
@@ -220,8 +223,8 @@ __device__ __forceinline__ Tile decode_tile(const int* sTP, const int* sEO, int 
   t.e = lo;
   const int local = idx - sTP[lo] * mb_count;
   int nb;
-  if (nb_fastest) {
-    const int ne = sTP[lo + 1] - sTP[lo];
+  const int ne = sTP[lo + 1] - sTP[lo];
+  if (nb_fastest && ne <= nb_cap) {
     t.mb = local / ne;
     nb = local - t.mb * ne;
   } else {
@@ -347,8 +350,11 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   const int n_cta = kCta2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const int mb_count = (kGateUp ? a.half_rows / 64 : a.n_rows / kBM) / (kCta2 ? 2 : 1);
   const uint64_t tmo = a.timeout_ns;
+  // token blocks of one expert whose activation rows (K bytes each) stay well
+  // inside L2 (32 MB of its 126 MB) while every weight-row block passes by
+  const int nb_cap = static_cast<int>((32ll << 20) / (static_cast<int64_t>(kTileN) * a.K));
   auto tile_at = [&](int idx) -> Tile {
-    Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, idx);
+    Tile t = decode_tile<kTileN>(sTP, sEO, a.E, mb_count, a.nb_fastest, nb_cap, idx);
     if (kCta2) t.mb = 2 * t.mb + static_cast<int>(crank);
     return t;
   };
