@@ -132,6 +132,11 @@ struct Shape {
   static constexpr int kUpBytes = 64 * TileN * 4;         // up-projection exchange
   static constexpr int kSumLd = kEpiN + 4;                // padded: 4-way bank spread on stores
   static constexpr int kTileScBufs = 2;                   // tile weight-scale buffers
+  // Decode shapes, down layer: the staged S_g are double-buffered and fetched
+  // one tile ahead (the rows are contiguous segment rows there)
+  static constexpr __host__ __device__ int sum_bufs(bool gate_up) {
+    return kEpiOffset && TileN == kTileNDecode && !gate_up ? 2 : 1;
+  }
   static constexpr uint32_t kACols = 32 * kGPU;           // TMEM columns per A slot
   static constexpr uint32_t kDCols = TileN * kGPU;        // TMEM columns per accumulator
   static constexpr uint32_t kTmemA = 0;                   // A slots
@@ -153,9 +158,10 @@ struct Shape {
   // converter set walks the tile's groups and correction chunks in order
   static_assert(!kOffsetTile || (!kUnified && ConvSets == 1), "per-tile correction rings");
   // Runtime-sized regions (G = K / 128 groups): staged S_g, per set
-  // [kEpiPerQuad][G][kSumLd] floats, and the tile scales, [kTileScBufs][G][128] bf16.
-  static constexpr __host__ __device__ int sum_bytes(int G) {
-    return kEpiOffset ? (EpiPerQuad * G * kSumLd * 4 + 127) & ~127 : 0;
+  // [sum_bufs][kEpiPerQuad][G][kSumLd] floats, and the tile scales,
+  // [kTileScBufs][G][128] bf16.
+  static constexpr __host__ __device__ int sum_bytes(int G, bool gate_up) {
+    return kEpiOffset ? (sum_bufs(gate_up) * EpiPerQuad * G * kSumLd * 4 + 127) & ~127 : 0;
   }
   static constexpr __host__ __device__ int tile_sc_bytes(int G) { return 256 * G; }
   // tile_prefix and expert_offsets, [E + 1] int32 each
@@ -163,7 +169,7 @@ struct Shape {
   // f8w: E4M3 weights (128 B per row and group, no tile-scale buffers)
   static constexpr int smem_bytes(bool gate_up, int G, int E, bool f8w = false) {
     return 1024 + WStages * (f8w ? 2 * kWStageBytes : kWStageBytes) + BStages * kBStageBytes +
-           EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G)) +
+           EpiSets * ((gate_up ? kUpBytes : 0) + sum_bytes(G, gate_up)) +
            (f8w ? 0 : kTileScBufs * tile_sc_bytes(G)) +
            table_bytes(E) + kNumBars * 8 + 16;
   }
@@ -307,7 +313,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   const int G = a.K / kGroup;
   // per epilogue set: [sU (gate/up only)][sS]
   constexpr int kUpPerSet = kGateUp ? kUpBytes : 0;
-  const int set_bytes = kUpPerSet + S::sum_bytes(G);
+  const int set_bytes = kUpPerSet + S::sum_bytes(G, kGateUp);
   uint8_t* sSet = sB + kBStages * kBStageBytes;
   uint8_t* sT = sSet + S::kEpiSets * set_bytes;
   int* sTP = reinterpret_cast<int*>(sT + kTileScTotal * S::tile_sc_bytes(G));
@@ -910,8 +916,26 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     const int j0 = slice * kEpiN;                   // first column (segment row) of this warp
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     float* sU = reinterpret_cast<float*>(sSet + set * set_bytes);
-    float* sSl = reinterpret_cast<float*>(sSet + set * set_bytes + kUpPerSet) +
-                 slice * G * kSumLd;                // [g][jj] activation group sums of the slice
+    float* const sSl0 = reinterpret_cast<float*>(sSet + set * set_bytes + kUpPerSet) +
+                        slice * G * kSumLd;         // [g][jj] activation group sums of the slice
+    // S_g fetched one tile ahead (down layer, decode shapes): lane g copies
+    // group g (and g + 32) of this warp's quarter of the columns of tile tt
+    // into buffer b; the copies land while the set's current tile runs
+    constexpr bool kSumsAhead = S::sum_bufs(kGateUp) == 2;
+    constexpr int kTok = kEpiN / 4;
+    auto fetch_sums = [&](const Tile& tt, int b) {
+      float* buf = sSl0 + b * S::kEpiPerQuad * G * kSumLd;
+#pragma unroll
+      for (int i = 0; i < kTok; ++i) {
+        const int jj = q * kTok + i;
+        const bool v = j0 + jj < tt.n_valid;
+        const float* src = a.act_gsum + (v ? (tt.row0 + j0 + jj) * G : 0);
+        const uint32_t nb = v ? 4u : 0u;
+        if (lane < G) cp_async_4(smem_u32(buf + lane * kSumLd + jj), src + lane, nb);
+        if (lane + 32 < G) cp_async_4(smem_u32(buf + (lane + 32) * kSumLd + jj), src + lane + 32, nb);
+      }
+    };
+    if (kSumsAhead && cta_x + set * n_cta < total) fetch_sums(tile_at(cta_x + set * n_cta), 0);
     uint64_t* my_sfull = &sfull[set * S::kEpiPerQuad + slice];
     uint64_t* my_sempty = &sempty[set * S::kEpiPerQuad + slice];
     uint64_t* my_upfull = &upfull[set];
@@ -998,8 +1022,16 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         if (lane == 0) mbar_arrive(&dempty[d]);
       } else {
       const uint32_t phs = lt & 1;
-      if constexpr (S::kEpiOffset) {  // stage S_g of this warp's quarter of the slice's columns
-        constexpr int kTok = kEpiN / 4;
+      float* const sSl = sSl0 + (kSumsAhead ? (lt & 1) * S::kEpiPerQuad * G * kSumLd : 0);
+      if constexpr (kSumsAhead) {  // publish this tile's S_g, fetch the next tile's
+        if (!mbar_wait(my_sempty, phs ^ 1, abort_flag, tmo)) break;
+        cp_async_wait_all();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(my_sfull);
+        // the other buffer's readers (the set's previous tile) are done: my_sempty
+        if (tile + S::kEpiSets * n_cta < total)
+          fetch_sums(tile_at(tile + S::kEpiSets * n_cta), (lt + 1) & 1);
+      } else if constexpr (S::kEpiOffset) {  // stage S_g of this warp's quarter of the slice's columns
         if (!mbar_wait(my_sempty, phs ^ 1, abort_flag, tmo)) break;
         constexpr int kBatch = kTok < 8 ? kTok : 8;   // loads in flight per lane
 #pragma unroll
@@ -1198,8 +1230,12 @@ __global__ void __launch_bounds__(S::kThreads, 1)
         const int n_here = t.n_valid - j0;
 #pragma unroll
         for (int jj = 0; jj < kEpiN; ++jj) {
+          // warp-uniform; decode tiles are mostly padding (the wide shapes
+          // keep the branch-free loop)
+          if (kTileN == kTileNDecode && jj >= n_here) break;
+          if (jj >= n_here) continue;
           const float tsj = __shfl_sync(kFull, ts[jj >> 5], jj & 31);
-          if (jj < n_here) yout[jj * a.out_ld] = acc[jj] * tsj;
+          yout[jj * a.out_ld] = acc[jj] * tsj;
         }
       }
     }

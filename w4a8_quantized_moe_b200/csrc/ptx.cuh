@@ -476,4 +476,17 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// 4-byte global -> shared copy by the load/store unit, asynchronous to the
+// issuing thread; src_bytes = 0 writes zero and reads nothing.
+__device__ __forceinline__ void cp_async_4(uint32_t sdst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(sdst), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// This thread's cp_async_4 copies have landed in shared memory.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 }  // namespace w4a8
