@@ -42,6 +42,9 @@ SHARED_KERNELS_PER_STEP = 5   # tables, input group quant, gate/up GEMM, h group
 # gemm1, inter_quant, gemm2, partial combine, and the final bf16 cast (each
 # GEMM twice under split tiling)
 EP_KERNELS_PER_STEP = 11
+# the all-to-all(v) dispatch adds the plan and the send-row gather; its
+# combine of the returned rows takes the place of the bf16 cast
+EP_A2A_EXTRA_KERNELS = 2
 L2_BYTES = 126 * 10**6
 SEGMENT_BINS = [(0, 0), (1, 8), (9, 32), (33, 128), (129, 512), (513, 2048), (2049, 1 << 31)]
 
@@ -517,7 +520,8 @@ def run_expert_parallel(cfg, args, device, w4, dist, rank, world):
     local = build_layer(cfg, device, w4, experts=(b, n)) if n else None
     weights = ((local.w13_packed, local.w13_scales, local.w2_packed, local.w2_scales)
                if local is not None else None)
-    ep = ExpertParallelMoE(weights, cfg.E, cfg.k, b, n, cfg.H, cfg.I, tokens_per_rank=cfg.T)
+    ep = ExpertParallelMoE(weights, cfg.E, cfg.k, b, n, cfg.H, cfg.I, tokens_per_rank=cfg.T,
+                           dispatch=args.ep_dispatch)
     rank_cfg = cfg.with_(seed=cfg.seed + 7919 * rank)      # each rank its own batch
     hidden = workloads.gen_hidden(rank_cfg, device=device)
     logits = workloads.gen_logits(rank_cfg, device=device)
@@ -526,8 +530,12 @@ def run_expert_parallel(cfg, args, device, w4, dist, rank, world):
     for _ in range(args.warmup):
         ep(hidden, logits, out=out)
     w4.w4a8_check_device_error(device)
-    # the experts this rank's share actually served (from the gathered ids)
-    gat_ids = next(iter(ep._bufs.values()))[1].ids.cpu().numpy()
+    # the rows this rank's experts serve: every rank's routed ids (each rank's
+    # batch comes from its own seed, so they are routed again here, untimed)
+    all_ids = [w4.w4a8_moe_route_topk(workloads.gen_logits(cfg.with_(seed=cfg.seed + 7919 * g),
+                                                           device=device), cfg.k)[0]
+               for g in range(world)]
+    gat_ids = torch.cat(all_ids).cpu().numpy()
     local_counts = np.array([np.count_nonzero(gat_ids == e) for e in range(b, b + n)])
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
@@ -598,6 +606,9 @@ def main():
                     help="on one GPU, also time every other workload into per_config (0: no)")
     ap.add_argument("--parallel", default="ep", choices=["ep", "replicas"],
                     help="more than one GPU: expert parallelism (default) or full replicas")
+    ap.add_argument("--ep-dispatch", default="all_gather", choices=["all_gather", "all_to_all"],
+                    help="expert parallelism: all-gather every token to every rank (default) or "
+                         "all-to-all(v) each token to the ranks of its experts")
     ap.add_argument("--digest", type=int, default=1,
                     help="log the sha256 of each workload's generated inputs (0: skip)")
     args = ap.parse_args()
@@ -693,15 +704,23 @@ def main():
                             parallelism=f"ep{world}", tokens_per_rank=T,
                             experts_per_rank=[n_ for _, n_ in expert_partition(cfg.E, world)],
                             rank0_experts_served=int(np.count_nonzero(r["local_counts"])),
-                            dispatch="all-gather of E4M3 codes, scales, ids, weights (NCCL)",
-                            combine="reduce-scatter of float32 partial sums (NCCL)"),
+                            dispatch=("all-gather of E4M3 codes, scales, ids, weights (NCCL)"
+                                      if args.ep_dispatch == "all_gather" else
+                                      "all-to-all(v) of each token's E4M3 codes, scale, ids, "
+                                      "weights to the ranks of its experts (NCCL)"),
+                            combine=("reduce-scatter of float32 partial sums (NCCL)"
+                                     if args.ep_dispatch == "all_gather" else
+                                     "all-to-all(v) of float32 partial sums back, summed in "
+                                     "rank order")),
                 roofline=roofline(work, ms / args.steps, T * world >= 4096, pk,
                                   "ep_step (rank 0: dispatch + local experts + combine)"),
                 e2e=dict(value=whole_job_throughput(T, world, args.steps, e2e_ms),
                          unit="tokens/s", h2d_bytes_per_step=world * (T * H * 2 + T * cfg.E * 4),
                          d2h_bytes_per_step=world * T * H * 2, host_round_trip_per_step=True),
                 gpu_launches=(EP_KERNELS_PER_STEP + w4.w4a8_moe_forward_launches(
-                    T * world, cfg.E, k) - KERNELS_PER_STEP) * args.steps,
+                    T * world, cfg.E, k) - KERNELS_PER_STEP
+                    + (EP_A2A_EXTRA_KERNELS if args.ep_dispatch == "all_to_all" else 0))
+                * args.steps,
                 clocks=r["clocks"])
         else:
             layer = build_layer(cfg, device, w4, args.variant)

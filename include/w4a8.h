@@ -553,6 +553,83 @@ W4A8_API w4a8_status w4a8_moe_forward_experts(
  */
 W4A8_API w4a8_status w4a8_cast_f32_bf16(const float* x, int64_t n, void* out_bf16, void* stream);
 
+/*
+ * The all-to-all(v) form of the dispatch and combine (for large batches, where
+ * sending every token to every rank would cost more than the per-step
+ * exchange of counts): each rank routes its own tokens, sends each token
+ * once to every rank that owns one of its k experts, and adds up the partial
+ * sums that come back.  Rank r of n_ranks owns the contiguous expert range in
+ * which the first E % n_ranks ranks hold one more expert than the others.
+ * One step on a rank with T tokens:
+ *   1. w4a8_quant_act_fp8_per_token and w4a8_moe_route_topk on its tokens;
+ *   2. w4a8_ep_dispatch_plan: how many of its tokens go to each rank, which,
+ *      and where each (token, rank) pair sits in the send buffers;
+ *   3. an all-to-all of the counts, w4a8_ep_gather_rows into the send
+ *      buffers, and all-to-all(v) of the codes, scales, ids and weights;
+ *   4. w4a8_moe_forward_experts on the rows received (its own experts);
+ *   5. an all-to-all(v) of the partial sums back to the senders, and
+ *      w4a8_ep_combine_rows: each token's returned rows summed in rank order
+ *      and rounded once to bf16.
+ * The collectives are the caller's (NCCL between GPUs).
+ *
+ * w4a8_ep_dispatch_plan - for each rank r, the tokens that go to r: token t
+ * goes to r once when at least one of its ids lies in r's range; ids outside
+ * [0, E) (the -1 of an empty slot) go nowhere.
+ *
+ *   topk_ids       [T, k] int32 (device)
+ *   T, k, E        T >= 0, k >= 1, E >= 1
+ *   n_ranks        1 .. 64
+ *   send_counts    [n_ranks] int32 (device), written: tokens for each rank
+ *   send_rows      [send_rows_capacity] int32 (device), written: rank 0's
+ *                  tokens in ascending order, then rank 1's, and so on
+ *                  (sum(send_counts) entries)
+ *   send_rows_capacity  >= T * min(k, n_ranks)
+ *   pos            [T, n_ranks] int32 (device), written: the index in
+ *                  send_rows of (t, r), or -1 when t does not go to r
+ * Errors: INVALID_ARG (NULL pointer, capacity too small, k or E < 1),
+ * UNSUPPORTED_SHAPE (n_ranks outside 1..64).  T = 0 writes zero counts.
+ */
+W4A8_API w4a8_status w4a8_ep_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k,
+                                           int32_t E, int32_t n_ranks, int32_t* send_counts,
+                                           int32_t* send_rows, int64_t send_rows_capacity,
+                                           int32_t* pos, void* stream);
+
+/*
+ * w4a8_ep_gather_rows - the send buffers: row i of each output is row
+ * send_rows[i] of the rank's quantised tokens.
+ *
+ *   codes [T, H] uint8, scales [T] float32, topk_ids [T, k] int32,
+ *   topk_w [T, k] float32   the rank's tokens (device)
+ *   T, H, k        H % 16 == 0
+ *   send_rows      [n_rows] int32 token indices in [0, T) (device)
+ *   codes_out [n_rows, H], scales_out [n_rows], ids_out [n_rows, k],
+ *   w_out [n_rows, k]       written (device)
+ * codes and codes_out 16-byte aligned.  An index outside [0, T) is skipped
+ * by the bounds-checking build (which raises the device latch) and is
+ * undefined behaviour in the release build.
+ */
+W4A8_API w4a8_status w4a8_ep_gather_rows(const uint8_t* codes, const float* scales,
+                                         const int32_t* topk_ids, const float* topk_w, int64_t T,
+                                         int64_t H, int32_t k, const int32_t* send_rows,
+                                         int64_t n_rows, uint8_t* codes_out, float* scales_out,
+                                         int32_t* ids_out, float* w_out, void* stream);
+
+/*
+ * w4a8_ep_combine_rows - the combine after the partial sums come back:
+ *   out[t] = bf16(sum over r = 0 .. n_ranks-1 with pos[t, r] >= 0 of
+ *                 back[pos[t, r]])
+ * summed in float32 in rank order and rounded to nearest even once; a token
+ * that went to no rank gets zeros.
+ *
+ *   back       [n_rows, H] float32 (device): row i = the partial sums of the
+ *              token-rank pair at send_rows index i
+ *   pos        [T, n_ranks] int32 from w4a8_ep_dispatch_plan (device)
+ *   out_bf16   [T, H] bf16, written;  H % 8 == 0, back and out 16-byte aligned
+ */
+W4A8_API w4a8_status w4a8_ep_combine_rows(const float* back, int64_t n_rows, int64_t H,
+                                          const int32_t* pos, int64_t T, int32_t n_ranks,
+                                          void* out_bf16, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

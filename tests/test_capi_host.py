@@ -116,6 +116,19 @@ def test_host_validation_without_device(L):
     # T == 0 is a no-op
     assert L.w4a8_moe_forward(None, None, None, None, None, None, 0, 256, 256, 8, 2, None, None, 0,
                               None, None) == 0
+    # all-to-all dispatch: rank count, send-list capacity, shapes
+    assert L.w4a8_ep_dispatch_plan(fake, 4, 2, 8, 65, fake, fake, 8, fake, None) == 2
+    assert L.w4a8_ep_dispatch_plan(fake, 4, 2, 8, 0, fake, fake, 8, fake, None) == 2
+    assert L.w4a8_ep_dispatch_plan(fake, 4, 2, 8, 4, fake, fake, 7, fake, None) == 1
+    assert b"capacity" in L.w4a8_last_error()
+    assert L.w4a8_ep_dispatch_plan(fake, 4, 0, 8, 4, fake, fake, 8, fake, None) == 1
+    assert L.w4a8_ep_gather_rows(fake, fake, fake, fake, 4, 200, 2, fake, 3, fake, fake, fake,
+                                 fake, None) == 2
+    assert L.w4a8_ep_gather_rows(None, None, None, None, 4, 256, 2, None, 0, None, None, None,
+                                 None, None) == 0
+    assert L.w4a8_ep_combine_rows(fake, 3, 100, fake, 4, 2, fake, None) == 2
+    assert L.w4a8_ep_combine_rows(fake, 3, 256, fake, 4, 65, fake, None) == 2
+    assert L.w4a8_ep_combine_rows(None, 0, 256, None, 0, 2, None, None) == 0
 
 
 def test_python_binding_refuses_cpu_tensors():

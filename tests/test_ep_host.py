@@ -4,7 +4,9 @@ compute steps.
 
 Each rank owns a contiguous expert range, quantises and routes its own
 tokens, all-gathers them, computes its experts' float32 partial sums and
-reduce-scatters them back.  Every rank's output must match the single-process
+reduce-scatters them back; or, with the all-to-all(v) dispatch, sends each
+token only to the ranks of its experts and adds the partial sums that come
+back.  Every rank's output must match the single-process
 oracle's ``moe_forward`` on that rank's tokens.  Cases: 2 and 4 ranks, equal
 and uneven batches (a rank with no tokens), a rank whose experts no token
 chooses, a rank that holds no experts (more ranks than experts), and a rank
@@ -23,6 +25,7 @@ import torch.multiprocessing as mp
 
 import oracle
 import workloads
+from ep_reference import combine_reference, plan_reference
 from w4a8_quantized_moe_b200.ep import ExpertParallelMoE, PaddedBatch, expert_partition
 
 
@@ -74,6 +77,20 @@ class OracleOps:
         out.copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
         return out
 
+    # the all-to-all(v) dispatch, from its definition: token t goes to rank r
+    # once when one of its ids lies in r's expert range; rank-major, tokens
+    # ascending; the combine sums a token's returned rows in rank order
+    def plan(self, ids, E, n):
+        return plan_reference(ids.numpy(), E, n)
+
+    def gather(self, batch, T, rows, n_rows):
+        r = rows[:n_rows].long()
+        return PaddedBatch(codes=batch.codes[:T][r], scales=batch.scales[:T][r],
+                           ids=batch.ids[:T][r], weights=batch.weights[:T][r])
+
+    def combine(self, back, pos, out):
+        return self.cast(torch.from_numpy(combine_reference(back.numpy(), pos.numpy())), out)
+
 
 def _cfg(E, forced_empty=0):
     return workloads.MoEConfig("ep", T=0, H=256, I=128, E=E, k=2, seed=77,
@@ -102,13 +119,13 @@ def _init(rank, world, port, timeout_s):
                             timeout=datetime.timedelta(seconds=timeout_s))
 
 
-def _ep_worker(rank, world, port, E, tokens, forced_empty, steps, q):
+def _ep_worker(rank, world, port, E, tokens, forced_empty, steps, q, dispatch):
     _init(rank, world, port, 60)
     try:
         cfg = _cfg(E, forced_empty)
         begin, count = expert_partition(E, world)[rank]
         layer = ExpertParallelMoE(_experts(cfg, begin, count) if count else None, E, cfg.k,
-                                  begin, count, cfg.H, cfg.I, ops=OracleOps())
+                                  begin, count, cfg.H, cfg.I, ops=OracleOps(), dispatch=dispatch)
         hidden, logits = _batch(cfg, rank, tokens[rank])
         outs = [layer(hidden, logits) for _ in range(steps)]
         # the single-process oracle on this rank's tokens, all experts
@@ -125,12 +142,12 @@ def _ep_worker(rank, world, port, E, tokens, forced_empty, steps, q):
         dist.destroy_process_group()
 
 
-def _run(world, E, tokens, forced_empty=0, steps=1):
+def _run(world, E, tokens, forced_empty=0, steps=1, dispatch="all_gather"):
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     procs = [ctx.Process(target=_ep_worker,
-                         args=(r, world, port, E, tokens, forced_empty, steps, q))
+                         args=(r, world, port, E, tokens, forced_empty, steps, q, dispatch))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -186,6 +203,58 @@ def test_more_ranks_than_experts():
     res = _run(3, 2, tokens)
     _check(res, tokens)
     assert [c for *_, c in res] == [1, 1, 0]
+
+
+def test_plan_reference_is_the_definition():
+    # 3 ranks over E = 7 experts: 3, 2, 2 (ranges [0,3), [3,5), [5,7))
+    ids = np.array([[0, 4], [6, 5], [-1, -1], [1, 2], [3, 6], [4, 4]], dtype=np.int32)
+    counts, rows, pos = plan_reference(ids, 7, 3)
+    assert counts.tolist() == [2, 3, 2]
+    assert rows[:7].tolist() == [0, 3, 0, 4, 5, 1, 4]
+    assert pos.tolist() == [[0, 2, -1], [-1, -1, 5], [-1, -1, -1], [1, -1, -1], [-1, 3, 6],
+                            [-1, 4, -1]]
+    back = np.arange(7 * 2, dtype=np.float32).reshape(7, 2)
+    out = combine_reference(back, pos.numpy())
+    assert out.tolist() == [[4, 6], [10, 11], [0, 0], [2, 3], [18, 20], [8, 9]]
+
+
+def test_all_to_all_two_ranks_two_steps():
+    tokens = [16, 16]
+    _check(_run(2, 8, tokens, steps=2, dispatch="all_to_all"), tokens)
+
+
+def test_all_to_all_four_ranks_uneven_batches_and_an_unchosen_rank():
+    tokens = [5, 16, 0, 3]
+    res = _run(4, 6, tokens, forced_empty=1, dispatch="all_to_all")
+    _check(res, tokens)
+    assert [c for *_, c in res] == [2, 2, 1, 1]
+
+
+def test_all_to_all_more_ranks_than_experts():
+    tokens = [4, 7, 2]
+    res = _run(3, 2, tokens, dispatch="all_to_all")
+    _check(res, tokens)
+
+
+def _range_worker(port, q):
+    _init(0, 1, port, 30)
+    try:
+        ExpertParallelMoE(None, 4, 2, 1, 3, 256, 128, ops=OracleOps(), dispatch="all_to_all")
+        q.put("accepted")
+    except ValueError:
+        q.put("ValueError")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_all_to_all_needs_the_partition_ranges():
+    # one rank must own all 4 experts under the partition; [1, 4) is refused
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_range_worker, args=(_free_port(), q))
+    p.start()
+    assert q.get(timeout=120) == "ValueError"
+    p.join(timeout=60)
 
 
 def _leaving_worker(rank, world, port, q):

@@ -7,7 +7,10 @@ float32 partial sums added, and one bf16 rounding (w4a8_cast_f32_bf16).  The
 result must match w4a8_moe_forward on the whole layer (up to float32
 summation order) and the oracle (relative Frobenius 2e-3).  Also: the
 top-k-only routing call is bit-exact against the oracle, and an expert id
-outside [-1, E) is skipped and reported by the device latch.
+outside [-1, E) is skipped and reported by the device latch.  The
+all-to-all(v) form: the dispatch plan, row gather and combine are bit-exact
+against their definition, and whole emulated steps of several ranks (the
+collectives as slices on the one GPU) match the layer on each rank's tokens.
 """
 import numpy as np
 import pytest
@@ -16,6 +19,7 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
+from ep_reference import combine_reference, plan_reference
 from gpu_helpers import aux_buffers, f64, rel_fro, small_case
 from w4a8_quantized_moe_b200.ep import expert_partition
 
@@ -145,3 +149,95 @@ def test_decode_workload_split_over_eight_shares():
     print(f"\n[decode, 8 shares of 32 experts, 512 tokens] vs layer: {same:.5f} bit-equal, "
           f"rel-Frobenius {dist:.2e}")
     assert same >= 0.999 and dist <= 1e-4
+
+
+# ------------------------------------------------ all-to-all(v) dispatch
+@pytest.mark.parametrize("T,k,E,n,pad", [
+    (0, 2, 6, 3, 0.0), (1, 1, 4, 1, 0.0), (37, 3, 6, 4, 0.1), (3000, 8, 256, 8, 0.05),
+    (500, 4, 7, 3, 0.0), (200, 2, 3, 5, 0.0), (1100, 8, 256, 64, 0.0), (64, 8, 256, 1, 0.0),
+], ids=lambda v: str(v))
+def test_dispatch_plan_bit_exact(T, k, E, n, pad):
+    g = np.random.default_rng(T * 31 + E)
+    ids = g.integers(0, E, size=(T, k)).astype(np.int32)
+    ids[g.random((T, k)) < pad] = -1                  # empty slots go nowhere
+    counts, rows, pos = w4.w4a8_ep_dispatch_plan(torch.from_numpy(ids).cuda(), E, n)
+    rc, rr, rp = plan_reference(ids, E, n)
+    m = int(rc.sum())
+    assert torch.equal(counts.cpu(), rc)
+    assert torch.equal(rows.cpu()[:m], rr[:m])
+    assert torch.equal(pos.cpu(), rp)
+
+
+def test_gather_and_combine_rows_bit_exact():
+    g = np.random.default_rng(3)
+    T, H, k, n = 333, 384, 4, 5
+    codes = torch.from_numpy(g.integers(0, 256, size=(T, H), dtype=np.uint8)).cuda()
+    scales = torch.from_numpy(g.random(T, dtype=np.float32)).cuda()
+    ids = torch.from_numpy(g.integers(-1, 20, size=(T, k)).astype(np.int32)).cuda()
+    w = torch.from_numpy(g.random((T, k), dtype=np.float32)).cuda()
+    counts, rows, pos = w4.w4a8_ep_dispatch_plan(ids, 20, n)
+    m = int(counts.sum())
+    c, s, i, ww = w4.w4a8_ep_gather_rows(codes, scales, ids, w, rows, m)
+    r = rows[:m].long()
+    assert torch.equal(c, codes[r]) and torch.equal(s, scales[r])
+    assert torch.equal(i, ids[r]) and torch.equal(ww, w[r])
+    back = torch.from_numpy(g.standard_normal((m, H)).astype(np.float32) * 3).cuda()
+    out = w4.w4a8_ep_combine_rows(back, pos)
+    ref = combine_reference(back.cpu().numpy(), pos.cpu().numpy())
+    bits = oracle.f64_to_bf16_bits(ref.astype(np.float64))
+    assert np.array_equal(out.cpu().view(torch.int16).numpy().view(np.uint16), bits)
+    none = (pos.cpu() < 0).all(dim=1)                 # tokens that went nowhere: zeros
+    assert not out.cpu()[none].any()
+
+
+@pytest.mark.parametrize("cfg,G,tokens", [
+    (workloads.MoEConfig("a2a_ragged", T=0, H=384, I=256, E=6, k=3, seed=31), 4, [37, 0, 5, 64]),
+    (workloads.MoEConfig("a2a_zipf", T=0, H=256, I=256, E=16, k=4, seed=32, zipf_s=1.1,
+                         forced_empty=5), 8, [50, 20, 1, 0, 33, 16, 64, 9]),
+    (workloads.MoEConfig("a2a_wide", T=0, H=256, I=128, E=4, k=2, seed=33), 3, [300, 129, 70]),
+], ids=lambda x: getattr(x, "name", str(x)))
+def test_all_to_all_step_emulated(cfg, G, tokens):
+    """G ranks' all-to-all(v) steps on one GPU: the collectives are slices of
+    the send buffers in source-rank order; each rank's output must match the
+    layer on its own tokens."""
+    ws = [workloads.gen_expert_weights(cfg, e) for e in range(cfg.E)]
+    w13 = torch.stack([a for a, _ in ws]).cuda()
+    w2 = torch.stack([b for _, b in ws]).cuda()
+    layer = w4.W4A8MoELayer.from_bf16(w13, w2, cfg.k)
+    batches = []
+    for s, T in enumerate(tokens):
+        c = cfg.with_(T=T, seed=cfg.seed + 7 * s)
+        hidden, logits = workloads.gen_hidden(c).cuda(), workloads.gen_logits(c).cuda()
+        codes, scales = w4.w4a8_quant_act_fp8_per_token(hidden)
+        ids, w = w4.w4a8_moe_route_topk(logits, cfg.k)
+        counts, rows, pos = w4.w4a8_ep_dispatch_plan(ids, cfg.E, G)
+        send = w4.w4a8_ep_gather_rows(codes, scales, ids, w, rows, int(counts.sum()))
+        batches.append((hidden, logits, counts.tolist(), send, pos))
+    offs = [np.concatenate([[0], np.cumsum(b[2])]) for b in batches]
+    parts = {}
+    for r in range(G):                                 # rank r: rows from every source
+        recv = [torch.cat([b[3][f][offs[s][r]:offs[s][r + 1]] for s, b in enumerate(batches)])
+                for f in range(4)]
+        b_, n_ = expert_partition(cfg.E, G)[r]
+        partial = torch.zeros(recv[0].shape[0], cfg.H, dtype=torch.float32, device="cuda")
+        if n_ and recv[0].shape[0]:
+            wl = (layer.w13_packed[b_:b_ + n_], layer.w13_scales[b_:b_ + n_],
+                  layer.w2_packed[b_:b_ + n_], layer.w2_scales[b_:b_ + n_])
+            partial = w4.w4a8_moe_forward_experts(*recv, cfg.E, b_, *wl)
+        o = 0
+        for s, b in enumerate(batches):                # split back by source
+            m = b[2][r]
+            parts[(s, r)] = partial[o:o + m]
+            o += m
+    w4.w4a8_check_device_error()
+    for s, (hidden, logits, counts, _, pos) in enumerate(batches):
+        back = torch.cat([parts[(s, r)] for r in range(G)])
+        out = w4.w4a8_ep_combine_rows(back, pos)
+        if hidden.shape[0] == 0:
+            assert out.shape == (0, cfg.H)
+            continue
+        ref = layer(hidden, logits)
+        same, dist = _agreement(out, ref)
+        print(f"\n[{cfg.name}, rank {s} of {G}, {hidden.shape[0]} tokens] vs layer: "
+              f"{same:.5f} bit-equal, rel-Frobenius {dist:.2e}")
+        assert same >= 0.999 and dist <= 1e-4

@@ -22,7 +22,8 @@ __all__ = ["W4A8Error", "lib", "LIB_PATH", "NUM_STAGES", "STAGE_NAMES", "w4a8_ab
            "w4a8_quant_fp8_block", "w4a8_quant_act_fp8_group", "w4a8_shared_expert_forward",
            "w4a8_moe_forward_shared", "SharedExpertFP8", "SHARED_STAGE_NAMES",
            "w4a8_moe_route_topk", "w4a8_moe_experts_workspace_size", "w4a8_moe_forward_experts",
-           "w4a8_cast_f32_bf16", "capture_graph"]
+           "w4a8_cast_f32_bf16", "w4a8_ep_dispatch_plan", "w4a8_ep_gather_rows",
+           "w4a8_ep_combine_rows", "capture_graph"]
 
 # W4A8_LIBRARY=debug selects the bounds-checking build (see build.py); an
 # absolute path to a .so selects that build of the library instead
@@ -99,6 +100,10 @@ def _declare(L):
         "w4a8_moe_forward_experts": (i32, [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
                                            vp, vp, vp, vp, vp, vp, sz, vp]),
         "w4a8_cast_f32_bf16": (i32, [vp, i64, vp, vp]),
+        "w4a8_ep_dispatch_plan": (i32, [vp, i64, i32, i32, i32, vp, vp, i64, vp, vp]),
+        "w4a8_ep_gather_rows": (i32, [vp, vp, vp, vp, i64, i64, i32, vp, i64, vp, vp, vp, vp,
+                                      vp]),
+        "w4a8_ep_combine_rows": (i32, [vp, i64, i64, vp, i64, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -791,4 +796,66 @@ def w4a8_cast_f32_bf16(x: torch.Tensor, out: Optional[torch.Tensor] = None) -> t
         raise ValueError("out must be a contiguous bf16 CUDA tensor of x's shape")
     _check("w4a8_cast_f32_bf16",
            lib().w4a8_cast_f32_bf16(_p(x), x.numel(), _p(out), _stream(x.device)))
+    return out
+
+
+def w4a8_ep_dispatch_plan(topk_ids: torch.Tensor, E: int, n_ranks: int):
+    """The all-to-all(v) dispatch plan of a rank's routed tokens:
+    (send_counts int32 [n_ranks], send_rows int32 [T * min(k, n_ranks)] (the
+    first sum(send_counts) entries used), pos int32 [T, n_ranks])."""
+    _need(topk_ids, "topk_ids", torch.int32, 2)
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    counts = torch.empty(n_ranks, dtype=torch.int32, device=dev)
+    rows = torch.empty(max(T * min(k, n_ranks), 1), dtype=torch.int32, device=dev)
+    pos = torch.empty(T, n_ranks, dtype=torch.int32, device=dev)
+    _check("w4a8_ep_dispatch_plan",
+           lib().w4a8_ep_dispatch_plan(_p(topk_ids), T, k, E, n_ranks, _p(counts), _p(rows),
+                                       rows.numel(), _p(pos), _stream(dev)))
+    return counts, rows, pos
+
+
+def w4a8_ep_gather_rows(codes: torch.Tensor, scales: torch.Tensor, topk_ids: torch.Tensor,
+                        topk_w: torch.Tensor, send_rows: torch.Tensor, n_rows: int):
+    """Rows ``send_rows[:n_rows]`` of a rank's codes, scales, ids and weights:
+    (uint8 [n, H], float32 [n], int32 [n, k], float32 [n, k])."""
+    _need(codes, "codes", torch.uint8, 2)
+    _need(scales, "scales", torch.float32, 1)
+    _need(topk_ids, "topk_ids", torch.int32, 2)
+    _need(topk_w, "topk_w", torch.float32, 2)
+    _need(send_rows, "send_rows", torch.int32, 1)
+    T, H = codes.shape
+    k = topk_ids.shape[1]
+    if scales.shape != (T,) or topk_ids.shape[0] != T or topk_w.shape != (T, k) or \
+            not 0 <= n_rows <= send_rows.numel():
+        raise ValueError("inconsistent shapes: codes [T,H], scales [T], ids/w [T,k], "
+                         "n_rows <= len(send_rows)")
+    dev = codes.device
+    out = (torch.empty(n_rows, H, dtype=torch.uint8, device=dev),
+           torch.empty(n_rows, dtype=torch.float32, device=dev),
+           torch.empty(n_rows, k, dtype=torch.int32, device=dev),
+           torch.empty(n_rows, k, dtype=torch.float32, device=dev))
+    _check("w4a8_ep_gather_rows",
+           lib().w4a8_ep_gather_rows(_p(codes), _p(scales), _p(topk_ids), _p(topk_w), T, H, k,
+                                     _p(send_rows), n_rows, *(_p(o) for o in out), _stream(dev)))
+    return out
+
+
+def w4a8_ep_combine_rows(back: torch.Tensor, pos: torch.Tensor,
+                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """bf16 [T, H]: each token's returned partial-sum rows ``back[pos[t, r]]``
+    summed in rank order (float32) and rounded once."""
+    _need(back, "back", torch.float32, 2)
+    _need(pos, "pos", torch.int32, 2)
+    n_rows, H = back.shape
+    T, n_ranks = pos.shape
+    dev = pos.device
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, 2)
+    if out.shape != (T, H):
+        raise ValueError("out must be [T, H]")
+    _check("w4a8_ep_combine_rows",
+           lib().w4a8_ep_combine_rows(_p(back), n_rows, H, _p(pos), T, n_ranks, _p(out),
+                                      _stream(dev)))
     return out

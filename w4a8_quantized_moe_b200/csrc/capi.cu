@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <climits>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -1208,6 +1209,74 @@ w4a8_status w4a8_cast_f32_bf16(const float* x, int64_t n, void* out_bf16, void* 
   if (w4a8_status st = device_info(&di)) return st;
   cudaError_t err = launch_cast_bf16(x, n, out_bf16, di.sms, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "cast launch");
+}
+
+w4a8_status w4a8_ep_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
+                                  int32_t n_ranks, int32_t* send_counts, int32_t* send_rows,
+                                  int64_t send_rows_capacity, int32_t* pos, void* stream) {
+  if (T < 0 || k < 1 || E < 1)
+    return fail(W4A8_ERR_INVALID_ARG, "T = %lld, k = %d, E = %d", static_cast<long long>(T), k, E);
+  if (n_ranks < 1 || n_ranks > kEpMaxRanks)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "n_ranks = %d outside [1, %d]", n_ranks, kEpMaxRanks);
+  if (!send_counts || (T > 0 && (!topk_ids || !send_rows || !pos)))
+    return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+  if (T > INT32_MAX / n_ranks)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "T * n_ranks exceeds int32 indices");
+  if (send_rows_capacity < T * std::min<int64_t>(k, n_ranks))
+    return fail(W4A8_ERR_INVALID_ARG, "send_rows_capacity %lld < T * min(k, n_ranks) = %lld",
+                static_cast<long long>(send_rows_capacity),
+                static_cast<long long>(T * std::min<int64_t>(k, n_ranks)));
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_ep_plan(topk_ids, T, k, E, n_ranks, send_counts, send_rows, pos,
+                                   static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "dispatch plan launch");
+}
+
+w4a8_status w4a8_ep_gather_rows(const uint8_t* codes, const float* scales, const int32_t* topk_ids,
+                                const float* topk_w, int64_t T, int64_t H, int32_t k,
+                                const int32_t* send_rows, int64_t n_rows, uint8_t* codes_out,
+                                float* scales_out, int32_t* ids_out, float* w_out, void* stream) {
+  if (T < 0 || H <= 0 || k < 1 || n_rows < 0)
+    return fail(W4A8_ERR_INVALID_ARG, "T = %lld, H = %lld, k = %d, n_rows = %lld",
+                static_cast<long long>(T), static_cast<long long>(H), k,
+                static_cast<long long>(n_rows));
+  if (H % 16) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld is not a multiple of 16",
+                          static_cast<long long>(H));
+  if (n_rows == 0) return W4A8_OK;
+  if (!codes || !scales || !topk_ids || !topk_w || !send_rows || !codes_out || !scales_out ||
+      !ids_out || !w_out)
+    return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+  if (!aligned16(codes) || !aligned16(codes_out))
+    return fail(W4A8_ERR_INVALID_ARG, "codes pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_ep_gather_rows(codes, scales, topk_ids, topk_w, T, H, k, send_rows,
+                                          n_rows, codes_out, scales_out, ids_out, w_out, di.sms,
+                                          static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "row gather launch");
+}
+
+w4a8_status w4a8_ep_combine_rows(const float* back, int64_t n_rows, int64_t H, const int32_t* pos,
+                                 int64_t T, int32_t n_ranks, void* out_bf16, void* stream) {
+  if (T < 0 || H <= 0 || n_rows < 0)
+    return fail(W4A8_ERR_INVALID_ARG, "T = %lld, H = %lld, n_rows = %lld",
+                static_cast<long long>(T), static_cast<long long>(H),
+                static_cast<long long>(n_rows));
+  if (n_ranks < 1 || n_ranks > kEpMaxRanks)
+    return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "n_ranks = %d outside [1, %d]", n_ranks, kEpMaxRanks);
+  if (H % 8) return fail(W4A8_ERR_UNSUPPORTED_SHAPE, "H = %lld is not a multiple of 8",
+                         static_cast<long long>(H));
+  if (T == 0) return W4A8_OK;
+  if (!pos || !out_bf16 || (n_rows > 0 && !back))
+    return fail(W4A8_ERR_INVALID_ARG, "NULL pointer argument");
+  if ((back && !aligned16(back)) || !aligned16(out_bf16))
+    return fail(W4A8_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceInfo di;
+  if (w4a8_status st = device_info(&di)) return st;
+  cudaError_t err = launch_ep_combine_rows(back, n_rows, H, pos, T, n_ranks, out_bf16, di.sms,
+                                           static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? W4A8_OK : cuda_fail(err, "combine rows launch");
 }
 
 }  // extern "C"

@@ -81,6 +81,19 @@ cudaError_t launch_ep_gather(const uint8_t* codes, int64_t T, int64_t H,
                              const int32_t* sorted_token_ids, const int32_t* rows_total,
                              int64_t max_rows, uint8_t* perm, float* gsum, uint16_t* sum_parts,
                              int num_sms, cudaStream_t s);
+// Expert-parallel all-to-all(v) dispatch (ranks <= kEpMaxRanks): the plan
+// (per-rank token counts, the rank-major token list, the (token, rank) -> list
+// index map or -1), the send-row gather and the combine of the returned rows.
+constexpr int kEpMaxRanks = 64;
+cudaError_t launch_ep_plan(const int32_t* topk_ids, int64_t T, int k, int E, int n_ranks,
+                           int32_t* counts, int32_t* rows, int32_t* pos, cudaStream_t s);
+cudaError_t launch_ep_gather_rows(const uint8_t* codes, const float* scales, const int32_t* ids,
+                                  const float* w, int64_t T, int64_t H, int k, const int32_t* rows,
+                                  int64_t n_rows, uint8_t* codes_out, float* scales_out,
+                                  int32_t* ids_out, float* w_out, int num_sms, cudaStream_t s);
+cudaError_t launch_ep_combine_rows(const float* back, int64_t n_rows, int64_t H,
+                                   const int32_t* pos, int64_t T, int n_ranks, void* out,
+                                   int num_sms, cudaStream_t s);
 // bf16 = round-to-nearest-even(x), n a multiple of 8.
 cudaError_t launch_cast_bf16(const float* x, int64_t n, void* out, int num_sms, cudaStream_t s);
 // sum_parts (nullable): [A, sum_parts_ld(I)] bf16 as for launch_act_quant.

@@ -875,6 +875,146 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   }
 }
 
+// ------------------------------------------- expert-parallel all-to-all(v)
+// Dispatch by all-to-all(v): each rank sends each of its tokens once to every
+// rank that owns one of the token's k experts, and adds the partial sums that
+// come back.  Rank r of n owns a contiguous expert range; the first E % n
+// ranks hold one more expert.
+__device__ __forceinline__ int ep_owner(int e, int E, int n) {
+  const int base = E / n, extra = E % n;
+  const int cut = extra * (base + 1);              // experts of the larger ranks
+  return e < cut ? e / (base + 1) : extra + (e - cut) / base;
+}
+
+// One CTA.  Pass 1 counts the tokens per rank; pass 2 walks the tokens in
+// chunks of the block size and places each (token, rank) pair: rank-major,
+// tokens ascending inside a rank (ballot prefix within a warp, a per-rank
+// prefix over the warps, a running offset per rank across chunks).
+constexpr int kPlanThreads = 1024;
+__global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(const int32_t* __restrict__ ids,
+                                                               int64_t T, int k, int E, int n,
+                                                               int32_t* __restrict__ counts,
+                                                               int32_t* __restrict__ rows,
+                                                               int32_t* __restrict__ pos) {
+  __shared__ int s_off[kEpMaxRanks];               // totals, then running offsets
+  __shared__ int s_warp[kPlanThreads / 32][kEpMaxRanks];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < kEpMaxRanks) s_off[tid] = 0;
+  __syncthreads();
+  auto ranks_of = [&](int64_t t) -> uint64_t {     // the ranks token t goes to
+    uint64_t m = 0;
+    if (t < T)
+      for (int j = 0; j < k; ++j) {
+        const int e = __ldg(ids + t * k + j);
+        if (e >= 0 && e < E) m |= 1ull << ep_owner(e, E, n);
+      }
+    return m;
+  };
+  for (int64_t c0 = 0; c0 < T; c0 += kPlanThreads) {
+    const uint64_t m = ranks_of(c0 + tid);
+    for (int r = 0; r < n; ++r) {
+      const unsigned b = __ballot_sync(kFull, (m >> r) & 1u);
+      if (lane == 0 && b) atomicAdd(&s_off[r], __popc(b));
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int r = 0; r < n; ++r) {
+      const int c = s_off[r];
+      counts[r] = c;
+      s_off[r] = acc;
+      acc += c;
+    }
+  }
+  __syncthreads();
+  for (int64_t c0 = 0; c0 < T; c0 += kPlanThreads) {
+    const int64_t t = c0 + tid;
+    const uint64_t m = ranks_of(t);
+    for (int r = 0; r < n; ++r) {
+      const unsigned b = __ballot_sync(kFull, (m >> r) & 1u);
+      if (lane == 0) s_warp[warp][r] = __popc(b);
+    }
+    __syncthreads();
+    if (tid < n) {                                 // thread r: warp bases of rank r
+      int acc = s_off[tid];
+      for (int w = 0; w < kPlanThreads / 32; ++w) {
+        const int c = s_warp[w][tid];
+        s_warp[w][tid] = acc;
+        acc += c;
+      }
+      s_off[tid] = acc;
+    }
+    __syncthreads();
+    for (int r = 0; r < n; ++r) {
+      const bool f = (m >> r) & 1u;
+      const unsigned b = __ballot_sync(kFull, f);
+      if (f) {
+        const int p = s_warp[warp][r] + __popc(b & ((1u << lane) - 1u));
+        rows[p] = static_cast<int32_t>(t);
+        pos[t * n + r] = p;
+      } else if (t < T) {
+        pos[t * n + r] = -1;
+      }
+    }
+    __syncthreads();                               // s_warp is refilled by the next chunk
+  }
+}
+
+// Row i of the send buffers = row rows[i] of the rank's codes, scales, ids and
+// weights.  One warp per row, 16 bytes of codes per lane per step.
+__global__ void __launch_bounds__(256) ep_gather_rows_kernel(
+    const uint8_t* __restrict__ codes, const float* __restrict__ scales,
+    const int32_t* __restrict__ ids, const float* __restrict__ w, int64_t T, int64_t H, int k,
+    const int32_t* __restrict__ rows, int64_t n_rows, uint8_t* __restrict__ codes_out,
+    float* __restrict__ scales_out, int32_t* __restrict__ ids_out, float* __restrict__ w_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nchunk = H / 16;
+  for (int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; i < n_rows;
+       i += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t t = __ldg(rows + i);
+    if (!W4A8_IN_BOUNDS(t >= 0 && t < T)) continue;   // warp-uniform
+    const uint4* src = reinterpret_cast<const uint4*>(codes + t * H);
+    uint4* dst = reinterpret_cast<uint4*>(codes_out + i * H);
+    for (int64_t c = lane; c < nchunk; c += 32) dst[c] = __ldg(src + c);
+    for (int j = lane; j < k; j += 32) {
+      ids_out[i * k + j] = __ldg(ids + t * k + j);
+      w_out[i * k + j] = __ldg(w + t * k + j);
+    }
+    if (lane == 0) scales_out[i] = __ldg(scales + t);
+  }
+}
+
+// out[t] = bf16(sum over ranks r ascending with pos[t, r] >= 0 of back[pos[t, r]]),
+// float32 sums; a token that went nowhere gets zeros.  One thread per 8 columns.
+__global__ void __launch_bounds__(256) ep_combine_rows_kernel(const float* __restrict__ back,
+                                                              int64_t n_rows, int64_t H,
+                                                              const int32_t* __restrict__ pos,
+                                                              int64_t T, int n,
+                                                              __nv_bfloat16* __restrict__ out) {
+  const int64_t nc = H / 8;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < T * nc;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = idx / nc, c = idx - t * nc;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int r = 0; r < n; ++r) {
+      const int64_t p = __ldg(pos + t * n + r);
+      if (p < 0 || !W4A8_IN_BOUNDS(p < n_rows)) continue;
+      const float4* src = reinterpret_cast<const float4*>(back + p * H + c * 8);
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      q[i] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    *reinterpret_cast<uint4*>(out + t * H + c * 8) = make_uint4(q[0], q[1], q[2], q[3]);
+  }
+}
+
 // Debug build: point g_debug_latch at the library's device error latch (once
 // per device, before the first checked kernel).  Release build: nothing.
 cudaError_t ensure_debug_latch() {
@@ -1141,6 +1281,35 @@ cudaError_t launch_act_quant_group(const void* x_bf16, const float* x_f32, int64
 cudaError_t launch_dense_tables(int32_t* offsets, int32_t* tile_prefix, int64_t T, int tile_n,
                                 cudaStream_t s) {
   dense_tables_kernel<<<1, 32, 0, s>>>(offsets, tile_prefix, static_cast<int32_t>(T), tile_n);
+  return cudaGetLastError();
+}
+
+
+cudaError_t launch_ep_plan(const int32_t* topk_ids, int64_t T, int k, int E, int n_ranks,
+                           int32_t* counts, int32_t* rows, int32_t* pos, cudaStream_t s) {
+  if (n_ranks < 1 || n_ranks > kEpMaxRanks) return cudaErrorInvalidValue;
+  ep_plan_kernel<<<1, kPlanThreads, 0, s>>>(topk_ids, T, k, E, n_ranks, counts, rows, pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_gather_rows(const uint8_t* codes, const float* scales, const int32_t* ids,
+                                  const float* w, int64_t T, int64_t H, int k, const int32_t* rows,
+                                  int64_t n_rows, uint8_t* codes_out, float* scales_out,
+                                  int32_t* ids_out, float* w_out, int num_sms, cudaStream_t s) {
+  if (n_rows == 0) return cudaSuccess;
+  if (cudaError_t err = ensure_debug_latch()) return err;
+  ep_gather_rows_kernel<<<grid_for(n_rows * 32, 256, num_sms), 256, 0, s>>>(
+      codes, scales, ids, w, T, H, k, rows, n_rows, codes_out, scales_out, ids_out, w_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_combine_rows(const float* back, int64_t n_rows, int64_t H,
+                                   const int32_t* pos, int64_t T, int n_ranks, void* out,
+                                   int num_sms, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (cudaError_t err = ensure_debug_latch()) return err;
+  ep_combine_rows_kernel<<<grid_for(T * (H / 8), 256, num_sms), 256, 0, s>>>(
+      back, n_rows, H, pos, T, n_ranks, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }
 

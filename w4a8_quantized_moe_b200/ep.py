@@ -16,6 +16,14 @@ each rank's own batch of tokens:
 4. combine: reduce-scatter (sum) of the partial sums, so each rank receives
    the complete sums of its own tokens, which it rounds once to bf16.
 
+With ``dispatch="all_to_all"`` (large batches) steps 2-4 send each token
+only to the ranks that own one of its k experts: a dispatch plan (counts per
+rank, the rank-major token list), an all-to-all of the counts, all-to-all(v)
+of the token rows, the experts on the rows received, all-to-all(v) of the
+partial sums back, and a combine that sums each token's returned rows in
+rank order and rounds once to bf16.  The counts cross to the host once per
+step (the all-to-all(v) split sizes).
+
 Every compute step is a call into ``libw4a8.so``; the collectives are
 ``torch.distributed`` (NCCL between GPUs).  The compute steps are behind a
 small interface (``ops``) so that the bookkeeping and the collectives can be
@@ -87,6 +95,20 @@ class LibraryOps:
     def cast(self, x, out):
         return self._cast(x, out=out)
 
+    def plan(self, ids, E, n_ranks):
+        from . import w4a8_ep_dispatch_plan
+        return w4a8_ep_dispatch_plan(ids, E, n_ranks)
+
+    def gather(self, batch: PaddedBatch, T, rows, n_rows) -> PaddedBatch:
+        from . import w4a8_ep_gather_rows
+        c, s, i, w = w4a8_ep_gather_rows(batch.codes[:T], batch.scales[:T], batch.ids[:T],
+                                         batch.weights[:T], rows, n_rows)
+        return PaddedBatch(codes=c, scales=s, ids=i, weights=w)
+
+    def combine(self, back, pos, out):
+        from . import w4a8_ep_combine_rows
+        return w4a8_ep_combine_rows(back, pos, out=out)
+
 
 class ExpertParallelMoE:
     """This rank's share of an expert-parallel W4A8 layer.
@@ -98,10 +120,14 @@ class ExpertParallelMoE:
     ``group`` is the process group (default: the world).
     ``tokens_per_rank``: if every rank always calls with this many tokens,
     the step skips the collective that agrees on the padded batch size.
+    ``dispatch``: ``"all_gather"`` (every token to every rank; decode) or
+    ``"all_to_all"`` (each token to the ranks of its experts; prefill).  Every
+    rank of the group must use the same.
     """
 
     def __init__(self, weights_local, E: int, k: int, e_begin: int, e_count: int, H: int,
-                 I: int, group=None, ops=None, tokens_per_rank: Optional[int] = None):
+                 I: int, group=None, ops=None, tokens_per_rank: Optional[int] = None,
+                 dispatch: str = "all_gather"):
         import torch.distributed as dist
         self.dist, self.group = dist, group
         self.world = dist.get_world_size(group)
@@ -113,6 +139,14 @@ class ExpertParallelMoE:
         self.weights_local = weights_local
         self.ops = ops if ops is not None else LibraryOps()
         self.tokens_per_rank = tokens_per_rank
+        if dispatch not in ("all_gather", "all_to_all"):
+            raise ValueError(f"dispatch must be 'all_gather' or 'all_to_all', not {dispatch!r}")
+        self.dispatch = dispatch
+        if dispatch == "all_to_all" and e_count:
+            # the rank's range must be the one the dispatch plan assigns it
+            if (e_begin, e_count) != expert_partition(E, self.world)[self.rank]:
+                raise ValueError("all_to_all dispatch needs the contiguous expert_partition "
+                                 "ranges")
         self._bufs = {}
 
     @classmethod
@@ -155,6 +189,8 @@ class ExpertParallelMoE:
 
     def __call__(self, hidden: torch.Tensor, logits: torch.Tensor,
                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if self.dispatch == "all_to_all":
+            return self._all_to_all_step(hidden, logits, out)
         dist, group = self.dist, self.group
         T = hidden.shape[0]
         dev = hidden.device
@@ -180,6 +216,45 @@ class ExpertParallelMoE:
             out = torch.empty(T, self.H, dtype=torch.bfloat16, device=dev)
         if T:
             self.ops.cast(summed[:T], out)
+        return out
+
+
+    def _all_to_all_step(self, hidden, logits, out):
+        dist, group, G = self.dist, self.group, self.world
+        H, k = self.H, self.k
+        T = hidden.shape[0]
+        dev = hidden.device
+        loc = PaddedBatch(codes=torch.empty(T, H, dtype=torch.uint8, device=dev),
+                          scales=torch.empty(T, dtype=torch.float32, device=dev),
+                          ids=torch.empty(T, k, dtype=torch.int32, device=dev),
+                          weights=torch.empty(T, k, dtype=torch.float32, device=dev))
+        self.ops.quant_route(hidden, logits, k, loc)
+        counts, rows, pos = self.ops.plan(loc.ids, self.E, G)
+        send = counts.to(torch.int64)
+        recv = torch.empty_like(send)
+        dist.all_to_all_single(recv, send, group=group)
+        send_l, recv_l = send.tolist(), recv.tolist()
+        n_send, n_recv = sum(send_l), sum(recv_l)
+        sb = self.ops.gather(loc, T, rows, n_send)
+        rb = PaddedBatch(codes=torch.empty(n_recv, H, dtype=torch.uint8, device=dev),
+                         scales=torch.empty(n_recv, dtype=torch.float32, device=dev),
+                         ids=torch.empty(n_recv, k, dtype=torch.int32, device=dev),
+                         weights=torch.empty(n_recv, k, dtype=torch.float32, device=dev))
+        for got, sent in ((rb.codes, sb.codes), (rb.scales, sb.scales), (rb.ids, sb.ids),
+                          (rb.weights, sb.weights)):
+            dist.all_to_all_single(got, sent, output_split_sizes=recv_l,
+                                   input_split_sizes=send_l, group=group)
+        partial = torch.zeros(n_recv, H, dtype=torch.float32, device=dev)
+        if self.e_count and n_recv:
+            self.ops.experts(rb.codes, rb.scales, rb.ids, rb.weights, self.E, self.e_begin,
+                             self.weights_local, partial)
+        back = torch.empty(n_send, H, dtype=torch.float32, device=dev)
+        dist.all_to_all_single(back, partial, output_split_sizes=send_l,
+                               input_split_sizes=recv_l, group=group)
+        if out is None:
+            out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        if T:
+            self.ops.combine(back, pos, out)
         return out
 
 
