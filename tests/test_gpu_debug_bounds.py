@@ -6,7 +6,8 @@ one out of range raises W4A8_ERR_DEVICE_INDEX at the next
 w4a8_check_device_error and the access is skipped.  The forward and
 expert-parallel parity cases run on it in a child process: they must pass
 with no check firing (each test ends with w4a8_check_device_error), and an
-expert id outside [-1, E) given to w4a8_moe_forward_experts must be reported.
+expert id outside [-1, E) given to w4a8_moe_forward_experts must be reported,
+as must bad indices given to the all-to-all row gather and combine.
 """
 import os
 import subprocess
@@ -34,7 +35,8 @@ def test_parity_cases_on_the_bounds_checking_build():
                         "no:cacheprovider", os.path.join(HERE, "test_gpu_forward.py"),
                         os.path.join(HERE, "test_gpu_ep.py"), "-k",
                         "tiny_workload or ragged or multi_block or zipf_empty or zero_token_row "
-                        "or padding or route_topk"],
+                        "or padding or route_topk or dispatch_plan or gather_and_combine "
+                        "or bad_send_rows"],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
     tail = "\n".join((r.stdout + r.stderr).splitlines()[-15:])
     assert r.returncode == 0, tail

@@ -241,3 +241,29 @@ def test_all_to_all_step_emulated(cfg, G, tokens):
         print(f"\n[{cfg.name}, rank {s} of {G}, {hidden.shape[0]} tokens] vs layer: "
               f"{same:.5f} bit-equal, rel-Frobenius {dist:.2e}")
         assert same >= 0.999 and dist <= 1e-4
+
+
+def test_bad_send_rows_are_reported_by_the_debug_build():
+    """Only on the bounds-checking build (W4A8_LIBRARY=debug): a send-row
+    index outside [0, T) and a send-list index outside [0, n_rows) are skipped
+    and raise the device latch.  The release build does not check them, so the
+    test does not run there."""
+    if not w4.w4a8_build_flags() & 1:
+        pytest.skip("release build: indices are not checked")
+    T, H, k = 8, 128, 2
+    codes = torch.zeros(T, H, dtype=torch.uint8, device="cuda")
+    scales = torch.ones(T, dtype=torch.float32, device="cuda")
+    ids = torch.zeros(T, k, dtype=torch.int32, device="cuda")
+    w = torch.ones(T, k, dtype=torch.float32, device="cuda")
+    rows = torch.tensor([0, 3, T + 5, 1], dtype=torch.int32, device="cuda")
+    c, s, i, ww = w4.w4a8_ep_gather_rows(codes, scales, ids, w, rows, 4)
+    with pytest.raises(w4.W4A8Error, match="DEVICE_INDEX"):
+        w4.w4a8_check_device_error()
+    back = torch.ones(4, H, dtype=torch.float32, device="cuda")
+    pos = torch.full((T, 2), -1, dtype=torch.int32, device="cuda")
+    pos[0, 0], pos[1, 1], pos[2, 0] = 0, 9, 3          # 9 is past the 4 rows
+    out = w4.w4a8_ep_combine_rows(back, pos)
+    with pytest.raises(w4.W4A8Error, match="DEVICE_INDEX"):
+        w4.w4a8_check_device_error()
+    assert out[0].float().eq(1).all() and out[1].float().eq(0).all()
+    w4.w4a8_check_device_error()                       # the latch was cleared
