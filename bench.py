@@ -227,6 +227,19 @@ def shared_work(cfg):
     return s1, s2
 
 
+def shared_fused(w4, cfg, variant: str) -> bool:
+    """Whether the library runs the shared expert's GEMMs inside the routed GEMM
+    launches for this workload: decode-sized batches (at most 32 tokens per
+    expert on average) without split tiling, the default decode shapes, and
+    W4A8_SHARED_FUSED not 0."""
+    if variant != "w4a8+shared" or os.environ.get("W4A8_SHARED_FUSED", "1") == "0":
+        return False
+    if int(os.environ.get("W4A8_GEMM_DECODE_SHAPE", "0") or 0) != 0:
+        return False
+    no_split = w4.w4a8_moe_forward_launches(cfg.T, cfg.E, cfg.k) == KERNELS_PER_STEP
+    return cfg.T * cfg.k <= 32 * cfg.E and no_split
+
+
 def layer_work(cfg, counts, variant: str = "w4a8"):
     """Algorithmic bytes and FLOPs of the whole layer (one step): the HBM bytes
     of every active expert's weights and scales, the hidden states and logits
@@ -471,7 +484,16 @@ def run_single(cfg, args, device, w4, cpu_tokens: int):
         roofline_layer=roofline(layer_work(cfg, counts, args.variant), ms / args.steps, prefill,
                                 pk),
         clocks=clk.summary(), digest=digest, l2_bytes=g1["bytes"] + g2["bytes"])
-    if shared:   # the shared expert's slower GEMM against the same peak
+    if shared and shared_fused(w4, cfg, args.variant):
+        # one launch per projection carries both experts' tiles: the dominant
+        # launch's work is the routed projection's plus the shared expert's
+        s1, s2 = shared_work(cfg)
+        fw = {k_: (g1 if gi == 2 else g2)[k_] + (s1 if gi == 2 else s2)[k_]
+              for k_ in ("bytes", "flops")}
+        res["roofline"] = roofline(fw, stage_ms[gi], prefill, pk,
+                                   kname + " (with the shared expert)")
+        res["shared_fused"] = True
+    elif shared:   # the shared expert's slower GEMM against the same peak
         s1, s2 = shared_work(cfg)
         # stages 6..9: shared input quantisation, gate/up GEMM, requantisation, down GEMM
         si = 1 if stage_ms[7] >= stage_ms[9] else 3
@@ -489,7 +511,11 @@ def step_launches(w4, cfg, variant: str) -> int:
     if variant == "channel-int8":
         return KERNELS_PER_STEP
     n = w4.w4a8_moe_forward_launches(cfg.T, cfg.E, cfg.k)
-    return n + (SHARED_KERNELS_PER_STEP if variant == "w4a8+shared" else 0)
+    if variant != "w4a8+shared":
+        return n
+    # the shared GEMMs inside the routed launches: tables and the two quantisers
+    return n + (SHARED_KERNELS_PER_STEP - 2 if shared_fused(w4, cfg, variant)
+                else SHARED_KERNELS_PER_STEP)
 
 
 def config_fields(cfg, res, args, world=1, parallelism="single"):
@@ -505,6 +531,9 @@ def config_fields(cfg, res, args, world=1, parallelism="single"):
                       "with per-stage events, %.4f ms per step)" % (res["ms_eager"] / args.steps))
     if res.get("digest"):
         c["inputs_sha256"] = res["digest"]
+    if args.variant == "w4a8+shared":
+        c["shared_gemms"] = ("second phase of the routed GEMM launches" if res.get("shared_fused")
+                             else "launches of their own")
     return c
 
 

@@ -470,6 +470,12 @@ W4A8_API size_t w4a8_moe_shared_workspace_size(int64_t T, int64_t H, int64_t I, 
  * The routed arguments, aux and errors are those of w4a8_moe_forward;
  * shared_aux those of w4a8_shared_expert_forward.  The workspace size is
  * w4a8_moe_shared_workspace_size.
+ * Decode-sized calls (T k <= 32 E, without split tiling) run the shared
+ * expert's two GEMMs inside the routed GEMM launches, as their second phase
+ * (each CTA takes shared tiles after its routed ones); the shared stage
+ * events 2/3 and 6/7 then bracket nothing and the routed GEMM stages include
+ * the shared GEMMs.  The environment variable W4A8_SHARED_FUSED=0 keeps them
+ * in launches of their own.
  */
 W4A8_API w4a8_status w4a8_moe_forward_shared(
     const void* hidden_bf16, const float* logits, const int32_t* w13_packed,

@@ -15,7 +15,7 @@ import torch
 import oracle
 import workloads
 import w4a8_quantized_moe_b200 as w4
-from gpu_helpers import codes_agree, f64, rel_fro, small_case
+from gpu_helpers import aux_buffers, codes_agree, f64, rel_fro, small_case
 
 pytestmark = pytest.mark.gpu
 
@@ -107,6 +107,84 @@ def test_layer_with_shared_expert(cfg):
     e_plain = rel_fro(f64(plain), res["out"])
     print(f"\n[{cfg.name} + shared] out {e_out:.2e} (routed only: {e_plain:.2e})")
     assert e_out <= 2e-3 and e_plain > 0.05
+
+
+def _shared_aux(T, H, I):
+    dev = "cuda"
+    return dict(act_codes=torch.empty(T, H, dtype=torch.uint8, device=dev),
+                act_scales=torch.empty(T, H // 128, dtype=torch.float32, device=dev),
+                h=torch.empty(T, I, dtype=torch.float32, device=dev),
+                h_codes=torch.empty(T, I, dtype=torch.uint8, device=dev),
+                h_scales=torch.empty(T, I // 128, dtype=torch.float32, device=dev))
+
+
+@pytest.mark.parametrize("cfg", [
+    workloads.CONFIGS[0],
+    workloads.MoEConfig("fused_even_groups", T=48, H=512, I=256, E=16, k=2, seed=41),
+    # gate/up K = 384 (three groups: the unpaired decode shape), two shared token blocks
+    workloads.MoEConfig("fused_odd_groups", T=100, H=384, I=256, E=32, k=2, seed=42),
+    workloads.MoEConfig("fused_one_token", T=1, H=256, I=128, E=8, k=2, seed=43),
+], ids=lambda c: c.name)
+def test_shared_gemms_inside_the_routed_launches(cfg):
+    """Decode-sized, unsplit batches: the shared expert's two GEMMs run as the
+    second phase of the routed GEMM launches (64-token tiles).  Its h and y
+    must be those of the shared expert's own launches (128-token tiles: the
+    same float32 arithmetic per element), and the layer must match the oracle."""
+    assert cfg.T * cfg.k <= 32 * cfg.E and cfg.T * cfg.k < 8 * cfg.E   # decode, no split
+    hidden, logits, w13, w2 = small_case(cfg)
+    ws13, ws2 = _shared_weights(cfg)
+    layer = w4.W4A8MoELayerShared.from_bf16_with_shared(w13.cuda(), w2.cuda(), cfg.k,
+                                                        ws13.cuda(), ws2.cuda())
+    Is = ws2.shape[1]
+    fused = _shared_aux(cfg.T, cfg.H, Is)
+    aux = aux_buffers(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k)
+    out = layer(hidden.cuda(), logits.cuda(), aux=aux, shared_aux=fused)
+    alone = _shared_aux(cfg.T, cfg.H, Is)
+    y_alone = layer.shared(hidden.cuda(), aux=alone)
+    w4.w4a8_check_device_error()
+    assert torch.equal(fused["act_codes"], alone["act_codes"])
+    assert torch.equal(fused["act_scales"], alone["act_scales"])
+    same_h = float((fused["h"] == alone["h"]).float().mean())
+    e_h = rel_fro(fused["h"].cpu().numpy(), alone["h"].cpu().numpy())
+    assert e_h <= 1e-6, e_h
+    frac, dist = codes_agree(fused["h_codes"].cpu().numpy(), alone["h_codes"].cpu().numpy())
+    assert frac >= 0.999 and dist <= 1, (frac, dist)
+    # the shared y of the fused down launch: the output is the routed sum from
+    # the same call's Y rows plus the shared expert's own y, rounded once to bf16
+    Y = aux["y_rows"].double().cpu().numpy()
+    w = aux["topk_w"].double().cpu().numpy()
+    rows = aux["row_of"].cpu().numpy()
+    ys = y_alone.double().cpu().numpy()
+    ref = np.einsum("tj,tjh->th", w, Y[rows]) + ys
+    # one bf16 rounding (half a unit, 2^-9 relative), float32 summation order
+    mag = np.einsum("tj,tjh->th", np.abs(w), np.abs(Y[rows])) + np.abs(ys)
+    dev_ = np.abs(f64(out) - ref)
+    assert np.all(dev_ <= 2.0 ** -8 * np.abs(ref) + 1e-6 * mag + 1e-30), \
+        float((dev_ / (np.abs(ref) + 1e-30)).max())
+    store = oracle.ExpertStore(cfg.E, lambda e: (f64(w13[e]), f64(w2[e])))
+    sh = (*oracle.quant_fp8_block(f64(ws13)), *oracle.quant_fp8_block(f64(ws2)))
+    res = oracle.moe_forward(f64(hidden), logits.numpy(), store, cfg.k, shared=sh)
+    e_out = rel_fro(f64(out), res["out"])
+    print(f"\n[{cfg.name}] shared h bit-equal {same_h:.5f} (rel {e_h:.1e}) against its own "
+          f"launches; layer out {e_out:.2e}")
+    assert e_out <= 2e-3
+
+
+def test_shared_gemms_in_launches_of_their_own():
+    """The same decode cases with W4A8_SHARED_FUSED=0 (the shared expert's GEMMs
+    in launches of their own), in a child process."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, W4A8_SHARED_FUSED="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p",
+                        "no:cacheprovider", os.path.join(here, "test_gpu_shared.py"), "-k",
+                        "test_layer_with_shared_expert and not full_size"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-15:])
+    assert r.returncode == 0, tail
+    assert " passed" in r.stdout, tail
 
 
 @pytest.mark.parametrize("ci", [1, 3], ids=lambda i: workloads.CONFIGS[i].name)

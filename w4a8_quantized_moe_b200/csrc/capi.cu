@@ -502,12 +502,29 @@ w4a8_status check_shared_shape(int64_t T, int64_t H, int64_t I) {
 // GEMM + SwiGLU, group-requantise h, down GEMM into y [T, H] float32.
 // Stage events (aux->stage_events, 8 handles): 0/1 input quantisation, 2/3
 // gate/up GEMM, 4/5 requantisation of h, 6/7 down GEMM.
-w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_codes,
-                                const float* w13_scales, const uint8_t* w2_codes,
-                                const float* w2_scales, int64_t T, int64_t H, int64_t I,
-                                float* y, SharedBufs b, const w4a8_shared_aux* aux,
-                                const DeviceInfo& di, cudaStream_t s) {
+// The FP8-block shared expert's steps, set up once per call: its tensor maps,
+// GEMM arguments and stage events.  The steps run in order; in a routed
+// decode call its two GEMMs run inside the routed GEMM launches instead.
+struct SharedRun {
+  CUtensorMap tw1, ta1, tw2, ta2;
+  GemmArgs g1, g2;
+  int ctas1 = 0, ctas2 = 0, tile_n = 0;
+  SharedBufs b;
+  const void* hidden = nullptr;
+  int64_t T = 0, H = 0, I = 0;
   void* const* ev = nullptr;
+};
+
+cudaError_t shared_record(const SharedRun& r, int i, cudaStream_t s) {
+  return r.ev && r.ev[i] ? cudaEventRecord(static_cast<cudaEvent_t>(r.ev[i]), s) : cudaSuccess;
+}
+
+// tile_n: token rows per tile of the shared expert's GEMM shape
+w4a8_status shared_setup(SharedRun& r, const void* hidden_bf16, const uint8_t* w13_codes,
+                         const float* w13_scales, const uint8_t* w2_codes,
+                         const float* w2_scales, int64_t T, int64_t H, int64_t I, float* y,
+                         SharedBufs b, const w4a8_shared_aux* aux, const DeviceInfo& di,
+                         int tile_n) {
   if (aux) {
     auto pick = [](auto* user, auto* ws) { return user ? user : ws; };
     b.act_codes = pick(aux->act_codes, b.act_codes);
@@ -519,43 +536,34 @@ w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_code
                           static_cast<const void*>(b.h), static_cast<const void*>(b.h_codes),
                           static_cast<const void*>(b.h_scales)})
       if (!aligned16(p)) return fail(W4A8_ERR_INVALID_ARG, "aux buffers must be 16-byte aligned");
-    ev = aux->stage_events;
+    r.ev = aux->stage_events;
   }
+  r.b = b;
+  r.hidden = hidden_bf16;
+  r.T = T;
+  r.H = H;
+  r.I = I;
+  r.tile_n = tile_n;
   // E4M3 weights [rows, K] bytes, 128-byte swizzle: boxes of 64 rows (the
   // gate and up halves of a gate/up tile) or 128 rows (down); activation codes
   // [T, K] in 16-row boxes, as for the routed experts.
-  CUtensorMap tw1, ta1, tw2, ta2;
-  if (w4a8_status st = encode_u8_2d(&tw1, w13_codes, static_cast<uint64_t>(H),
+  if (w4a8_status st = encode_u8_2d(&r.tw1, w13_codes, static_cast<uint64_t>(H),
                                     static_cast<uint64_t>(2 * I), 128, 64,
                                     CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
-  if (w4a8_status st = encode_u8_2d(&ta1, b.act_codes, static_cast<uint64_t>(H),
+  if (w4a8_status st = encode_u8_2d(&r.ta1, b.act_codes, static_cast<uint64_t>(H),
                                     static_cast<uint64_t>(T), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
-  if (w4a8_status st = encode_u8_2d(&tw2, w2_codes, static_cast<uint64_t>(I),
+  if (w4a8_status st = encode_u8_2d(&r.tw2, w2_codes, static_cast<uint64_t>(I),
                                     static_cast<uint64_t>(H), 128, 128,
                                     CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
-  if (w4a8_status st = encode_u8_2d(&ta2, b.h_codes, static_cast<uint64_t>(I),
+  if (w4a8_status st = encode_u8_2d(&r.ta2, b.h_codes, static_cast<uint64_t>(I),
                                     static_cast<uint64_t>(T), 128, 16, CU_TENSOR_MAP_SWIZZLE_128B))
     return st;
-  auto record = [&](int i) -> cudaError_t {
-    return ev && ev[i] ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
-  };
-  cudaError_t err = cudaSuccess;
-#define W4A8_STEP(call, what)                              \
-  do {                                                     \
-    err = (call);                                          \
-    if (err != cudaSuccess) return cuda_fail(err, what);   \
-  } while (0)
-  const int tile_n = grouped_gemm_tile_n(false);
-  W4A8_STEP(launch_dense_tables(b.tables, b.tables + 2, T, tile_n, s), "dense tables launch");
-  W4A8_STEP(record(0), "cudaEventRecord");
-  W4A8_STEP(launch_act_quant_group(hidden_bf16, nullptr, T, H, b.act_codes, b.act_scales, di.sms, s),
-            "shared input quantisation launch");
-  W4A8_STEP(record(1), "cudaEventRecord");
   const int64_t tiles_n = (T + tile_n - 1) / tile_n;
-  GemmArgs g1{};
+  GemmArgs& g1 = r.g1;
+  g1 = GemmArgs{};
   g1.K = static_cast<int>(H);
   g1.n_rows = static_cast<int>(2 * I);
   g1.half_rows = static_cast<int>(I);
@@ -571,15 +579,9 @@ w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_code
   g1.nb_fastest = 1;
   g1.n_seg_rows = T;
   g1.n_tokens = T;
-  const int ctas1 = static_cast<int>(std::min<int64_t>(tiles_n * (I / 64), di.sms));
-  W4A8_STEP(record(2), "cudaEventRecord");
-  W4A8_STEP(launch_fp8_block_gemm(true, tw1, ta1, g1, ctas1, s), "shared gate/up GEMM launch");
-  W4A8_STEP(record(3), "cudaEventRecord");
-  W4A8_STEP(record(4), "cudaEventRecord");
-  W4A8_STEP(launch_act_quant_group(nullptr, b.h, T, I, b.h_codes, b.h_scales, di.sms, s),
-            "shared intermediate quantisation launch");
-  W4A8_STEP(record(5), "cudaEventRecord");
-  GemmArgs g2 = g1;
+  r.ctas1 = static_cast<int>(std::min<int64_t>(tiles_n * (I / 64), di.sms));
+  GemmArgs& g2 = r.g2;
+  g2 = g1;
   g2.K = static_cast<int>(I);
   g2.n_rows = static_cast<int>(H);
   g2.half_rows = 0;
@@ -587,12 +589,71 @@ w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_code
   g2.wscale = w2_scales;
   g2.out = y;
   g2.out_ld = H;
-  const int ctas2 = static_cast<int>(std::min<int64_t>(tiles_n * (H / kGroup), di.sms));
-  W4A8_STEP(record(6), "cudaEventRecord");
-  W4A8_STEP(launch_fp8_block_gemm(false, tw2, ta2, g2, ctas2, s), "shared down GEMM launch");
-  W4A8_STEP(record(7), "cudaEventRecord");
-#undef W4A8_STEP
+  r.ctas2 = static_cast<int>(std::min<int64_t>(tiles_n * (H / kGroup), di.sms));
   return W4A8_OK;
+}
+
+#define W4A8_STEP(call, what)                              \
+  do {                                                     \
+    cudaError_t err_ = (call);                             \
+    if (err_ != cudaSuccess) return cuda_fail(err_, what); \
+  } while (0)
+
+// the dense tables of the one expert, and the input's group quantisation
+w4a8_status shared_front(const SharedRun& r, const DeviceInfo& di, cudaStream_t s) {
+  W4A8_STEP(launch_dense_tables(r.b.tables, r.b.tables + 2, r.T, r.tile_n, s),
+            "dense tables launch");
+  W4A8_STEP(shared_record(r, 0, s), "cudaEventRecord");
+  W4A8_STEP(launch_act_quant_group(r.hidden, nullptr, r.T, r.H, r.b.act_codes, r.b.act_scales,
+                                   di.sms, s),
+            "shared input quantisation launch");
+  W4A8_STEP(shared_record(r, 1, s), "cudaEventRecord");
+  return W4A8_OK;
+}
+
+w4a8_status shared_gemm(const SharedRun& r, bool gate_up, cudaStream_t s) {
+  W4A8_STEP(shared_record(r, gate_up ? 2 : 6, s), "cudaEventRecord");
+  W4A8_STEP(gate_up ? launch_fp8_block_gemm(true, r.tw1, r.ta1, r.g1, r.ctas1, s)
+                    : launch_fp8_block_gemm(false, r.tw2, r.ta2, r.g2, r.ctas2, s),
+            gate_up ? "shared gate/up GEMM launch" : "shared down GEMM launch");
+  W4A8_STEP(shared_record(r, gate_up ? 3 : 7, s), "cudaEventRecord");
+  return W4A8_OK;
+}
+
+// h requantised per token and 128-group
+w4a8_status shared_mid(const SharedRun& r, const DeviceInfo& di, cudaStream_t s) {
+  W4A8_STEP(shared_record(r, 4, s), "cudaEventRecord");
+  W4A8_STEP(launch_act_quant_group(nullptr, r.b.h, r.T, r.I, r.b.h_codes, r.b.h_scales, di.sms,
+                                   s),
+            "shared intermediate quantisation launch");
+  W4A8_STEP(shared_record(r, 5, s), "cudaEventRecord");
+  return W4A8_OK;
+}
+#undef W4A8_STEP
+
+w4a8_status shared_forward_impl(const void* hidden_bf16, const uint8_t* w13_codes,
+                                const float* w13_scales, const uint8_t* w2_codes,
+                                const float* w2_scales, int64_t T, int64_t H, int64_t I,
+                                float* y, SharedBufs b, const w4a8_shared_aux* aux,
+                                const DeviceInfo& di, cudaStream_t s) {
+  SharedRun r;
+  if (w4a8_status st = shared_setup(r, hidden_bf16, w13_codes, w13_scales, w2_codes, w2_scales, T,
+                                    H, I, y, b, aux, di, grouped_gemm_tile_n(false)))
+    return st;
+  if (w4a8_status st = shared_front(r, di, s)) return st;
+  if (w4a8_status st = shared_gemm(r, true, s)) return st;
+  if (w4a8_status st = shared_mid(r, di, s)) return st;
+  return shared_gemm(r, false, s);
+}
+
+// Whether a routed decode call runs the shared expert's GEMMs inside its own
+// GEMM launches (W4A8_SHARED_FUSED = 0 keeps them apart).
+bool shared_fused_by_default() {
+  static const int v = [] {
+    const char* e = std::getenv("W4A8_SHARED_FUSED");
+    return e ? std::atoi(e) : 1;
+  }();
+  return v != 0;
 }
 
 // The layer's optional FP8-block shared expert.
@@ -746,11 +807,24 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
 
   // the shared expert first: it reads only the hidden states, and the combine
   // adds its output
+  // decode: the shared expert's two GEMMs run inside the routed GEMM launches
+  // (their second phase, on the CTAs that finish their routed tiles first);
+  // otherwise it runs first, in launches of its own
+  const bool fuse_shared = sh && !i8 && !split && decode && shared_fused_by_default() &&
+                           grouped_gemm_shared_fusable();
+  SharedRun sr;
   if (sh) {
-    if (w4a8_status st = shared_forward_impl(hidden_bf16, sh->w13_codes, sh->w13_scales,
-                                             sh->w2_codes, sh->w2_scales, T, H, sh->I, sb.y, sb,
-                                             sh->aux, di, s))
+    if (w4a8_status st = shared_setup(sr, hidden_bf16, sh->w13_codes, sh->w13_scales,
+                                      sh->w2_codes, sh->w2_scales, T, H, sh->I, sb.y, sb, sh->aux,
+                                      di, fuse_shared ? grouped_gemm_shared_tile_n()
+                                                      : grouped_gemm_tile_n(false)))
       return st;
+    if (w4a8_status st = shared_front(sr, di, s)) return st;
+    if (!fuse_shared) {
+      if (w4a8_status st = shared_gemm(sr, true, s)) return st;
+      if (w4a8_status st = shared_mid(sr, di, s)) return st;
+      if (w4a8_status st = shared_gemm(sr, false, s)) return st;
+    }
   }
   // routing first: the activation quantiser writes each token's codes to its
   // segment rows as well, so both GEMMs read contiguous activation tiles
@@ -794,6 +868,14 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
     W4A8_STEP(launch_grouped_gemm_split(true, tw1, ta1, ts1, tg1, g1, b.route.tile_prefix_wide,
                                         di.sms, s),
               "gate/up GEMM launch");
+  } else if (fuse_shared) {
+    // the shared expert's gate/up stage events bracket nothing: its GEMM is
+    // inside this launch
+    W4A8_STEP(shared_record(sr, 2, s), "cudaEventRecord");
+    W4A8_STEP(shared_record(sr, 3, s), "cudaEventRecord");
+    W4A8_STEP(launch_grouped_gemm_with_shared(true, decode, tw1, ta1, ts1, tg1, sr.tw1, sr.ta1,
+                                              g1, sr.g1, di.sms, s),
+              "gate/up GEMM launch (with the shared expert)");
   } else {
     W4A8_STEP(i8 ? launch_grouped_gemm_i8(true, decode, tw1, ta1, g1, di.sms, s)
                  : launch_grouped_gemm(true, decode, tw1, ta1, ts1, tg1, g1, di.sms, s),
@@ -807,6 +889,8 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
                                i8 ? b.inter_rowsum : nullptr, parts ? b.inter_parts : nullptr),
             "intermediate quant launch");
   W4A8_STEP(record(7), "cudaEventRecord");
+  if (fuse_shared)
+    if (w4a8_status st = shared_mid(sr, di, s)) return st;
 
   GemmArgs g2{};
   g2.K = static_cast<int>(I);
@@ -835,6 +919,12 @@ w4a8_status moe_forward_impl(const void* hidden_bf16, const float* logits,
     W4A8_STEP(launch_grouped_gemm_split(false, tw2, ta2, ts2, tg2, g2, b.route.tile_prefix_wide,
                                         di.sms, s),
               "down GEMM launch");
+  } else if (fuse_shared) {
+    W4A8_STEP(shared_record(sr, 6, s), "cudaEventRecord");
+    W4A8_STEP(shared_record(sr, 7, s), "cudaEventRecord");
+    W4A8_STEP(launch_grouped_gemm_with_shared(false, decode, tw2, ta2, ts2, tg2, sr.tw2, sr.ta2,
+                                              g2, sr.g2, di.sms, s),
+              "down GEMM launch (with the shared expert)");
   } else {
     W4A8_STEP(i8 ? launch_grouped_gemm_i8(false, decode, tw2, ta2, g2, di.sms, s)
                  : launch_grouped_gemm(false, decode, tw2, ta2, ts2, tg2, g2, di.sms, s),

@@ -194,6 +194,10 @@ using Prefill16EpiEpilogueOffset = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2,
 using PrefillTileCorr = Shape<kTileNPrefill, 4, 5, 4, 3, 1, 4, 16, 2, 1, 2>;
 // E4M3-weight (FP8 block) shape: A from shared memory, no converter warps
 using F8Block = Shape<kTileNPrefill, 4, 4, 1, 3, 0, 4, 16, 2, 1, 0>;
+// ... at decode, as the second phase of a routed launch: 64 token rows, eight
+// epilogue warps of 32 columns (384 threads, as the routed decode shapes' 384
+// or within their 512)
+using F8Decode = Shape<kTileNShared, 6, 4, 1, 3, 0, 2, 32, 2, 1, 0>;
 // INT8 per-channel shapes: one accumulator per tile, single MMA issuer
 using I8Decode  = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 1, 1, 0>;
 using I8Decode2 = Shape<kTileNDecode, 16, 8, 8, 8, 1, 1, 32, 2, 1, 0>;  // 4 tiles x 2 chains
@@ -291,12 +295,20 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
   }
 }
 
-template <class S, bool kGateUp, bool kI8, bool kF8W>
-__global__ void __launch_bounds__(S::kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
-                        const __grid_constant__ CUtensorMap tmap_act,
-                        const __grid_constant__ CUtensorMap tmap_sc,
-                        const __grid_constant__ CUtensorMap tmap_gs, const GemmArgs a) {
+// One launch's work for one projection.  kPhase 0: the whole launch (TMEM
+// allocated and freed here).  Two phases of one launch (the routed experts,
+// then the shared expert): phase 1 allocates TMEM and returns it, and retires
+// its barriers at the end, because phase 2 lays out shared memory anew;
+// phase 2 takes the TMEM (phase_tmem) and frees it.  In a phase, the CTA's
+// place in the tile schedule is (phase_cta_x, phase_n_cta).
+template <class S, bool kGateUp, bool kI8, bool kF8W, int kPhase = 0>
+__device__ __forceinline__ uint32_t gemm_body(const CUtensorMap& tmap_w,
+                                              const CUtensorMap& tmap_act,
+                                              const CUtensorMap& tmap_sc,
+                                              const CUtensorMap& tmap_gs, const GemmArgs& a,
+                                              int phase_cta_x, int phase_n_cta,
+                                              uint32_t phase_tmem) {
+  static_assert(kPhase == 0 || !S::kCta2, "CTA pairs run as a launch of their own");
   constexpr int kTileN = S::kTileN, kWStages = S::kWStages, kBStages = S::kBStages;
   constexpr int kASlots = S::kASlots, kDBufs = S::kDBufs, kEpiN = S::kEpiN;
   constexpr int kBStageBytes = S::kBStageBytes, kUpBytes = S::kUpBytes;
@@ -352,8 +364,10 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   // CTA pairs: both CTAs of a cluster walk the same tiles (cta_x of n_cta);
   // this CTA takes weight-row block 2 mb + crank of the pair's block mb
   const uint32_t crank = kCta2 ? cluster_ctarank() : 0u;
-  const int cta_x = kCta2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int n_cta = kCta2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int cta_x = kPhase ? phase_cta_x
+                           : kCta2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_cta = kPhase ? phase_n_cta
+                           : kCta2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const int mb_count = (kGateUp ? a.half_rows / 64 : a.n_rows / kBM) / (kCta2 ? 2 : 1);
   const uint64_t tmo = a.timeout_ns;
   // token blocks of one expert whose activation rows (K bytes each) stay well
@@ -365,40 +379,44 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     return t;
   };
 
-  if (threadIdx.x == 0) {
+  // every barrier of this launch (or phase), with its arrival count
+  auto each_barrier = [&](auto&& f) {
     for (int s = 0; s < kWStages; ++s) {
-      mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], kF8W ? 1 : 4);  // E4M3 weights: released by the MMA commit
+      f(&wfull[s], 1);
+      f(&wempty[s], kF8W ? 1 : 4);  // E4M3 weights: released by the MMA commit
     }
     for (int s = 0; s < kBStages; ++s) {
-      mbar_init(&bfull[s], 1);
-      if (!kUniAB) mbar_init(&bempty[s], 1);
+      f(&bfull[s], 1);
+      if (!kUniAB) f(&bempty[s], 1);
     }
     for (int s = 0; s < kASlots; ++s) {
-      mbar_init(&afull[s], kCta2 ? 8 : 4);  // pairs: both CTAs' converter warps (first CTA's)
-      mbar_init(&aempty[s], 1);
+      f(&afull[s], kCta2 ? 8 : 4);  // pairs: both CTAs' converter warps (first CTA's)
+      f(&aempty[s], 1);
     }
     for (int d = 0; d < kDBufs; ++d) {
-      if (!kUniAll) mbar_init(&dfull[d], kI8 ? S::kMmaWarps : 1);
+      if (!kUniAll) f(&dfull[d], kI8 ? S::kMmaWarps : 1);
       // each group is read by one set (of both CTAs of a pair, on the first CTA's barrier)
-      mbar_init(&dempty[d], S::kEpiPerSet * (kCta2 ? 2 : 1));
+      f(&dempty[d], S::kEpiPerSet * (kCta2 ? 2 : 1));
     }
     for (int i = 0; i < S::kEpiSets; ++i) {
-      mbar_init(&upfull[i], S::kEpiPerSet / 2);
-      mbar_init(&upempty[i], S::kEpiPerSet / 2);
+      f(&upfull[i], S::kEpiPerSet / 2);
+      f(&upempty[i], S::kEpiPerSet / 2);
     }
-    mbar_init(drain, S::kMmaWarps);
+    f(drain, S::kMmaWarps);
     for (int i = 0; i < S::kEpiSets * S::kEpiPerQuad; ++i) {
-      mbar_init(&sfull[i], 4);
-      mbar_init(&sempty[i], 4);
+      f(&sfull[i], 4);
+      f(&sempty[i], 4);
     }
     for (int i = 0; i < S::kTileScBufs; ++i) {
-      mbar_init(&tfull[i], 1);
+      f(&tfull[i], 1);
       // a tile's scales are read by one epilogue set (and, for the per-tile
       // correction, by the 4 converter warps)
-      mbar_init(&tempty[i], S::kEpiPerSet + (S::kOffsetTile ? 4 : 0));
+      f(&tempty[i], S::kEpiPerSet + (S::kOffsetTile ? 4 : 0));
     }
-    mbar_init(loopdone, S::kEpiPerSet);
+    f(loopdone, S::kEpiPerSet);
+  };
+  if (threadIdx.x == 0) {
+    each_barrier([](uint64_t* b, int count) { mbar_init(b, count); });
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -410,7 +428,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
     prefetch_tmap(&tmap_act);
     if (S::kOffsetTile) prefetch_tmap(&tmap_gs);
   }
-  if (warp == 0) {
+  if (kPhase != 2 && warp == 0) {
     if constexpr (kCta2) {
       tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
       tmem_relinquish_pair();
@@ -446,7 +464,7 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   // pairs: the other CTA's barriers are initialised before anything arrives on them
   if constexpr (kCta2) cluster_sync();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = kPhase == 2 ? phase_tmem : *tmem_slot;
   const int total = sTP[a.E] * mb_count;
   const int my_tiles = cta_x < total ? (total - cta_x + n_cta - 1) / n_cta : 0;
   const int n_groups = my_tiles * G;  // every tile has G groups
@@ -1248,11 +1266,45 @@ __global__ void __launch_bounds__(S::kThreads, 1)
   // pairs: the first CTA's MMAs read and write both CTAs' TMEM and the CTAs
   // arrive on each other's barriers: neither frees or exits before both are done
   if constexpr (kCta2) cluster_sync();
-  if (warp == 0) {
+  if constexpr (kPhase == 1) {
+    // every copy and MMA of this phase has completed (each stage was waited
+    // on, the MMA issuers drained); the barriers' memory is reused next phase
+    if (threadIdx.x == 0) each_barrier([](uint64_t* b, int) { mbar_inval(b); });
+    __syncthreads();
+  } else if (warp == 0) {
     tc_fence_after();
     if constexpr (kCta2) tmem_dealloc_pair(tmem, kTmemCols);
     else tmem_dealloc(tmem, kTmemCols);
   }
+  return tmem;
+}
+
+template <class S, bool kGateUp, bool kI8, bool kF8W>
+__global__ void __launch_bounds__(S::kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                        const __grid_constant__ CUtensorMap tmap_act,
+                        const __grid_constant__ CUtensorMap tmap_sc,
+                        const __grid_constant__ CUtensorMap tmap_gs, const GemmArgs a) {
+  gemm_body<S, kGateUp, kI8, kF8W>(tmap_w, tmap_act, tmap_sc, tmap_gs, a, 0, 0, 0u);
+}
+
+// The routed experts' projection and the shared expert's in one launch: each
+// CTA runs its routed tiles, then its share of the shared expert's tiles,
+// which start on the CTAs whose routed share is one tile shorter.
+template <class SR, class SS, bool kGateUp>
+__global__ void __launch_bounds__(SR::kThreads > SS::kThreads ? SR::kThreads : SS::kThreads, 1)
+    grouped_gemm_shared_kernel(const __grid_constant__ CUtensorMap r_w,
+                               const __grid_constant__ CUtensorMap r_act,
+                               const __grid_constant__ CUtensorMap r_sc,
+                               const __grid_constant__ CUtensorMap r_gs,
+                               const __grid_constant__ CUtensorMap s_w,
+                               const __grid_constant__ CUtensorMap s_act, const GemmArgs ar,
+                               const GemmArgs as) {
+  const int n = static_cast<int>(gridDim.x), x = static_cast<int>(blockIdx.x);
+  const uint32_t tmem = gemm_body<SR, kGateUp, false, false, 1>(r_w, r_act, r_sc, r_gs, ar, x, n, 0u);
+  const int mb_r = kGateUp ? ar.half_rows / 64 : ar.n_rows / kBM;
+  const int first = (__ldg(ar.tile_prefix + ar.E) * mb_r) % n;
+  gemm_body<SS, kGateUp, false, true, 2>(s_w, s_act, s_w, s_act, as, (x + n - first) % n, n, tmem);
 }
 
 constexpr int kMaxSmemPerBlock = 232448;  // 227 KB opt-in limit of sm_100
@@ -1293,6 +1345,33 @@ cudaError_t launch_shape(const CUtensorMap& tmap_w, const CUtensorMap& tmap_act,
   }
   grouped_gemm_kernel<S, kGateUp, kI8, kF8W><<<num_ctas, S::kThreads, smem, s>>>(
       tmap_w, tmap_act, tmap_sc, tmap_gs, a);
+  return cudaGetLastError();
+}
+
+template <class SR, class SS, bool kGateUp>
+cudaError_t launch_two_phase(const CUtensorMap& rw, const CUtensorMap& ra, const CUtensorMap& rsc,
+                             const CUtensorMap& rgs, const CUtensorMap& sw, const CUtensorMap& sa,
+                             const GemmArgs& ar, const GemmArgs& as, int num_ctas,
+                             cudaStream_t s) {
+  constexpr int kThreads = SR::kThreads > SS::kThreads ? SR::kThreads : SS::kThreads;
+  constexpr int kSmemR = SR::smem_bytes(kGateUp, kMaxGroups, kMaxExperts, false);
+  constexpr int kSmemS = SS::smem_bytes(kGateUp, kMaxGroups, 1, true);
+  constexpr int kSmemMax = kSmemR > kSmemS ? kSmemR : kSmemS;
+  static_assert(kSmemMax <= kMaxSmemPerBlock, "shared memory");
+  auto kernel = grouped_gemm_shared_kernel<SR, SS, kGateUp>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev >= 64 || !attr_set[dev]) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+    if (err != cudaSuccess) return err;
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const int smem_r = SR::smem_bytes(kGateUp, ar.K / kGroup, ar.E, false);
+  const int smem_s = SS::smem_bytes(kGateUp, as.K / kGroup, as.E, true);
+  kernel<<<num_ctas, kThreads, smem_r > smem_s ? smem_r : smem_s, s>>>(rw, ra, rsc, rgs, sw, sa, ar,
+                                                                       as);
   return cudaGetLastError();
 }
 
@@ -1363,6 +1442,46 @@ cudaError_t launch_grouped_gemm(bool gate_up, bool decode, const CUtensorMap& tm
   if (p == 4) return launch_either<PrefillTileCorr>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
   return launch_either<Prefill16Epi>(gate_up, tw, ta, tsc, tgs, a, num_ctas, s);
 }
+
+cudaError_t launch_grouped_gemm_with_shared(bool gate_up, bool decode, const CUtensorMap& tmap_w,
+                                            const CUtensorMap& tmap_act,
+                                            const CUtensorMap& tmap_sc,
+                                            const CUtensorMap& tmap_gs,
+                                            const CUtensorMap& shared_w,
+                                            const CUtensorMap& shared_act, const GemmArgs& a,
+                                            const GemmArgs& shared, int num_ctas,
+                                            cudaStream_t s) {
+  if (a.K % kGroup || a.K / kGroup > kMaxGroups || a.K <= 0 || shared.K % kGroup ||
+      shared.K / kGroup > kMaxGroups || shared.K <= 0 || shared.E != 1 ||
+      shared.n_rows % kBM || (gate_up && shared.half_rows % kBM))
+    return cudaErrorInvalidValue;
+  // the default shapes only (a forced shape runs the two projections apart)
+  if (decode_shape_forced() != 0 || shape_choice("W4A8_GEMM_PREFILL_SHAPE") != 0)
+    return cudaErrorNotSupported;
+  const CUtensorMap &tw = tmap_w, &ta = tmap_act, &tsc = tmap_sc, &tgs = tmap_gs;
+  if (decode) {
+    const bool even = (a.K / kGroup) % 2 == 0;
+    if (gate_up)
+      return even ? launch_two_phase<DecodePair, F8Decode, true>(tw, ta, tsc, tgs, shared_w,
+                                                                 shared_act, a, shared, num_ctas, s)
+                  : launch_two_phase<DecodeOneSet, F8Decode, true>(tw, ta, tsc, tgs, shared_w,
+                                                                   shared_act, a, shared, num_ctas,
+                                                                   s);
+    return even ? launch_two_phase<DecodePairTwoSets, F8Decode, false>(tw, ta, tsc, tgs, shared_w,
+                                                                       shared_act, a, shared,
+                                                                       num_ctas, s)
+                : launch_two_phase<DecodeTwoSets, F8Decode, false>(tw, ta, tsc, tgs, shared_w,
+                                                                   shared_act, a, shared, num_ctas,
+                                                                   s);
+  }
+  // prefill: the shared expert's own launches already fill the GPU, and its
+  // shape would lose registers inside the routed prefill shape's 768 threads
+  return cudaErrorNotSupported;
+}
+
+int grouped_gemm_shared_tile_n() { return kTileNShared; }
+
+bool grouped_gemm_shared_fusable() { return decode_shape_forced() == 0; }
 
 namespace {
 

@@ -12,6 +12,7 @@ constexpr int kGroup = 128;        // INT4 group size along K
 constexpr int kRouteTok = 256;     // tokens per routing block
 constexpr int kTileNDecode = 32;   // tokens per grouped-GEMM tile, decode shape
 constexpr int kTileNPrefill = 128; // tokens per grouped-GEMM tile, prefill shape
+constexpr int kTileNShared = 64;   // tokens per tile of the shared expert in a routed decode launch
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxGroups = 64;     // K / 128 per GEMM (K <= 8192)
@@ -180,6 +181,22 @@ bool grouped_gemm_uses_sum_parts(bool decode);
 cudaError_t launch_grouped_gemm_i8(bool gate_up, bool decode, const CUtensorMap& tmap_w,
                                    const CUtensorMap& tmap_act, const GemmArgs& a, int num_ctas,
                                    cudaStream_t s);
+// The routed projection (as launch_grouped_gemm with the default decode
+// shapes, no split tiling) and the shared expert's (as launch_fp8_block_gemm,
+// tiles of grouped_gemm_shared_tile_n() token rows) in one launch.
+// cudaErrorNotSupported for the prefill shapes and when a shape is forced by
+// the environment: the caller then launches the two apart.
+cudaError_t launch_grouped_gemm_with_shared(bool gate_up, bool decode, const CUtensorMap& tmap_w,
+                                            const CUtensorMap& tmap_act,
+                                            const CUtensorMap& tmap_sc,
+                                            const CUtensorMap& tmap_gs,
+                                            const CUtensorMap& shared_w,
+                                            const CUtensorMap& shared_act, const GemmArgs& a,
+                                            const GemmArgs& shared, int num_ctas,
+                                            cudaStream_t s);
+int grouped_gemm_shared_tile_n();
+// Whether the decode shapes in use are the defaults the two-phase launch takes.
+bool grouped_gemm_shared_fusable();
 // Dense GEMM with E4M3 weights and 128 x 128 block scales (one expert, E = 1):
 // tmap_w = codes [n_rows, K] bytes, box [64 (gate/up) or 128 rows x 128 B],
 // 128-byte swizzle; wscale = float32 [n_rows / 128, K / 128]; act_gsum = the
