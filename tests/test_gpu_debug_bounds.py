@@ -3,9 +3,10 @@
 Its kernels check every routing-derived index before use (the expert
 offsets and tile tables the grouped GEMM decodes, segment rows, token ids);
 one out of range raises W4A8_ERR_DEVICE_INDEX at the next
-w4a8_check_device_error and the access is skipped.  The forward and
-expert-parallel parity cases run on it in a child process: they must pass
-with no check firing (each test ends with w4a8_check_device_error), and an
+w4a8_check_device_error and the access is skipped.  The forward,
+expert-parallel and shared-expert parity cases run on it in a child process:
+they must pass with no check firing (each test ends with
+w4a8_check_device_error), and an
 expert id outside [-1, E) given to w4a8_moe_forward_experts must be reported,
 as must bad indices given to the all-to-all row gather and combine.
 """
@@ -33,10 +34,11 @@ def test_parity_cases_on_the_bounds_checking_build():
     assert r.returncode == 0, r.stdout + r.stderr
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p",
                         "no:cacheprovider", os.path.join(HERE, "test_gpu_forward.py"),
-                        os.path.join(HERE, "test_gpu_ep.py"), "-k",
+                        os.path.join(HERE, "test_gpu_ep.py"),
+                        os.path.join(HERE, "test_gpu_shared.py"), "-k",
                         "tiny_workload or ragged or multi_block or zipf_empty or zero_token_row "
                         "or padding or route_topk or dispatch_plan or gather_and_combine "
-                        "or bad_send_rows"],
+                        "or bad_send_rows or shared_gemms_inside"],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
     tail = "\n".join((r.stdout + r.stderr).splitlines()[-15:])
     assert r.returncode == 0, tail
