@@ -106,3 +106,28 @@ def test_segment_histogram_bins_every_expert_once():
     assert h["bins"] == {"0": 2, "1-8": 2, "9-32": 2, "33-128": 2, "129-512": 2,
                          "513-2048": 2, ">=2049": 2}
     assert h["active"] == 12 and h["max"] == 60000
+
+
+def test_shared_fused_rule_and_launch_counts(monkeypatch):
+    """The bench's account of where the shared expert's GEMMs run follows the
+    library's rule: decode-sized batches (T k <= 32 E) without split tiling, the
+    default decode shapes, W4A8_SHARED_FUSED not 0; then a step launches the
+    routed kernels plus the tables and two quantisers, else also the two GEMMs."""
+    import w4a8_quantized_moe_b200 as w4
+    monkeypatch.delenv("W4A8_SHARED_FUSED", raising=False)
+    monkeypatch.delenv("W4A8_GEMM_DECODE_SHAPE", raising=False)
+    decode = workloads.CONFIGS[1]                         # T=64, E=256, k=8
+    prefill = workloads.CONFIGS[3]
+    assert bench.shared_fused(w4, decode, "w4a8+shared")
+    assert not bench.shared_fused(w4, decode, "w4a8")
+    assert not bench.shared_fused(w4, prefill, "w4a8+shared")
+    assert bench.step_launches(w4, decode, "w4a8") == bench.KERNELS_PER_STEP
+    assert bench.step_launches(w4, decode, "w4a8+shared") == \
+        bench.KERNELS_PER_STEP + bench.SHARED_KERNELS_PER_STEP - 2
+    assert bench.step_launches(w4, prefill, "w4a8+shared") == \
+        w4.w4a8_moe_forward_launches(prefill.T, prefill.E, prefill.k) + bench.SHARED_KERNELS_PER_STEP
+    monkeypatch.setenv("W4A8_SHARED_FUSED", "0")
+    assert not bench.shared_fused(w4, decode, "w4a8+shared")
+    monkeypatch.setenv("W4A8_SHARED_FUSED", "1")
+    monkeypatch.setenv("W4A8_GEMM_DECODE_SHAPE", "3")
+    assert not bench.shared_fused(w4, decode, "w4a8+shared")
